@@ -1,0 +1,300 @@
+"""Plain, slow, fp64 reference of the routed-expert MoE layer (test infrastructure).
+
+Imported only by ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s
+CPU-baseline / reference leg.  Nothing in the CUDA library calls it, and it
+calls nothing of the library.
+
+Sources (the Flash-MoE pages):
+
+* hotdry.top article "48GB内存运行397B模型", section "MoE稀疏架构": a layer has
+  512 routed experts of which K are active per token, plus one shared expert.
+* same article, section "量化策略", and the juejin.cn article section
+  "Metal 着色器": expert weights are 4-bit (or 2-bit) codes dequantised as
+  ``code * scale + bias`` before they meet the activation; the FMA rewrite
+  ``fma(code, scale*x, bias*x)`` is the same sum reordered.
+* same article, section "Metal GPU管线", and the juejin.cn list of shaders:
+  fused SwiGLU ``silu(gate) * up``; fused combine of the expert outputs with the
+  residual and a sigmoid-gated shared expert; two-pass RMS normalisation.
+* tinai-dev README page, "Pipeline mỗi lớp": routing on the GPU, then
+  softmax and top-K on the CPU.
+* intelliparadigm.com page, section 2.1 (router snippet): softmax over all
+  experts, then top-K on the probabilities.
+
+Readings where the pages are silent (each listed in the design notes):
+
+* group size 64 along the input (reduction) dimension, one (scale, bias) pair
+  per group and row; codes low-bits-first inside little-endian uint32 words;
+* top-K ordered by probability descending, ties to the lower expert index;
+  the K probabilities are renormalised to sum to one;
+* shared expert gate ``sigma = 1 / (1 + exp(-g_s . x))`` with a vector g_s;
+* single-layer output ``y = resid + sum_k w_k o_k + sigma o_s``;
+* stacked layers are pre-norm blocks ``h <- h + MoE(RMSNorm(h))`` with gamma = 1,
+  eps = 1e-6, the normalised vector rounded to bf16.
+
+Everything is float64.  Dequantised weights ``scale * q + bias`` are exact in
+float64 (a bf16 times a <= 4-bit integer needs <= 12 significand bits).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+import fmoe_synth as synth
+
+GROUP = 64
+
+
+# ----------------------------------------------------------------------------
+# storage decoding
+# ----------------------------------------------------------------------------
+def bf16_to_f64(bits) -> np.ndarray:
+    """bf16 bit patterns -> float64 (exact)."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def f64_to_bf16_bits(v) -> np.ndarray:
+    """Round float64 values to bf16 (nearest, ties to even); returns bit patterns.
+
+    Written from the definition: keep 8 significant bits of the binary
+    significand, rounding the discarded part to nearest with ties to even.
+    Normal-range values only (the layer's values never leave it)."""
+    v = np.atleast_1d(np.asarray(v, dtype=np.float64))
+    out = np.zeros(v.shape, dtype=np.uint16)
+    for idx, x in np.ndenumerate(v):
+        if x == 0.0:
+            out[idx] = 0x8000 if math.copysign(1.0, x) < 0 else 0
+            continue
+        m, e = math.frexp(abs(x))          # |x| = m 2^e, m in [0.5, 1)
+        scaled = m * 256.0                 # exact
+        lo = math.floor(scaled)
+        frac = scaled - lo
+        if frac > 0.5 or (frac == 0.5 and lo % 2 == 1):
+            lo += 1
+        r = math.ldexp(lo, e - 8)
+        if x < 0:
+            r = -r
+        out[idx] = np.float32(r).view(np.uint32) >> 16
+    return out
+
+
+def unpack_codes(words: np.ndarray, bits: int) -> np.ndarray:
+    """uint32 words [..., W] -> integer codes [..., W * 32/bits], code k of a word
+    taken from bits [bits*k, bits*k + bits) (lowest bits first)."""
+    words = np.asarray(words, dtype=np.uint32)
+    per = 32 // bits
+    mask = (1 << bits) - 1
+    codes = np.empty(words.shape + (per,), dtype=np.int64)
+    for k in range(per):
+        codes[..., k] = (words.astype(np.int64) >> (bits * k)) & mask
+    return codes.reshape(words.shape[:-1] + (words.shape[-1] * per,))
+
+
+def dequantise(codes: np.ndarray, sb: np.ndarray) -> np.ndarray:
+    """Explicit dequantisation W[r, c] = scale[r, c//64] * q[r, c] + bias[r, c//64].
+
+    ``sb`` holds one uint32 per (row, group): bf16 scale in the low half,
+    bf16 bias in the high half."""
+    sb = np.asarray(sb, dtype=np.uint32)
+    scale = bf16_to_f64((sb & 0xFFFF).astype(np.uint16))
+    bias = bf16_to_f64((sb >> 16).astype(np.uint16))
+    rows, cols = codes.shape
+    g = np.arange(cols) // GROUP
+    return scale[:, g] * codes.astype(np.float64) + bias[:, g]
+
+
+@dataclass
+class DenseExpert:
+    Wg: np.ndarray  # [I, H]
+    Wu: np.ndarray  # [I, H]
+    Wd: np.ndarray  # [H, I]
+
+
+def record_regions(H: int, I: int, bits: int) -> dict:
+    """Byte layout of one packed expert record (the library's weight format):
+    four regions, each starting at a multiple of 256 bytes:
+    gate/up code rows interleaved by row, gate/up (scale, bias) rows interleaved
+    by row, down code rows, down (scale, bias) rows."""
+    def al(n):
+        return (n + 255) // 256 * 256
+    qh, qi = H * bits // 8, I * bits // 8
+    sh, si = H // GROUP * 4, I // GROUP * 4
+    o0 = 0
+    o1 = al(o0 + I * 2 * qh)
+    o2 = al(o1 + I * 2 * sh)
+    o3 = al(o2 + H * qi)
+    size = al(o3 + H * si)
+    return dict(gu_q=o0, gu_sb=o1, d_q=o2, d_sb=o3, size=size, qh=qh, qi=qi, sh=sh, si=si)
+
+
+def decode_record(rec: np.ndarray, H: int, I: int, bits: int) -> DenseExpert:
+    """Read one packed record and dequantise its three matrices to float64."""
+    R = record_regions(H, I, bits)
+    rec = np.asarray(rec, dtype=np.uint8)
+    wh, wi = H * bits // 32, I * bits // 32
+    gu_q = rec[R["gu_q"]:R["gu_q"] + I * 2 * R["qh"]].view(np.uint32).reshape(I, 2, wh)
+    gu_sb = rec[R["gu_sb"]:R["gu_sb"] + I * 2 * R["sh"]].view(np.uint32).reshape(I, 2, H // GROUP)
+    d_q = rec[R["d_q"]:R["d_q"] + H * R["qi"]].view(np.uint32).reshape(H, wi)
+    d_sb = rec[R["d_sb"]:R["d_sb"] + H * R["si"]].view(np.uint32).reshape(H, I // GROUP)
+    Wg = dequantise(unpack_codes(gu_q[:, 0, :], bits), gu_sb[:, 0, :])
+    Wu = dequantise(unpack_codes(gu_q[:, 1, :], bits), gu_sb[:, 1, :])
+    Wd = dequantise(unpack_codes(d_q, bits), d_sb)
+    return DenseExpert(Wg, Wu, Wd)
+
+
+# ----------------------------------------------------------------------------
+# the layer, step by step
+# ----------------------------------------------------------------------------
+def router_logits(x: np.ndarray, Wr: np.ndarray, bias: Optional[np.ndarray] = None) -> np.ndarray:
+    """l_e = sum_c Wr[e, c] x_c (+ b_e), float64 (router GEMV)."""
+    l = Wr.astype(np.float64) @ np.asarray(x, dtype=np.float64)
+    if bias is not None:
+        l = l + np.asarray(bias, dtype=np.float64)
+    return l
+
+
+def softmax(l: np.ndarray) -> np.ndarray:
+    m = np.max(l)
+    e = np.exp(l - m)
+    return e / np.sum(e)
+
+
+def topk_renorm(l: np.ndarray, K: int):
+    """Softmax over all experts, top-K by probability (descending, ties to the
+    lower index), then the K probabilities renormalised to sum to one."""
+    p = softmax(l)
+    order = sorted(range(len(p)), key=lambda e: (-p[e], e))
+    idx = np.array(order[:K], dtype=np.int64)
+    w = p[idx] / np.sum(p[idx])
+    return idx, w
+
+
+def silu(t: np.ndarray) -> np.ndarray:
+    return t / (1.0 + np.exp(-t))
+
+
+def expert_ffn(ex: DenseExpert, x: np.ndarray) -> np.ndarray:
+    """o = W_d (silu(W_g x) * (W_u x)) in float64."""
+    x = np.asarray(x, dtype=np.float64)
+    g = ex.Wg @ x
+    u = ex.Wu @ x
+    h = silu(g) * u
+    return ex.Wd @ h
+
+
+def expert_hidden(ex: DenseExpert, x: np.ndarray) -> np.ndarray:
+    x = np.asarray(x, dtype=np.float64)
+    return silu(ex.Wg @ x) * (ex.Wu @ x)
+
+
+def shared_sigma(gs: np.ndarray, x: np.ndarray) -> float:
+    s = float(np.asarray(gs, dtype=np.float64) @ np.asarray(x, dtype=np.float64))
+    return 1.0 / (1.0 + math.exp(-s))
+
+
+@dataclass
+class LayerResult:
+    y: np.ndarray        # float64 [H], unrounded
+    idx: np.ndarray      # int64 [K]
+    w: np.ndarray        # float64 [K]
+    sigma: float
+    logits: np.ndarray   # float64 [E]
+
+
+class OracleLayer:
+    """One MoE layer held as packed records (numpy uint8) plus router tensors.
+
+    ``records`` may be a callable ``e -> record bytes`` so that full-size layers
+    regenerate only the experts a token selects."""
+
+    def __init__(self, H, I, E, K, bits, records, router, shared_gate=None,
+                 router_bias=None, has_shared=True):
+        self.H, self.I, self.E, self.K, self.bits = H, I, E, K, bits
+        self._records = records
+        self.router = np.asarray(router, dtype=np.float32)
+        self.shared_gate = None if shared_gate is None else np.asarray(shared_gate, dtype=np.float32)
+        self.router_bias = None if router_bias is None else np.asarray(router_bias, dtype=np.float32)
+        self.has_shared = has_shared
+        self._cache = {}
+
+    def expert(self, e: int) -> DenseExpert:
+        if e not in self._cache:
+            if callable(self._records):
+                rec = self._records(e)
+            else:
+                rb = record_regions(self.H, self.I, self.bits)["size"]
+                rec = self._records[e * rb:(e + 1) * rb]
+            self._cache[e] = decode_record(rec, self.H, self.I, self.bits)
+        return self._cache[e]
+
+    def route(self, x: np.ndarray):
+        l = router_logits(x, self.router, self.router_bias)
+        idx, w = topk_renorm(l, self.K)
+        sig = shared_sigma(self.shared_gate, x) if self.has_shared else 0.0
+        return idx, w, sig, l
+
+    def forward(self, x: np.ndarray, resid: Optional[np.ndarray] = None) -> LayerResult:
+        """y = resid + sum_k w_k o_k(x) + sigma o_s(x); resid defaults to x."""
+        x = np.asarray(x, dtype=np.float64)
+        r = x if resid is None else np.asarray(resid, dtype=np.float64)
+        idx, w, sig, l = self.route(x)
+        y = r.copy()
+        for k in range(self.K):
+            y = y + w[k] * expert_ffn(self.expert(int(idx[k])), x)
+        if self.has_shared:
+            y = y + sig * expert_ffn(self.expert(self.E), x)
+        return LayerResult(y=y, idx=idx, w=w, sigma=sig, logits=l)
+
+    def expert_forward(self, x, resid, idx, w, sig) -> np.ndarray:
+        """Combine for given routing (the split entry point)."""
+        x = np.asarray(x, dtype=np.float64)
+        y = np.asarray(resid, dtype=np.float64).copy()
+        for k in range(len(idx)):
+            y = y + float(w[k]) * expert_ffn(self.expert(int(idx[k])), x)
+        if self.has_shared:
+            y = y + float(sig) * expert_ffn(self.expert(self.E), x)
+        return y
+
+
+def rmsnorm_bf16(h: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """n = bf16(h / sqrt(mean(h^2) + eps)), gamma = 1; returns bf16 bit patterns.
+
+    Two passes as on the pages: the sum of squares, then the scaling."""
+    h = np.asarray(h, dtype=np.float64)
+    ss = 0.0
+    for v in h:
+        ss += v * v
+    r = math.sqrt(ss / h.size + eps)
+    return f64_to_bf16_bits(h / r)
+
+
+# ----------------------------------------------------------------------------
+# synthetic layers built from the shared generator
+# ----------------------------------------------------------------------------
+def synthetic_layer(seed: int, layer: int, shape: "synth.LayerShape", lazy: bool = False) -> OracleLayer:
+    H, I, E = shape.hidden, shape.inter, shape.n_experts
+    if lazy:
+        def rec(e, _s=seed, _l=layer):
+            return synth.gen_record(_s, _l, e, H, I, shape.bits)
+        records = rec
+    else:
+        records = synth.gen_layer_records(seed, layer, shape)
+    router = synth.gen_router(seed, layer, E, H)
+    gs = synth.gen_shared_gate(seed, layer, H) if shape.has_shared else None
+    rb = synth.gen_router_bias(seed, layer, E) if shape.router_bias else None
+    return OracleLayer(H, I, E, shape.top_k, shape.bits, records, router, gs, rb,
+                       has_shared=bool(shape.has_shared))
+
+
+def within_tolerance(gpu: np.ndarray, ref: np.ndarray, rel: float = 2e-3):
+    """Per-element bound |gpu - ref| <= rel * (|ref| + rms(ref)); returns
+    (ok, worst ratio of error to bound)."""
+    ref = np.asarray(ref, dtype=np.float64)
+    gpu = np.asarray(gpu, dtype=np.float64)
+    rms = math.sqrt(float(np.mean(ref * ref)))
+    bound = rel * (np.abs(ref) + rms)
+    ratio = np.abs(gpu - ref) / np.maximum(bound, 1e-300)
+    return bool(np.all(ratio <= 1.0)), float(np.max(ratio)) if ratio.size else 0.0
