@@ -1,0 +1,322 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-expert MoE decode layer on B200.
+
+Metric: MoE-layer decode tokens/s, with the effective expert-weight HBM GB/s
+(and its fraction of HBM peak) for the full-size 4-bit top-4 layer: hidden 4096,
+expert intermediate 1024, 512 routed experts + 1 shared, 1000 tokens with
+independent seeded activations.  One step = the 1000 tokens, each a single-token
+fmoe_layer_forward call (one fused kernel launch), the 1000 launches replayed
+from one CUDA graph.  Weights (3.64 GB) are resident in HBM; the L2 is flushed
+between steps.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs an independent
+replica on its own GPU (the layer has no exchange step): value = tokens of all
+ranks / max over ranks of the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HBM_NOMINAL_GBS = 8000.0
+METRIC = "MoE-layer decode tokens/s; expert-weight HBM GB/s (% of ~8 TB/s), 4-bit K=4"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fmoe", choices=["fmoe", "reference"])
+    ap.add_argument("--config", default="layer4096")
+    ap.add_argument("--tokens", type=int, default=None)
+    ap.add_argument("--cpu-sample", type=int, default=4, help="tokens timed for the CPU oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def layer_bytes(shape):
+    """Algorithmic bytes of one single-token layer forward."""
+    import fmoe_synth as synth
+    rb = synth.record_bytes(shape.hidden, shape.inter, shape.bits)
+    experts = (shape.top_k + shape.has_shared) * rb
+    router = shape.n_experts * shape.hidden * 4 + (shape.hidden * 4 if shape.has_shared else 0)
+    io = 3 * shape.hidden * 2
+    return experts, router + io
+
+
+def cpu_oracle_rate(shape, n_tokens: int, seed: int = 0):
+    """The fp64 oracle (as it stands) on n_tokens tokens of the workload: returns
+    (tokens/s, threads used, description).  Expert records are regenerated before
+    each token's timed forward, which is then run from the packed bytes."""
+    import numpy as np
+
+    import fmoe_synth as synth
+    import oracle
+    olay = oracle.synthetic_layer(seed, 0, shape, lazy=True)
+    total = 0.0
+    for t in range(n_tokens):
+        x = oracle.bf16_to_f64(synth.gen_x_token(seed, t, shape.hidden))
+        idx, _, _, _ = olay.route(x)
+        recs = {int(e): synth.gen_record(seed, 0, int(e), shape.hidden, shape.inter, shape.bits)
+                for e in list(idx) + [shape.n_experts]}
+        olay._cache = {}
+        olay._records = lambda e, _r=recs: _r[e]
+        t0 = time.perf_counter()
+        olay.forward(x)
+        total += time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        threads = 1
+    return n_tokens / total, threads, f"{n_tokens} tokens of the {shape.hidden}x{shape.inter} layer"
+
+
+def run_reference(args, rank):
+    """The reference arm: the fp64 CPU oracle, timed on the host cores."""
+    import fmoe_synth as synth
+    if rank != 0:
+        return
+    shape = synth.CONFIGS[args.config]["shape"]
+    per_step = max(1, args.cpu_sample)
+    for _ in range(args.warmup and 1):
+        cpu_oracle_rate(shape, 1)
+    t_all = 0.0
+    tok = 0
+    threads, desc = 1, ""
+    for _ in range(args.steps):
+        rate, threads, desc = cpu_oracle_rate(shape, per_step)
+        t_all += per_step / rate
+        tok += per_step
+    value = tok / t_all
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * t_all / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{args.config}: single-token decode, hidden {shape.hidden}, "
+                                   f"inter {shape.inter}, {shape.n_experts}+{shape.has_shared} experts, "
+                                   f"top-{shape.top_k}, {shape.bits}-bit",
+                       "tokens_per_step": per_step},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{per_step} tokens per step ({desc})"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import fmoe_synth as synth
+    from bit_dequant_expert_softmax_b200 import fmoe
+    from fmoe_synth.torch_layer import make_device_layer, make_device_x
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    shape = synth.CONFIGS[args.config]["shape"]
+    tokens = args.tokens or synth.CONFIGS[args.config]["tokens"]
+    H = shape.hidden
+
+    w = make_device_layer(shape, 0, 0)
+    cfg = fmoe.fmoe_config(H, shape.inter, shape.n_experts, shape.top_k, shape.bits, shape.has_shared,
+                           shape.router_bias)
+    L = fmoe.Layer.create(cfg, w.experts, w.router, w.router_bias, w.shared_gate)
+    x = make_device_x(0, rank * tokens, tokens, H)
+    y = torch.empty_like(x)
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+
+    def run_tokens(s):
+        for t in range(tokens):
+            fmoe.fmoe_layer_forward(L.handle, x[t:t + 1], x[t:t + 1], 1, y[t:t + 1], stream=s)
+
+    with torch.cuda.stream(stream):
+        run_tokens(stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        run_tokens(stream)
+    torch.cuda.synchronize()
+
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)  # L2 flush between steps (outside the timed events)
+            starts[i].record(stream)
+            graph.replay()
+            ends[i].record(stream)
+    barrier()
+    clocks = sampler.stop()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    err = L.error()
+    if err:
+        raise RuntimeError(f"device-side error bits {err:#x} during the benchmark")
+
+    # end to end through the C ABI from pinned host buffers
+    xh = x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    e_s = torch.cuda.Event(enable_timing=True)
+    e_e = torch.cuda.Event(enable_timing=True)
+    barrier()
+    with torch.cuda.stream(stream):
+        e_s.record(stream)
+        for i in range(args.steps):
+            x.copy_(xh, non_blocking=True)
+            graph.replay()
+            yh.copy_(y, non_blocking=True)
+        e_e.record(stream)
+    barrier()
+    e2e_ms = e_s.elapsed_time(e_e)
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+
+    total_tokens = tokens * args.steps * world
+    value = total_tokens / (total_ms / 1e3)
+    e2e_value = total_tokens / (e2e_ms / 1e3)
+    expert_b, other_b = layer_bytes(shape)
+    launch_s = (total_ms / 1e3) / (tokens * args.steps)
+    peak, peak_kind = measured_peaks()
+    achieved = (expert_b + other_b) / launch_s / 1e9
+    expert_gbs = expert_b / launch_s / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_kind": peak_kind, "kernel": "fmoe_layer_kernel<4>",
+            "bytes_per_launch": expert_b + other_b, "expert_bytes_per_launch": expert_b,
+            "expert_gbs": round(expert_gbs, 1), "expert_frac_of_8tbs": round(expert_gbs / HBM_NOMINAL_GBS, 4),
+            "expert_frac_of_measured": round(expert_gbs / peak, 4), "avg_launch_us": round(launch_s * 1e6, 3)}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, threads, desc = cpu_oracle_rate(shape, args.cpu_sample)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{args.cpu_sample} tokens ({desc}), fp64 numpy oracle"}
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "u4-dequant/f32-accum",
+                "data": "synthetic",
+                "config": {"workload": f"{args.config}: single-token decode, hidden {H}, inter {shape.inter}, "
+                                       f"{shape.n_experts}+{shape.has_shared} experts, top-{shape.top_k}, "
+                                       f"{shape.bits}-bit group-64",
+                           "tokens_per_step": tokens, "l2": "flushed between steps (512 MiB write)",
+                           "parallelism": f"replicas x{world}"},
+                "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": xh.numel() * 2,
+                        "d2h_bytes_per_step": yh.numel() * 2},
+                "gpu_launches": tokens * args.steps,
+                "roofline": roof, "cpu_baseline": cpu, "clocks": clocks,
+                "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)}}
+        print(json.dumps(line), flush=True)
+    del graph
+    L.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

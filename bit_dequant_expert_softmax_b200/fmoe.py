@@ -1,0 +1,208 @@
+"""Thin ctypes binding of libfmoe.so (see include/fmoe.h for the contract).
+
+Functions keep the C names; arguments are marshalled from torch CUDA tensors
+(device memory and streams only: every step of the layer runs in the library's
+kernels).  Loading fails loudly when the library is missing."""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SO = os.path.join(HERE, "libfmoe.so")
+
+FMOE_OK = 0
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "CUDA error",
+          4: "workspace missing or too small", 5: "device-side error"}
+DEVERR_BARRIER_TIMEOUT = 0x1
+DEVERR_COPY_TIMEOUT = 0x2
+DEVERR_BAD_EXPERT = 0x4
+
+# every symbol include/fmoe.h declares
+EXPORTS = ["fmoe_record_bytes", "fmoe_workspace_bytes", "fmoe_layer_create", "fmoe_layer_destroy",
+           "fmoe_layer_set_workspace", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward",
+           "fmoe_rmsnorm", "fmoe_layer_get_error", "fmoe_layer_set_wait_limit",
+           "fmoe_layer_debug_hold_block", "fmoe_layer_grid_size", "fmoe_status_string"]
+
+
+class FmoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class fmoe_config(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("inter", ctypes.c_int), ("n_experts", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("bits", ctypes.c_int), ("has_shared", ctypes.c_int),
+                ("has_router_bias", ctypes.c_int)]
+
+
+class fmoe_weights(ctypes.Structure):
+    _fields_ = [("experts", ctypes.c_void_p), ("router", ctypes.c_void_p),
+                ("router_bias", ctypes.c_void_p), ("shared_gate", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(SO):
+            raise RuntimeError(f"{SO} is missing: build it with bit_dequant_expert_softmax_b200.build.build()")
+        L = ctypes.CDLL(SO)
+        vp, i32, u64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
+        L.fmoe_record_bytes.restype = sz
+        L.fmoe_record_bytes.argtypes = [i32, i32, i32]
+        L.fmoe_workspace_bytes.restype = sz
+        L.fmoe_workspace_bytes.argtypes = [ctypes.POINTER(fmoe_config)]
+        L.fmoe_layer_create.argtypes = [ctypes.POINTER(fmoe_config), ctypes.POINTER(fmoe_weights),
+                                        ctypes.POINTER(vp)]
+        L.fmoe_layer_destroy.argtypes = [vp]
+        L.fmoe_layer_set_workspace.argtypes = [vp, vp, sz]
+        L.fmoe_route.argtypes = [vp, vp, i32, vp, vp, vp, vp]
+        L.fmoe_expert_forward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp]
+        L.fmoe_layer_forward.argtypes = [vp, vp, vp, i32, vp, vp]
+        L.fmoe_rmsnorm.argtypes = [vp, vp, i32, i32, ctypes.c_double, vp]
+        L.fmoe_layer_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.fmoe_layer_set_wait_limit.argtypes = [vp, u64]
+        L.fmoe_layer_debug_hold_block.argtypes = [vp, i32]
+        L.fmoe_layer_grid_size.argtypes = [vp]
+        L.fmoe_layer_grid_size.restype = i32
+        L.fmoe_status_string.argtypes = [i32]
+        L.fmoe_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(st: int, what: str):
+    if st != FMOE_OK:
+        raise FmoeError(st, what)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def fmoe_record_bytes(hidden: int, inter: int, bits: int) -> int:
+    return lib().fmoe_record_bytes(hidden, inter, bits)
+
+
+def fmoe_workspace_bytes(cfg: fmoe_config) -> int:
+    return lib().fmoe_workspace_bytes(ctypes.byref(cfg))
+
+
+def fmoe_layer_create(cfg: fmoe_config, experts, router, router_bias=None, shared_gate=None) -> int:
+    w = fmoe_weights(_ptr(experts), _ptr(router), _ptr(router_bias), _ptr(shared_gate))
+    h = ctypes.c_void_p()
+    _check(lib().fmoe_layer_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)), "fmoe_layer_create")
+    return h.value
+
+
+def fmoe_layer_destroy(handle: int):
+    _check(lib().fmoe_layer_destroy(handle), "fmoe_layer_destroy")
+
+
+def fmoe_layer_set_workspace(handle: int, ws):
+    _check(lib().fmoe_layer_set_workspace(handle, ws.data_ptr(), ws.numel() * ws.element_size()),
+           "fmoe_layer_set_workspace")
+
+
+def fmoe_route(handle, x, T, idx, w, shared_sigma=None, stream=None):
+    _check(lib().fmoe_route(handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(shared_sigma), _stream(stream)),
+           "fmoe_route")
+
+
+def fmoe_expert_forward(handle, x, resid, T, idx, w, shared_sigma, y, stream=None):
+    _check(lib().fmoe_expert_forward(handle, _ptr(x), _ptr(resid), T, _ptr(idx), _ptr(w), _ptr(shared_sigma),
+                                     _ptr(y), _stream(stream)), "fmoe_expert_forward")
+
+
+def fmoe_layer_forward(handle, x, resid, T, y, stream=None):
+    _check(lib().fmoe_layer_forward(handle, _ptr(x), _ptr(resid), T, _ptr(y), _stream(stream)),
+           "fmoe_layer_forward")
+
+
+def fmoe_rmsnorm(h, out, T, H, eps=1e-6, stream=None):
+    _check(lib().fmoe_rmsnorm(_ptr(h), _ptr(out), T, H, eps, _stream(stream)), "fmoe_rmsnorm")
+
+
+def fmoe_layer_get_error(handle) -> int:
+    e = ctypes.c_uint32(0)
+    st = lib().fmoe_layer_get_error(handle, ctypes.byref(e))
+    if st not in (0, 5):
+        raise FmoeError(st, "fmoe_layer_get_error")
+    return e.value
+
+
+def fmoe_layer_set_wait_limit(handle, ns: int):
+    _check(lib().fmoe_layer_set_wait_limit(handle, ns), "fmoe_layer_set_wait_limit")
+
+
+def fmoe_layer_debug_hold_block(handle, cta: int):
+    _check(lib().fmoe_layer_debug_hold_block(handle, cta), "fmoe_layer_debug_hold_block")
+
+
+def fmoe_layer_grid_size(handle) -> int:
+    return lib().fmoe_layer_grid_size(handle)
+
+
+# ---------------------------------------------------------------------------
+@dataclass
+class Layer:
+    """A layer handle plus the torch tensors it borrows (weights, workspace)."""
+    handle: int
+    cfg: fmoe_config
+    experts: object
+    router: object
+    router_bias: object
+    shared_gate: object
+    workspace: object
+
+    @staticmethod
+    def create(cfg: fmoe_config, experts, router, router_bias=None, shared_gate=None) -> "Layer":
+        import torch
+        h = fmoe_layer_create(cfg, experts, router, router_bias, shared_gate)
+        ws = torch.empty(fmoe_workspace_bytes(cfg), dtype=torch.uint8, device=experts.device)
+        fmoe_layer_set_workspace(h, ws)
+        return Layer(h, cfg, experts, router, router_bias, shared_gate, ws)
+
+    def forward(self, x, resid=None, y=None, stream=None):
+        import torch
+        T = x.shape[0]
+        resid = x if resid is None else resid
+        y = torch.empty_like(x) if y is None else y
+        fmoe_layer_forward(self.handle, x, resid, T, y, stream)
+        return y
+
+    def route(self, x, stream=None):
+        import torch
+        T = x.shape[0]
+        K = self.cfg.top_k
+        idx = torch.empty(T, K, dtype=torch.int32, device=x.device)
+        w = torch.empty(T, K, dtype=torch.float32, device=x.device)
+        sig = torch.empty(T, dtype=torch.float32, device=x.device)
+        fmoe_route(self.handle, x, T, idx, w, sig, stream)
+        return idx, w, sig
+
+    def expert_forward(self, x, resid, idx, w, sig, y=None, stream=None):
+        import torch
+        y = torch.empty_like(x) if y is None else y
+        fmoe_expert_forward(self.handle, x, resid, x.shape[0], idx, w, sig, y, stream)
+        return y
+
+    def error(self) -> int:
+        return fmoe_layer_get_error(self.handle)
+
+    def close(self):
+        if self.handle:
+            fmoe_layer_destroy(self.handle)
+            self.handle = 0

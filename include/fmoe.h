@@ -1,0 +1,176 @@
+/*
+ * fmoe.h — C ABI of the B200 (sm_100a) routed-expert MoE layer library (libfmoe.so).
+ *
+ * The library computes, per token, the routed-expert forward of one sparse
+ * Mixture-of-Experts layer as the Flash-MoE pages describe it:
+ *
+ *   logits = W_r x (+ b)                      router matvec  (tinai-dev README,
+ *                                             "Pipeline mỗi lớp": routing on the GPU)
+ *   top-K of softmax(logits), renormalised    (same page: softmax + topK routing;
+ *                                             intelliparadigm.com §2.1 router snippet)
+ *   for each selected expert k and the shared expert s:
+ *     W = scale * code + bias  (4- or 2-bit codes, one bf16 (scale, bias) per
+ *                               64-element group)       (hotdry.top "量化策略",
+ *                                                        juejin.cn "Metal 着色器")
+ *     h = silu(W_g x) * (W_u x); o = W_d h               (hotdry.top "Metal GPU管线":
+ *                                                        fused SwiGLU)
+ *   y = resid + sum_k w_k o_k + sigmoid(g_s . x) o_s     (hotdry.top "Metal GPU管线":
+ *                                                        fused combine + residual +
+ *                                                        sigmoid-gated shared expert)
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device, owned by the
+ *     caller and borrowed (weights and workspace for the layer's lifetime, inputs and
+ *     outputs for the call).  bf16 values are passed as uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy default stream.
+ *   - Forward entry points are asynchronous: they validate on the host, enqueue kernels
+ *     on `stream` and return.  They allocate nothing, copy nothing between host and
+ *     device and do not synchronise.
+ *   - Host-detectable problems (bad config, NULL or misaligned pointer, missing
+ *     workspace) return an error status before anything is enqueued.  Problems found
+ *     on the device (an expert index out of range, a bounded wait that ran out) set a
+ *     sticky error word in the layer's workspace; while it is set, further forward
+ *     calls on that layer do no work.  fmoe_layer_get_error() reads and clears it.
+ *   - Calls on one layer must be ordered (one stream, or streams ordered by events):
+ *     they share the layer's workspace.
+ *   - No CPU fallback exists: without a usable sm_100 device, fmoe_layer_create fails.
+ */
+#ifndef FMOE_H
+#define FMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FMOE_OK = 0,
+  FMOE_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or config value        */
+  FMOE_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels are built for    */
+  FMOE_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed         */
+  FMOE_ERR_NO_WORKSPACE = 4,  /* workspace missing or smaller than required          */
+  FMOE_ERR_DEVICE = 5         /* fmoe_layer_get_error found a device-side error      */
+} fmoe_status;
+
+/* Device-side error bits reported by fmoe_layer_get_error(). */
+#define FMOE_DEVERR_BARRIER_TIMEOUT 0x1u  /* a grid-wide wait ran past its time limit  */
+#define FMOE_DEVERR_COPY_TIMEOUT    0x2u  /* a wait for a bulk copy ran past the limit */
+#define FMOE_DEVERR_BAD_EXPERT      0x4u  /* fmoe_expert_forward got idx out of range  */
+
+/* Layer geometry.  hidden (H) and inter (I) are multiples of 64; bits is 4 or 2;
+ * 1 <= top_k (K) <= n_experts (E); has_shared and has_router_bias are 0 or 1. */
+typedef struct {
+  int hidden;
+  int inter;
+  int n_experts;
+  int top_k;
+  int bits;
+  int has_shared;
+  int has_router_bias;
+} fmoe_config;
+
+/* Weights, all device pointers.
+ *
+ * experts: (n_experts + has_shared) packed expert records back to back, routed experts
+ *   0..E-1 first and the shared expert last; base 256-byte aligned; each record is
+ *   fmoe_record_bytes(H, I, bits) bytes.  One record holds four regions, each starting
+ *   at a multiple of 256 bytes from the record start:
+ *     GU_Q : for r in 0..I-1: gate code row r (H*bits/8 bytes), then up code row r
+ *     GU_SB: for r in 0..I-1: gate (scale,bias) row r (H/64 uint32), then up row r
+ *     D_Q  : for j in 0..H-1: down code row j (I*bits/8 bytes)
+ *     D_SB : for j in 0..H-1: down (scale,bias) row j (I/64 uint32)
+ *   A code row is little-endian uint32 words holding 32/bits codes each; code c of a
+ *   word occupies bits [bits*c, bits*c + bits) and is the weight of column
+ *   32/bits * word + c.  A (scale,bias) uint32 holds the bf16 scale in its low half and
+ *   the bf16 bias in its high half and covers 64 consecutive columns of its row.
+ *   Dequantised weight: W[r][c] = scale[r][c/64] * code[r][c] + bias[r][c/64].
+ *   (Format of the expert records: 8 nibbles / 16 crumbs per uint32 and bf16 scale
+ *   and bias per 64-group; 7,077,888 bytes per 4-bit expert at H=4096, I=1024 — the
+ *   "~6.75MB per expert" of hotdry.top "MoE稀疏架构".)
+ * router: fp32 [E][H] row-major, 16-byte aligned.
+ * router_bias: fp32 [E] added to the logits, or NULL when has_router_bias == 0.
+ * shared_gate: fp32 [H], 16-byte aligned, or NULL when has_shared == 0. */
+typedef struct {
+  const void* experts;
+  const float* router;
+  const float* router_bias;
+  const float* shared_gate;
+} fmoe_weights;
+
+typedef struct fmoe_layer* fmoe_layer_t;
+
+/* Bytes of one packed expert record (0 if H or I is not a positive multiple of 64 or
+ * bits is not 2 or 4). */
+size_t fmoe_record_bytes(int hidden, int inter, int bits);
+
+/* Device workspace bytes a layer with this config needs (0 for an invalid config). */
+size_t fmoe_workspace_bytes(const fmoe_config* cfg);
+
+/* Validates cfg and the weight pointers and creates a layer handle on the current
+ * device.  The handle keeps copies of cfg and the pointers (not the data).  Errors:
+ * INVALID_ARG (NULL/misaligned pointers, bad values), UNSUPPORTED (shapes whose
+ * working set does not fit the kernels' shared-memory plan), CUDA (no sm_100 device). */
+fmoe_status fmoe_layer_create(const fmoe_config* cfg, const fmoe_weights* w, fmoe_layer_t* out);
+
+/* Releases the handle (host memory only).  NULL is accepted. */
+fmoe_status fmoe_layer_destroy(fmoe_layer_t layer);
+
+/* Attaches a caller-owned device workspace of at least fmoe_workspace_bytes() bytes,
+ * 256-byte aligned, and zeroes it (synchronously).  Must precede forward calls. */
+fmoe_status fmoe_layer_set_workspace(fmoe_layer_t layer, void* dev_ptr, size_t bytes);
+
+/* Routing only.  x: bf16 [T][H] (16-byte aligned).  Writes idx int32 [T][K] (experts
+ * in descending router probability, ties to the lower index), w fp32 [T][K] (the K
+ * probabilities renormalised to sum to 1) and, if shared_sigma != NULL and the layer
+ * has a shared expert, fp32 [T] sigmoid(g_s . x).  T == 0 is a no-op. */
+fmoe_status fmoe_route(fmoe_layer_t layer, const uint16_t* x, int T, int32_t* idx, float* w,
+                       float* shared_sigma, void* stream);
+
+/* Experts and combine for given routing: y[t] = resid[t] + sum_k w[t][k] o_{idx[t][k]}(x[t])
+ * + shared_sigma[t] o_s(x[t]).  x, resid, y: bf16 [T][H], 16-byte aligned; y may alias
+ * resid but not x.  idx int32 [T][K], w fp32 [T][K], shared_sigma fp32 [T] (ignored
+ * without a shared expert).  An idx outside [0, E) sets FMOE_DEVERR_BAD_EXPERT and
+ * that token's y is not written. */
+fmoe_status fmoe_expert_forward(fmoe_layer_t layer, const uint16_t* x, const uint16_t* resid, int T,
+                                const int32_t* idx, const float* w, const float* shared_sigma,
+                                uint16_t* y, void* stream);
+
+/* The whole layer: routing, experts and combine, one token after another:
+ * y[t] = resid[t] + sum_k w_k o_k(x[t]) + sigma o_s(x[t]).  resid may equal x; y may
+ * alias resid but not x. */
+fmoe_status fmoe_layer_forward(fmoe_layer_t layer, const uint16_t* x, const uint16_t* resid, int T,
+                               uint16_t* y, void* stream);
+
+/* RMS normalisation with unit gain (hotdry.top "Metal GPU管线": two-pass RMSNorm, a
+ * sum of squares then the scaling): out[t] = bf16(h[t] / sqrt(mean(h[t]^2) + eps)),
+ * computed in double and rounded once.  h, out: bf16 [T][H], may alias. */
+fmoe_status fmoe_rmsnorm(const uint16_t* h, uint16_t* out, int T, int H, double eps, void* stream);
+
+/* Synchronises the device, returns the layer's device error bits in *device_error
+ * (0 if none) and clears them (and the layer's barrier state).  Returns FMOE_OK when no
+ * error was set, FMOE_ERR_DEVICE when one was. */
+fmoe_status fmoe_layer_get_error(fmoe_layer_t layer, uint32_t* device_error);
+
+/* Upper bound, in nanoseconds, of every device-side wait of this layer (grid-wide
+ * barriers, bulk-copy completion).  Default 2e9 (2 s).  A wait that exceeds it sets an
+ * error bit and the kernel returns. */
+fmoe_status fmoe_layer_set_wait_limit(fmoe_layer_t layer, uint64_t nanoseconds);
+
+/* Test hook for the failure path: when cta >= 0, thread block `cta` of the next forward
+ * calls returns before its first grid-wide barrier, so the other blocks' bounded wait
+ * runs out and FMOE_DEVERR_BARRIER_TIMEOUT is set.  -1 (default) disables it. */
+fmoe_status fmoe_layer_debug_hold_block(fmoe_layer_t layer, int cta);
+
+/* Number of thread blocks one forward launch uses (one per SM of the device). */
+int fmoe_layer_grid_size(fmoe_layer_t layer);
+
+/* Human-readable name of a status value. */
+const char* fmoe_status_string(fmoe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FMOE_H */

@@ -1,0 +1,56 @@
+"""The C-ABI library loads on a machine without a GPU and exports every symbol
+include/fmoe.h declares; host-only entry points answer without a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fmoe_synth as synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_dequant_expert_softmax_b200 import build, fmoe
+    build.build()
+    return fmoe
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "fmoe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fmoe_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) == 14
+    L = lib.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(lib.EXPORTS) == names
+
+
+def test_record_bytes_matches_format(lib):
+    for (H, I, b) in [(4096, 1024, 4), (4096, 1024, 2), (512, 128, 4), (64, 64, 2), (192, 320, 4)]:
+        assert lib.fmoe_record_bytes(H, I, b) == synth.record_bytes(H, I, b)
+    assert lib.fmoe_record_bytes(4096, 1000, 4) == 0
+    assert lib.fmoe_record_bytes(4096, 1024, 3) == 0
+
+
+def test_workspace_and_argument_checks(lib):
+    cfg = lib.fmoe_config(4096, 1024, 512, 4, 4, 1, 0)
+    assert lib.fmoe_workspace_bytes(cfg) > 0
+    bad = lib.fmoe_config(4096, 1024, 512, 600, 4, 1, 0)
+    assert lib.fmoe_workspace_bytes(bad) == 0
+    L = lib.lib()
+    h = ctypes.c_void_p()
+    w = lib.fmoe_weights(None, None, None, None)
+    assert L.fmoe_layer_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)) == 1
+    assert L.fmoe_layer_create(None, ctypes.byref(w), ctypes.byref(h)) == 1
+    assert L.fmoe_route(None, None, 1, None, None, None, None) == 1
+    assert L.fmoe_layer_forward(None, None, None, 1, None, None) == 1
+    assert L.fmoe_rmsnorm(None, None, 1, 64, -1.0, None) == 1
+    assert L.fmoe_status_string(4) == b"workspace missing or too small"
