@@ -289,12 +289,36 @@ def synthetic_layer(seed: int, layer: int, shape: "synth.LayerShape", lazy: bool
                        has_shared=bool(shape.has_shared))
 
 
-def within_tolerance(gpu: np.ndarray, ref: np.ndarray, rel: float = 2e-3):
-    """Per-element bound |gpu - ref| <= rel * (|ref| + rms(ref)); returns
-    (ok, worst ratio of error to bound)."""
+def bf16_half_ulp(v) -> np.ndarray:
+    """Half a unit in the last place of bf16 (8 significant bits) at magnitude |v|:
+    the largest error of round-to-nearest to bf16 for values of that binade."""
+    v = np.abs(np.asarray(v, dtype=np.float64))
+    _, e = np.frexp(np.where(v > 0, v, 1.0))
+    return np.where(v > 0, np.ldexp(1.0, e - 9), 0.0)
+
+
+def within_tolerance(gpu: np.ndarray, ref: np.ndarray, rel: float = 2e-3, out_bf16: bool = True):
+    """Per-element bound |gpu - ref| <= rel * (|ref| + rms(ref)) on the value before
+    the output's rounding to bf16: with ``out_bf16`` the bf16 half-ulp at the
+    bound's edge is added, because a correctly rounded bf16 value can itself be
+    2^-8 |ref| away from ref, more than rel * |ref| for rel = 2e-3.
+    Returns (ok, worst ratio of error to bound)."""
     ref = np.asarray(ref, dtype=np.float64)
     gpu = np.asarray(gpu, dtype=np.float64)
     rms = math.sqrt(float(np.mean(ref * ref)))
     bound = rel * (np.abs(ref) + rms)
+    if out_bf16:
+        bound = bound + bf16_half_ulp(np.abs(ref) + bound)
     ratio = np.abs(gpu - ref) / np.maximum(bound, 1e-300)
     return bool(np.all(ratio <= 1.0)), float(np.max(ratio)) if ratio.size else 0.0
+
+
+def bf16_agreement(gpu: np.ndarray, ref: np.ndarray):
+    """(fraction of elements equal to ref rounded to nearest-even bf16,
+    largest distance in bf16 ulps of ref's binade)."""
+    ref = np.asarray(ref, dtype=np.float64)
+    gpu = np.asarray(gpu, dtype=np.float64)
+    rb = bf16_to_f64(f64_to_bf16_bits(ref))
+    ulp = 2.0 * bf16_half_ulp(ref)
+    d = np.abs(gpu - rb) / np.where(ulp > 0, ulp, 1.0)
+    return float(np.mean(gpu == rb)), float(np.max(d)) if d.size else 0.0

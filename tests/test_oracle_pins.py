@@ -316,10 +316,34 @@ def test_rmsnorm_constant_and_library():
 def test_tolerance_helper():
     ref = np.array([1.0, -2.0, 0.0, 4.0])
     rms = math.sqrt(np.mean(ref ** 2))
-    ok, worst = oracle.within_tolerance(ref + 2e-3 * (np.abs(ref) + rms) * 0.99, ref)
+    ok, worst = oracle.within_tolerance(ref + 2e-3 * (np.abs(ref) + rms) * 0.99, ref, out_bf16=False)
     assert ok and worst < 1.0
-    ok, _ = oracle.within_tolerance(ref + np.array([0, 0, 2e-3 * rms * 1.01, 0]), ref)
+    ok, _ = oracle.within_tolerance(ref + np.array([0, 0, 2e-3 * rms * 1.01, 0]), ref, out_bf16=False)
     assert not ok
+
+
+def test_bf16_rounded_values_always_pass_and_two_ulps_fail():
+    """A correctly rounded bf16 output passes the bound whatever its magnitude; an
+    output two bf16 ulps off fails wherever |ref| dominates rms."""
+    rng = np.random.default_rng(5)
+    ref = rng.standard_normal(20000) * np.exp(rng.standard_normal(20000))
+    rounded = oracle.bf16_to_f64(oracle.f64_to_bf16_bits(ref))
+    assert oracle.within_tolerance(rounded, ref)[0]
+    assert oracle.bf16_agreement(rounded, ref) == (1.0, 0.0)
+    # the bound before rounding alone would reject some correctly rounded values
+    assert not oracle.within_tolerance(rounded, ref, out_bf16=False)[0]
+    big = np.argmax(np.abs(ref))
+    bad = rounded.copy()
+    bad[big] += 4 * oracle.bf16_half_ulp(ref[big])
+    assert not oracle.within_tolerance(bad, ref)[0]
+    assert oracle.bf16_agreement(bad, ref)[1] == 2.0
+
+
+def test_bf16_half_ulp_values():
+    assert oracle.bf16_half_ulp(1.0) == 2.0 ** -8
+    assert oracle.bf16_half_ulp(8.2759) == 2.0 ** -5
+    assert oracle.bf16_half_ulp(-0.75) == 2.0 ** -9
+    assert oracle.bf16_half_ulp(0.0) == 0.0
 
 
 def test_golden_tiny_regression():
