@@ -38,12 +38,12 @@ bool record_layout(int H, int I, int bits, RecordLayout* L) {
 }
 
 struct WsLayout {
-  size_t err, bar, lpart, hbuf, size;
+  size_t err, tokens, rflags, hflags, lpart, hbuf, size;
 };
 
 int router_splits(int H) {
   int nq = 1;
-  for (int n = 2; n <= 8; n *= 2)
+  for (int n = 2; n <= kMaxSplits; n *= 2)
     if (H % (n * 128) == 0 && H / n >= 1024) nq = n;
   return nq;
 }
@@ -51,9 +51,12 @@ int router_splits(int H) {
 WsLayout ws_layout(const fmoe_config& c) {
   WsLayout w;
   const int nq = router_splits(c.hidden);
+  const size_t flag_bytes = (size_t)kMaxGrid * kFlagStride * sizeof(uint32_t);
   w.err = 0;
-  w.bar = 64;
-  w.lpart = 256;
+  w.tokens = 128;
+  w.rflags = 256;
+  w.hflags = w.rflags + flag_bytes;
+  w.lpart = w.hflags + flag_bytes;
   w.hbuf = al256(w.lpart + 2 * (size_t)(c.n_experts + 1) * nq * sizeof(double));
   w.size = al256(w.hbuf + 2 * (size_t)(c.top_k + 1) * c.inter * sizeof(float));
   return w;
@@ -87,6 +90,8 @@ struct fmoe_layer {
   WsLayout wsl;
   uint64_t wait_ns;
   int hold_cta;
+  uint64_t* timeline;
+  int timeline_token;
 };
 
 namespace {
@@ -103,7 +108,7 @@ fmoe_status plan(fmoe_layer* L) {
   const fmoe_config& c = L->cfg;
   const int cols = c.bits == 4 ? chunk_cols<4>() : chunk_cols<2>();
   const int nslots = c.top_k + c.has_shared;
-  if (c.top_k > kMaxK) return FMOE_ERR_UNSUPPORTED;
+  if (c.top_k > kMaxK || c.n_experts + c.has_shared > kMaxExperts || L->sms > kMaxGrid) return FMOE_ERR_UNSUPPORTED;
   L->nq = router_splits(c.hidden);
   int rp = 1;
   while (rp < 8 && (size_t)(rp * 2) * 2 * L->rec.qh <= 8192 && c.inter % (rp * 2) == 0) rp *= 2;
@@ -114,16 +119,21 @@ fmoe_status plan(fmoe_layer* L) {
   if (fixed >= (uint32_t)kMaxSmem) return FMOE_ERR_UNSUPPORTED;
   const uint32_t staging = (uint32_t)kMaxSmem - fixed;
   const int G = L->sms;
-  // P1: x in doubles, the router rows a block touches, its shared gate/up rows
+  // P1: x in doubles and the router rows a block touches from the start of the
+  // staging area, its shared gate/up rows at the end; top-K's logits and
+  // candidates must not reach the shared rows either (they are consumed after it)
   const long long U = (long long)(c.n_experts + c.has_shared) * L->nq;
   const uint32_t rows_touched = (uint32_t)(((U + G - 1) / G + L->nq - 1) / L->nq + 1);
   const int shared_rows = (c.inter + G - 1) / G;
-  const uint64_t p1 = r128((uint32_t)c.hidden * 8u) + (uint64_t)rows_touched * g.router_item() +
-                      (c.has_shared ? (uint64_t)g.gu_bytes(shared_rows) : 0ull);
+  const uint32_t sc_off = c.has_shared ? ((staging - g.gu_bytes(shared_rows)) & ~127u) : staging;
+  const uint64_t p1 = r128((uint32_t)c.hidden * 8u) + (uint64_t)rows_touched * g.router_item();
   const uint32_t p1_items = rows_touched + (c.has_shared ? (uint32_t)g.gu_items(shared_rows) : 0u);
-  if (p1 > staging || p1_items > (uint32_t)kMaxRoundItems) return FMOE_ERR_UNSUPPORTED;
-  // logits and selection keys for top-K
-  if ((uint64_t)r128((uint32_t)(c.n_experts + 1) * 8u) + (uint64_t)c.n_experts * 8u > staging)
+  if (c.has_shared && g.gu_bytes(shared_rows) >= staging) return FMOE_ERR_UNSUPPORTED;
+  if (p1 > sc_off || p1_items > (uint32_t)kMaxRoundItems) return FMOE_ERR_UNSUPPORTED;
+  // top-K: logits, selection keys, per-warp candidates
+  if ((uint64_t)r128((uint32_t)(c.n_experts + 1) * 8u) + (uint64_t)((c.n_experts + 15) & ~15) * 8u +
+          (uint64_t)kWarps * c.top_k * 12u >
+      sc_off)
     return FMOE_ERR_UNSUPPORTED;
   // P2: at least one gate/up row pair per round
   if (g.gu_bytes(1) > staging) return FMOE_ERR_UNSUPPORTED;
@@ -165,12 +175,16 @@ Params base_params(const fmoe_layer* L, int mode, int T) {
   p.sgate = L->w.shared_gate;
   uint8_t* ws = static_cast<uint8_t*>(L->ws);
   p.err = reinterpret_cast<uint32_t*>(ws + L->wsl.err);
-  p.bar = reinterpret_cast<unsigned long long*>(ws + L->wsl.bar);
+  p.tokens = reinterpret_cast<uint32_t*>(ws + L->wsl.tokens);
+  p.rflags = reinterpret_cast<uint32_t*>(ws + L->wsl.rflags);
+  p.hflags = reinterpret_cast<uint32_t*>(ws + L->wsl.hflags);
   p.lpart = reinterpret_cast<double*>(ws + L->wsl.lpart);
   p.hbuf = reinterpret_cast<float*>(ws + L->wsl.hbuf);
   p.staging_bytes = L->staging_bytes;
   p.wait_ns = L->wait_ns;
   p.hold_cta = L->hold_cta;
+  p.timeline = reinterpret_cast<unsigned long long*>(L->timeline);
+  p.timeline_token = L->timeline_token;
   return p;
 }
 
@@ -347,9 +361,9 @@ fmoe_status fmoe_layer_get_error(fmoe_layer_t L, uint32_t* device_error) {
   if (cudaMemcpy(&e, ws + L->wsl.err, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return FMOE_ERR_CUDA;
   *device_error = e;
   if (e == 0) return FMOE_OK;
-  // clear the error word and the barrier counter (left mid-epoch by an aborted launch)
-  if (cudaMemset(ws + L->wsl.err, 0, 4) != cudaSuccess) return FMOE_ERR_CUDA;
-  if (cudaMemset(ws + L->wsl.bar, 0, 8) != cudaSuccess) return FMOE_ERR_CUDA;
+  // clear the whole workspace: the error word, the tag base and any values an
+  // aborted launch left behind
+  if (cudaMemset(ws, 0, L->wsl.size) != cudaSuccess) return FMOE_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
   return FMOE_ERR_DEVICE;
 }
@@ -363,6 +377,13 @@ fmoe_status fmoe_layer_set_wait_limit(fmoe_layer_t L, uint64_t nanoseconds) {
 fmoe_status fmoe_layer_debug_hold_block(fmoe_layer_t L, int cta) {
   if (!L || cta < -1 || cta >= L->sms) return FMOE_ERR_INVALID_ARG;
   L->hold_cta = cta;
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_layer_debug_timeline(fmoe_layer_t L, uint64_t* dev_buf, int token) {
+  if (!L || token < 0) return FMOE_ERR_INVALID_ARG;
+  L->timeline = dev_buf;
+  L->timeline_token = token;
   return FMOE_OK;
 }
 

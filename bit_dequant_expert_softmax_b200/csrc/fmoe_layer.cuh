@@ -30,6 +30,10 @@ constexpr int kNumBars = 96;
 constexpr int kMaxRoundItems = kNumBars / 2;
 constexpr int kMaxDownBlock = 2 * kWarps;  // output rows per down item (two per warp)
 constexpr int kMaxChunks = 8;              // gate/up chunks per round
+constexpr int kMaxExperts = 2048;          // routed experts a layer may have
+constexpr int kMaxSplits = 4;              // router column splits
+constexpr int kMaxGrid = 256;              // blocks a launch may have (flag words reserved)
+constexpr int kFlagStride = 8;             // uint32 per flag (one 32-byte sector each)
 
 enum Mode : int { MODE_ROUTE = 1, MODE_EXPERTS = 2, MODE_FULL = 3 };
 
@@ -55,12 +59,16 @@ struct Params {
   const float* w_in;
   const float* sig_in;
   uint32_t* err;
-  unsigned long long* bar;
-  double* lpart;  // [2][(E+1)*nq]
-  float* hbuf;    // [2][(K+1)*I]
+  uint32_t* tokens;  // tokens this workspace has seen (tag base)
+  uint32_t* rflags;  // [kMaxGrid * kFlagStride] per-block "router partials written" tags
+  uint32_t* hflags;  // [kMaxGrid * kFlagStride] per-block "h rows written" tags
+  double* lpart;     // [2][(E+1)*nq] router partials
+  float* hbuf;       // [2][(K+1)*I]  h values
   int staging_bytes;
   unsigned long long wait_ns;
   int hold_cta;
+  unsigned long long* timeline;  // diagnostic: [grid][16] phase timestamps of one token, or null
+  int timeline_token;
 };
 
 // Shared-memory header (activations and the staging area follow it).
@@ -70,6 +78,7 @@ struct alignas(128) SmemHeader {
   float wsl[kMaxK + 1];  // weight of each slot (w_k; slot K = sigma)
   int abort_flag;
   int skip_token;
+  uint32_t tok_base;
 };
 
 __host__ __device__ constexpr uint32_t r16(uint32_t n) { return (n + 15u) & ~15u; }
@@ -121,11 +130,13 @@ struct LayerKernel {
   const Params& p;
   Geometry g;
   SmemHeader* hdr;
-  float* xs;       // pre-scaled, lane-interleaved activations [H]
+  float* xs;       // pre-scaled, lane-interleaved activations [padded H]
   float* xsum;     // per-chunk sums of the unscaled activations [H / kCols]
   uint8_t* stage;  // staging area
+  uint32_t cap;    // staging bytes
   uint32_t nitem;  // items issued so far (same value in every thread)
   int nslots;
+  int tok_;
 
   __device__ LayerKernel(const Params& pp, uint8_t* smem) : p(pp) {
     nslots = p.K + (p.has_shared ? 1 : 0);
@@ -134,7 +145,9 @@ struct LayerKernel {
     xs = reinterpret_cast<float*>(smem + sizeof(SmemHeader));
     xsum = xs + g.padded(p.H);
     stage = smem + g.fixed_bytes(sizeof(SmemHeader));
+    cap = static_cast<uint32_t>(p.staging_bytes);
     nitem = 0;
+    tok_ = -1;
   }
 
   __device__ __forceinline__ uint64_t* bar_of(uint32_t n) const { return &hdr->bars[n % kNumBars]; }
@@ -148,6 +161,12 @@ struct LayerKernel {
     return p.experts + static_cast<unsigned long long>(expert) * p.rec_bytes;
   }
 
+  // diagnostic timestamps (token 0 only; off unless a timeline buffer is attached)
+  __device__ __forceinline__ void mark(int i) const {
+    if (p.timeline != nullptr && tok_ == p.timeline_token && threadIdx.x == 0)
+      p.timeline[static_cast<size_t>(blockIdx.x) * 16 + i] = global_timer_ns();
+  }
+
   // Waits (bounded) for every copy this block may still have in flight.
   __device__ void drain() {
     __syncthreads();
@@ -158,93 +177,227 @@ struct LayerKernel {
     __syncthreads();
   }
 
-  // ---------------------------------------------------------------- grid barrier
-  __device__ bool grid_sync() {
+  // ---------------------------------------------------------------- exchanges
+  // Values every block needs from all others (router partials, h rows) are written
+  // with plain stores; then the block publishes the token's tag in its own flag word
+  // with a release store.  A reader's warp 0 polls the grid's flags (each lane a few,
+  // all of a lane's loads in flight together, relaxed loads, bounded), fences, and
+  // the block then reads the values once from L2.  Buffers alternate by token parity;
+  // no block can run two tokens ahead of another because each token needs every
+  // block's values.
+  uint32_t tbase_;
+  __device__ __forceinline__ uint32_t tag32(int t) const {
+    return (tbase_ + static_cast<uint32_t>(t)) % 0xFFFFFFFFu + 1u;
+  }
+
+  __device__ __forceinline__ void publish(uint32_t* flags, int t) {
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int ok = hdr->abort_flag == 0;
-      __threadfence();
-      const unsigned long long old = atomicAdd(p.bar, 1ull);
-      const unsigned long long target = (old / gridDim.x + 1ull) * gridDim.x;
-      const uint64_t t0 = global_timer_ns();
-      while (ok && ld_acquire_u64(p.bar) < target) {
-        if ((ld_relaxed_u32(p.err) & FMOE_DEVERR_BARRIER_TIMEOUT) || global_timer_ns() - t0 > p.wait_ns) {
-          atomicOr(p.err, FMOE_DEVERR_BARRIER_TIMEOUT);
-          ok = 0;
+    if (threadIdx.x == 0) st_release_u32(flags + blockIdx.x * kFlagStride, tag32(t));
+  }
+
+  __device__ bool wait_all(const uint32_t* flags, int t) {
+    int fail = 0;
+    if (threadIdx.x < 32) {
+      const int G = gridDim.x, lane = threadIdx.x;
+      const uint32_t want = tag32(t);
+      constexpr int NF = kMaxGrid / 32;
+      uint32_t got[NF];
+#pragma unroll
+      for (int i = 0; i < NF; ++i) {
+        const int b = lane + 32 * i;
+        got[i] = b < G ? ld_relaxed_u32(flags + b * kFlagStride) : want;
+      }
+      uint64_t t0 = 0;
+      for (int it = 0;; ++it) {
+        bool all = true;
+#pragma unroll
+        for (int i = 0; i < NF; ++i) all &= got[i] == want;
+        if (__all_sync(0xffffffffu, all)) break;
+        if ((it & 15) == 15) {
+          if (t0 == 0) t0 = global_timer_ns();
+          const bool bad =
+              (ld_relaxed_u32(p.err) & FMOE_DEVERR_BARRIER_TIMEOUT) || global_timer_ns() - t0 > p.wait_ns;
+          if (__any_sync(0xffffffffu, bad)) {
+            if (lane == 0) atomicOr(p.err, FMOE_DEVERR_BARRIER_TIMEOUT);
+            fail = 1;
+            break;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < NF; ++i) {
+          const int b = lane + 32 * i;
+          if (got[i] != want) got[i] = ld_relaxed_u32(flags + b * kFlagStride);
         }
       }
       __threadfence();
-      if (!ok) hdr->abort_flag = 1;
     }
-    __syncthreads();
-    return hdr->abort_flag == 0;
+    return __syncthreads_or(fail) == 0;
   }
 
   // ---------------------------------------------------------------- activations
-  __device__ void stage_vec(const float* src_f32, const uint16_t* src_bf16, int n, float* dst, float* dsum) {
-    for (int c = threadIdx.x; c < n; c += blockDim.x) {
-      const float v = src_bf16 ? bf16_to_f32(src_bf16[c]) : __ldcg(src_f32 + c);
-      dst[C::phys(c)] = v * prescale_factor(C::shift_of(c));
+  // Column group q = columns [4q, 4q+4).  Two passes, all loads in flight together:
+  //  natural (thread -> consecutive groups): chunk sums by shuffles over the kCols/4
+  //    threads of a chunk, and for x the doubles of the router (split in two double2
+  //    arrays so the router's loads are conflict-free);
+  //  transposed (thread -> consecutive float4 slots of the lane-interleaved layout):
+  //    pre-scaled floats, conflict-free 16-byte stores.
+  __device__ __forceinline__ float4 prescale4(float4 v, int c0) const {
+    return make_float4(v.x * prescale_factor(C::shift_of(c0)), v.y * prescale_factor(C::shift_of(c0 + 1)),
+                       v.z * prescale_factor(C::shift_of(c0 + 2)), v.w * prescale_factor(C::shift_of(c0 + 3)));
+  }
+  // column of the first element of float4 slot `idx` of the interleaved layout (-1: padding)
+  __device__ __forceinline__ int slot_col(int idx, int nch) const {
+    const int lane_m = idx & 31, f = (idx >> 5) % C::kF4, hi = (idx >> 5) / C::kF4;
+    const int m = hi * 32 + lane_m;
+    return m < nch ? m * C::kCols + 4 * f : -1;
+  }
+
+  __device__ __forceinline__ float4 bf16x4(uint2 u) const {
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
+                       __uint_as_float(u.y & 0xFFFF0000u));
+  }
+
+  __device__ void stage_x(const uint16_t* xt, double2* xa, double2* xb) {
+    constexpr int TPC = C::kCols / 4;
+    const int n4 = p.H / 4, nch = p.H / C::kCols;
+    const int F = static_cast<int>(g.padded(p.H) / 4);
+    const uint2* src = reinterpret_cast<const uint2*>(xt);
+    for (int base = 0; base < max(n4, F); base += 2 * kThreads) {
+      uint2 nat[2], tr[2];
+      int trc[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
+        nat[k] = q < n4 ? src[q] : make_uint2(0, 0);
+        trc[k] = q < F ? slot_col(q, nch) : -1;
+        tr[k] = trc[k] >= 0 ? src[trc[k] / 4] : make_uint2(0, 0);
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
+        const float4 v = bf16x4(nat[k]);
+        float sum = (v.x + v.y) + (v.z + v.w);
+#pragma unroll
+        for (int o = 1; o < TPC; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (q < n4) {
+          if (xa) {
+            xa[q] = make_double2(v.x, v.y);
+            xb[q] = make_double2(v.z, v.w);
+          }
+          if (q % TPC == 0) xsum[q / TPC] = sum;
+        }
+        if (q < F) {
+          const float4 w = trc[k] >= 0 ? prescale4(bf16x4(tr[k]), trc[k]) : make_float4(0.f, 0.f, 0.f, 0.f);
+          reinterpret_cast<float4*>(xs)[q] = w;
+        }
+      }
     }
-    for (int m = threadIdx.x; m < n / C::kCols; m += blockDim.x) {
-      float s = 0.f;
-      for (int j = 0; j < C::kCols; ++j)
-        s += src_bf16 ? bf16_to_f32(src_bf16[m * C::kCols + j]) : __ldcg(src_f32 + m * C::kCols + j);
-      dsum[m] = s;
+  }
+
+  // h of every slot (fp32, written by other blocks, read from L2 once every block
+  // has published): natural pass for the chunk sums, transposed pass for the
+  // conflict-free stores; all loads of a thread in flight together.
+  __device__ void stage_h(const float* hb, float* hs, uint32_t hstride, float* hsum) {
+    constexpr int TPC = C::kCols / 4;
+    const int per_slot = p.I / 4, nch = p.I / C::kCols;
+    const int n4 = nslots * per_slot;
+    const int F1 = static_cast<int>(hstride / 4), F = nslots * F1;
+    const float4* src = reinterpret_cast<const float4*>(hb);
+    for (int base = 0; base < max(n4, F); base += 2 * kThreads) {
+      float4 nat[2], tr[2];
+      int trc[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
+        nat[k] = q < n4 ? __ldcg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        trc[k] = q < F ? slot_col(q % F1, nch) : -1;
+        tr[k] = trc[k] >= 0 ? __ldcg(src + (q / F1) * per_slot + trc[k] / 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
+        float sum = (nat[k].x + nat[k].y) + (nat[k].z + nat[k].w);
+#pragma unroll
+        for (int o = 1; o < TPC; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (q < n4 && q % TPC == 0) hsum[(q / per_slot) * nch + (q % per_slot) / TPC] = sum;
+        if (q < F) {
+          const float4 w = trc[k] >= 0 ? prescale4(tr[k], trc[k]) : make_float4(0.f, 0.f, 0.f, 0.f);
+          reinterpret_cast<float4*>(hs)[(q / F1) * (hstride / 4) + q % F1] = w;
+        }
+      }
     }
   }
 
   // ---------------------------------------------------------------- dot products
   // Lane partial of sum_c W[r][c] v[c] over the lane's chunks, for up to two rows
   // sharing the activation loads (W = scale*code + bias; v pre-scaled, interleaved).
+  // Two accumulator pairs per row halve the dependent FMA chains.
   __device__ __forceinline__ void dot2(const uint8_t* q0, const uint32_t* s0, const uint8_t* q1,
                                        const uint32_t* s1, bool two, const float* vs, const float* vsum,
                                        int nch, float& r0, float& r1) const {
     const int lane = threadIdx.x & 31;
+#pragma unroll 2
     for (int m = lane; m < nch; m += 32) {
       const uint4 a4 = *reinterpret_cast<const uint4*>(q0 + 16 * m);
       uint4 b4 = make_uint4(0, 0, 0, 0);
       if (two) b4 = *reinterpret_cast<const uint4*>(q1 + 16 * m);
       const uint32_t wa[4] = {a4.x, a4.y, a4.z, a4.w};
       const uint32_t wb[4] = {b4.x, b4.y, b4.z, b4.w};
-      float2 aa = make_float2(0.f, 0.f), ab = make_float2(0.f, 0.f);
+      float2 aa0 = make_float2(0.f, 0.f), aa1 = aa0, ab0 = aa0, ab1 = aa0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         float4 xv[C::kF4PerWord];
 #pragma unroll
         for (int f = 0; f < C::kF4PerWord; ++f) xv[f] = *C::f4(vs, m, j * C::kF4PerWord + f);
-        word_fma<BITS>(wa[j], xv, aa);
-        if (two) word_fma<BITS>(wb[j], xv, ab);
+        word_fma<BITS>(wa[j], xv, j < 2 ? aa0 : aa1);
+        if (two) word_fma<BITS>(wb[j], xv, j < 2 ? ab0 : ab1);
       }
       const float vm = vsum[m];
       const uint32_t sa = s0[C::sb_index(m)];
-      r0 = fmaf(sb_scale(sa), (aa.x + aa.y) * kUnscale, r0);
+      r0 = fmaf(sb_scale(sa), ((aa0.x + aa0.y) + (aa1.x + aa1.y)) * kUnscale, r0);
       r0 = fmaf(sb_bias(sa), vm, r0);
       if (two) {
         const uint32_t sbv = s1[C::sb_index(m)];
-        r1 = fmaf(sb_scale(sbv), (ab.x + ab.y) * kUnscale, r1);
+        r1 = fmaf(sb_scale(sbv), ((ab0.x + ab0.y) + (ab1.x + ab1.y)) * kUnscale, r1);
         r1 = fmaf(sb_bias(sbv), vm, r1);
       }
     }
   }
 
   // ---------------------------------------------------------------- gate/up chunks
-  __device__ void issue_gu(const GuChunk& c) {
+  // Item i of chunk c (row pairs [ra + i*rp, ...)); the chunk's (scale,bias) cover
+  // rides on item 0.  Called by one lane per item.
+  __device__ void issue_gu_item(const GuChunk& c, int i) {
     const uint8_t* rec = record(hdr->sel[c.slot]);
     const int n = c.rb - c.ra;
-    const unsigned long long sb_start = p.o_gu_sb + static_cast<unsigned long long>(c.ra) * 2u * p.sh;
-    const unsigned long long sb_a = sb_start & ~15ull;
-    const unsigned long long sb_end = (sb_start + static_cast<unsigned long long>(n) * 2u * p.sh + 15ull) & ~15ull;
-    const uint32_t sbb = static_cast<uint32_t>(sb_end - sb_a);
-    const int items = g.gu_items(n);
-    for (int i = 0; i < items; ++i) {
-      const int a = c.ra + i * p.rp, b = min(c.rb, a + p.rp);
-      const uint32_t qb = static_cast<uint32_t>(b - a) * 2u * p.qh;
-      uint64_t* bar = bar_of(c.first + i);
-      mbar_arrive_expect_tx(bar, qb + (i == 0 ? sbb : 0u));
-      bulk_g2s(stage + c.off + static_cast<uint32_t>(a - c.ra) * 2u * p.qh,
-               rec + static_cast<unsigned long long>(a) * 2u * p.qh, qb, bar);
-      if (i == 0) bulk_g2s(stage + c.off + g.gu_q(n), rec + sb_a, sbb, bar);
+    const int a = c.ra + i * p.rp, b = min(c.rb, a + p.rp);
+    const uint32_t qb = static_cast<uint32_t>(b - a) * 2u * p.qh;
+    uint32_t sbb = 0;
+    unsigned long long sb_a = 0;
+    if (i == 0) {
+      const unsigned long long sb_start = p.o_gu_sb + static_cast<unsigned long long>(c.ra) * 2u * p.sh;
+      sb_a = sb_start & ~15ull;
+      const unsigned long long sb_end =
+          (sb_start + static_cast<unsigned long long>(n) * 2u * p.sh + 15ull) & ~15ull;
+      sbb = static_cast<uint32_t>(sb_end - sb_a);
+    }
+    uint64_t* bar = bar_of(c.first + i);
+    mbar_arrive_expect_tx(bar, qb + sbb);
+    bulk_g2s(stage + c.off + static_cast<uint32_t>(a - c.ra) * 2u * p.qh,
+             rec + static_cast<unsigned long long>(a) * 2u * p.qh, qb, bar);
+    if (i == 0) bulk_g2s(stage + c.off + g.gu_q(n), rec + sb_a, sbb, bar);
+  }
+
+  // Warp 0: issue every item of `nc` chunks, one lane per item.
+  __device__ void issue_gu(const GuChunk* ch, int nc) {
+    if (threadIdx.x >= 32) return;
+    fence_proxy_async_smem();
+    int base = 0;
+    for (int k = 0; k < nc; ++k) {
+      const int items = g.gu_items(ch[k].rb - ch[k].ra);
+      for (int i = static_cast<int>(threadIdx.x) - base; i < items; i += 32)
+        if (i >= 0) issue_gu_item(ch[k], i);
+      base = (base + items) % 32;
     }
   }
 
@@ -270,13 +423,12 @@ struct LayerKernel {
     return true;
   }
 
-  // Consume every row pair of `nc` chunks, spread over the warps.
+  // Consume every row pair of `nc` chunks, spread over the warps (unit u -> warp u % kWarps).
   __device__ void gu_consume(const GuChunk* ch, int nc, int buf) {
     const int warp = threadIdx.x >> 5;
     int base = 0;
     for (int k = 0; k < nc; ++k) {
       const int n = ch[k].rb - ch[k].ra;
-      // unit u of this round goes to warp u % kWarps
       int first = (warp - base) % kWarps;
       if (first < 0) first += kWarps;
       for (int i = first; i < n; i += kWarps) {
@@ -289,9 +441,9 @@ struct LayerKernel {
     }
   }
 
-  // Gate/up of units [v0, v1) of the slot list starting at slot s_lo (unit = s*I + r):
-  // chunks per slot, in rounds that fit `cap` bytes from staging offset `base`.
-  __device__ bool gu_rounds(int s_lo, int v0, int v1, uint32_t base, uint32_t cap, int buf) {
+  // Gate/up of routed units [v0, v1) (unit = slot*I + r) in rounds that fit the
+  // whole staging area (used when the block's share does not fit at once).
+  __device__ bool gu_rounds(int v0, int v1, int buf) {
     GuChunk ch[kMaxChunks];
     int nc = 0, items = 0;
     uint32_t used = 0;
@@ -316,10 +468,7 @@ struct LayerKernel {
           hdr->abort_flag = 1;
           return false;
         }
-        if (threadIdx.x == 0) {
-          fence_proxy_async_smem();
-          for (int k = 0; k < nc; ++k) issue_gu(ch[k]);
-        }
+        issue_gu(ch, nc);
         nitem += static_cast<uint32_t>(items);
         gu_consume(ch, nc, buf);
         __syncthreads();
@@ -330,10 +479,10 @@ struct LayerKernel {
         if (v >= v1) return true;
         continue;
       }
-      ch[nc] = GuChunk{s_lo + s, r, r + n, base + used, nitem + static_cast<uint32_t>(items)};
+      ch[nc] = GuChunk{s, r, r + n, used, nitem + static_cast<uint32_t>(items)};
       ++nc;
       items += g.gu_items(n);
-      used += g.gu_bytes(n);
+      used = r128(used + g.gu_bytes(n));
       v += n;
     }
   }
@@ -361,14 +510,13 @@ struct LayerKernel {
     }
   }
 
-  // Items [ka, kb) of the block's rows [j0, j1) placed from staging offset `base`.
+  // Warp 0: items [ka, kb) of the block's rows [j0, j1) from staging offset `base`.
   __device__ void issue_down_items(int j0, int j1, int ka, int kb, uint32_t first, uint32_t base) {
-    if (threadIdx.x == 0) {
-      fence_proxy_async_smem();
-      for (int k = ka; k < kb; ++k) {
-        const int ja = j0 + k * p.db, n = min(j1, ja + p.db) - ja;
-        issue_down(first + (k - ka), base + (k - ka) * g.dn_item(p.db), ja, n);
-      }
+    if (threadIdx.x >= 32) return;
+    fence_proxy_async_smem();
+    for (int k = ka + static_cast<int>(threadIdx.x); k < kb; k += 32) {
+      const int ja = j0 + k * p.db, n = min(j1, ja + p.db) - ja;
+      issue_down(first + (k - ka), base + (k - ka) * g.dn_item(p.db), ja, n);
     }
   }
 
@@ -408,141 +556,219 @@ struct LayerKernel {
 
   // ---------------------------------------------------------------- P1
   // Router units [u0, u1) over (E + has_shared) rows x nq splits (the shared gate
-  // vector is the last row), plus the block's slice of the shared expert's gate/up.
-  __device__ bool phase1(int buf, bool route, bool shared_gu) {
+  // vector is the last row) staged after the router's doubles; the block's slice of
+  // the shared expert's gate/up rows staged at the end of the staging area, to be
+  // consumed after top-K while the routed rows are in flight.  All copies are issued
+  // before the activations are staged (they do not depend on them).
+  int u0_, u1_, row0_, row1_;
+  uint32_t p1first_, rbase_;
+  GuChunk sc_;
+  bool has_sc_;
+
+  __device__ void phase1_issue(bool route, bool shared_gu) {
     const int rows = p.E + (p.has_shared ? 1 : 0);
     const int G = gridDim.x, b = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int u0 = 0, u1 = 0, row0 = 0, row1 = 0;
+    u0_ = u1_ = row0_ = row1_ = 0;
     if (route) {
       const long long U = static_cast<long long>(rows) * p.nq;
-      u0 = static_cast<int>(U * b / G);
-      u1 = static_cast<int>(U * (b + 1) / G);
-      row0 = u0 / p.nq;
-      row1 = (u1 + p.nq - 1) / p.nq;
+      u0_ = static_cast<int>(U * b / G);
+      u1_ = static_cast<int>(U * (b + 1) / G);
+      row0_ = u0_ / p.nq;
+      row1_ = (u1_ + p.nq - 1) / p.nq;
     }
     const int hc = p.H / p.nq;
     const uint32_t rib = g.router_item();
-    const uint32_t rbase = route ? r128(static_cast<uint32_t>(p.H) * 8u) : 0u;
-    const int nrouter = row1 - row0;
-    const uint32_t first = nitem;
-    GuChunk sc{p.K, 0, 0, rbase + static_cast<uint32_t>(nrouter) * rib, first + static_cast<uint32_t>(nrouter)};
+    rbase_ = route ? r128(static_cast<uint32_t>(p.H) * 8u) : 0u;
+    const int nrouter = row1_ - row0_;
+    p1first_ = nitem;
+    sc_ = GuChunk{p.K, 0, 0, 0, p1first_ + static_cast<uint32_t>(nrouter)};
     if (shared_gu) {
-      sc.ra = static_cast<int>(static_cast<long long>(p.I) * b / G);
-      sc.rb = static_cast<int>(static_cast<long long>(p.I) * (b + 1) / G);
+      sc_.ra = static_cast<int>(static_cast<long long>(p.I) * b / G);
+      sc_.rb = static_cast<int>(static_cast<long long>(p.I) * (b + 1) / G);
     }
-    const int nsh = sc.rb > sc.ra ? g.gu_items(sc.rb - sc.ra) : 0;
-    if (threadIdx.x == 0) {
+    has_sc_ = sc_.rb > sc_.ra;
+    const int nsh = has_sc_ ? g.gu_items(sc_.rb - sc_.ra) : 0;
+    if (has_sc_) sc_.off = (cap - g.gu_bytes(sc_.rb - sc_.ra)) & ~127u;
+    if (threadIdx.x < 32) {
       fence_proxy_async_smem();
-      for (int r = row0; r < row1; ++r) {
-        const int ua = max(u0, r * p.nq), ub = min(u1, r * p.nq + p.nq);
-        uint64_t* bar = bar_of(first + (r - row0));
+      for (int r = row0_ + static_cast<int>(threadIdx.x); r < row1_; r += 32) {
+        const int ua = max(u0_, r * p.nq), ub = min(u1_, r * p.nq + p.nq);
+        uint64_t* bar = bar_of(p1first_ + (r - row0_));
         const uint32_t bytes = static_cast<uint32_t>(ub - ua) * hc * 4u;
         const float* src = (r < p.E) ? p.router + static_cast<size_t>(r) * p.H : p.sgate;
         src += static_cast<size_t>(ua - r * p.nq) * hc;
         mbar_arrive_expect_tx(bar, bytes);
-        bulk_g2s(stage + rbase + (r - row0) * rib + static_cast<uint32_t>(ua - r * p.nq) * hc * 4u, src, bytes, bar);
+        bulk_g2s(stage + rbase_ + (r - row0_) * rib + static_cast<uint32_t>(ua - r * p.nq) * hc * 4u, src, bytes,
+                 bar);
       }
-      if (nsh) issue_gu(sc);
+      for (int i = static_cast<int>(threadIdx.x) - (nrouter % 32); i < nsh; i += 32)
+        if (i >= 0) issue_gu_item(sc_, i);
     }
     nitem += static_cast<uint32_t>(nrouter + nsh);
+  }
+
+  // Router dot products of this block's units: fp64 sums of exact fp32 x bf16 products.
+  __device__ bool phase1_consume(int buf, bool route) {
     if (route) {
-      const double* x64 = reinterpret_cast<const double*>(stage);
+      const int rows = p.E + (p.has_shared ? 1 : 0);
+      const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+      const int hc = p.H / p.nq;
+      const uint32_t rib = g.router_item();
+      const double2* xa = reinterpret_cast<const double2*>(stage);
+      const double2* xb = xa + p.H / 4;
       double* lpart = p.lpart + static_cast<size_t>(buf) * rows * p.nq;
-      for (int u = u0 + warp; u < u1; u += kWarps) {
-        const int r = u / p.nq, q = u % p.nq;
-        if (!wait_item(first + (r - row0))) {
+      for (int u = u0_ + warp; u < u1_; u += kWarps) {
+        const int r = u / p.nq, qq = u % p.nq;
+        if (!wait_item(p1first_ + (r - row0_))) {
           hdr->abort_flag = 1;
           break;
         }
-        const float* wrow = reinterpret_cast<const float*>(stage + rbase + (r - row0) * rib) + q * hc;
-        const double* xq = x64 + q * hc;
-        double acc = 0.0;
-        for (int c = 4 * lane; c < hc; c += 128) {
-          const float4 wv = *reinterpret_cast<const float4*>(wrow + c);
-          const double2 xa = *reinterpret_cast<const double2*>(xq + c);
-          const double2 xb = *reinterpret_cast<const double2*>(xq + c + 2);
-          acc = fma(static_cast<double>(wv.x), xa.x, acc);
-          acc = fma(static_cast<double>(wv.y), xa.y, acc);
-          acc = fma(static_cast<double>(wv.z), xb.x, acc);
-          acc = fma(static_cast<double>(wv.w), xb.y, acc);
+        const float4* wrow = reinterpret_cast<const float4*>(stage + rbase_ + (r - row0_) * rib) + qq * (hc / 4);
+        const int k0 = qq * (hc / 4);
+        double acc0 = 0.0, acc1 = 0.0;
+#pragma unroll 4
+        for (int k = lane; k < hc / 4; k += 32) {
+          const float4 wv = wrow[k];
+          const double2 a = xa[k0 + k];
+          const double2 bb = xb[k0 + k];
+          acc0 = fma(static_cast<double>(wv.x), a.x, acc0);
+          acc1 = fma(static_cast<double>(wv.y), a.y, acc1);
+          acc0 = fma(static_cast<double>(wv.z), bb.x, acc0);
+          acc1 = fma(static_cast<double>(wv.w), bb.y, acc1);
         }
-        acc = warp_sum_d(acc);
+        const double acc = warp_sum_d(acc0 + acc1);
         if (lane == 0) lpart[u] = acc;
       }
     }
-    if (nsh && hdr->abort_flag == 0) gu_consume(&sc, 1, buf);
     __syncthreads();
     return hdr->abort_flag == 0;
   }
 
   // ---------------------------------------------------------------- routing
-  // Warp 0 of every block: logits, top-K (descending, ties to the lower index),
-  // renormalised softmax weights, shared sigmoid gate.
+  // Every block: logits (all threads, one per expert), top-K in two levels -- each
+  // warp selects its K best, warp 0 merges the 16*K candidates -- ordered by logit
+  // descending with ties to the lower index, then the renormalised softmax weights
+  // of the K and the shared sigmoid gate.  Selection uses warp max-reductions on the
+  // order-preserving 64-bit key of each fp64 logit.
+  __device__ __forceinline__ void warp_argmax(unsigned long long bk, int bi, unsigned long long& best, int& win) const {
+    const uint32_t hi = static_cast<uint32_t>(bk >> 32);
+    const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t lo = (hi == mhi) ? static_cast<uint32_t>(bk) : 0u;
+    const uint32_t mlo = __reduce_max_sync(0xffffffffu, lo);
+    best = (static_cast<unsigned long long>(mhi) << 32) | mlo;
+    const uint32_t cand = (bk == best) ? static_cast<uint32_t>(bi) : 0xffffffffu;
+    win = static_cast<int>(__reduce_min_sync(0xffffffffu, cand));
+  }
+
   __device__ void topk(int buf, int t) {
-    if (threadIdx.x < 32) {
-      const int lane = threadIdx.x;
-      const int rows = p.E + (p.has_shared ? 1 : 0);
-      double* slog = reinterpret_cast<double*>(stage);
-      unsigned long long* skey = reinterpret_cast<unsigned long long*>(stage + r128(static_cast<uint32_t>(rows) * 8u));
-      const double* lpart = p.lpart + static_cast<size_t>(buf) * rows * p.nq;
-      for (int e = lane; e < rows; e += 32) {
-        double l = 0.0;
+    mark(3);
+    if (!wait_all(p.rflags, t)) {
+      if (threadIdx.x == 0) hdr->abort_flag = 1;
+      __syncthreads();
+      return;
+    }
+    mark(10);
+    const int rows = p.E + (p.has_shared ? 1 : 0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    double* slog = reinterpret_cast<double*>(stage);
+    unsigned long long* skey = reinterpret_cast<unsigned long long*>(stage + r128(static_cast<uint32_t>(rows) * 8u));
+    unsigned long long* ckey = skey + ((p.E + 15) & ~15);
+    int* cidx = reinterpret_cast<int*>(ckey + kWarps * p.K);
+    const double* lpart = p.lpart + static_cast<size_t>(buf) * rows * p.nq;
+    for (int e = threadIdx.x; e < rows; e += kThreads) {
+      double l = 0.0;
+      if (p.nq == 4) {
+        const double2 a = __ldcg(reinterpret_cast<const double2*>(lpart + static_cast<size_t>(e) * 4));
+        const double2 b = __ldcg(reinterpret_cast<const double2*>(lpart + static_cast<size_t>(e) * 4 + 2));
+        l = ((a.x + a.y) + b.x) + b.y;
+      } else {
         for (int q = 0; q < p.nq; ++q) l += __ldcg(lpart + static_cast<size_t>(e) * p.nq + q);
-        if (e < p.E && p.has_rbias) l += static_cast<double>(p.rbias[e]);
-        slog[e] = l;
-        if (e < p.E) skey[e] = dkey(l);
       }
-      __syncwarp();
-      unsigned long long bk = 0;
-      int bi = 0x7fffffff;
-      for (int e = lane; e < p.E; e += 32)
-        if (skey[e] > bk) {
-          bk = skey[e];
-          bi = e;
+      if (e < p.E && p.has_rbias) l += static_cast<double>(__ldg(p.rbias + e));
+      slog[e] = l;
+      if (e < p.E) skey[e] = dkey(l);
+    }
+    __syncthreads();
+    // level 1: each warp's K best of the experts its threads hold
+    unsigned long long bk = 0;
+    int bi = 0x7fffffff;
+    for (int e = threadIdx.x; e < p.E; e += kThreads)
+      if (skey[e] > bk) {
+        bk = skey[e];
+        bi = e;
+      }
+    for (int k = 0; k < p.K; ++k) {
+      unsigned long long best;
+      int win;
+      warp_argmax(bk, bi, best, win);
+      if (lane == 0) {
+        ckey[warp * p.K + k] = best;
+        cidx[warp * p.K + k] = best ? win : 0x7fffffff;
+      }
+      if (best && win == bi) {
+        skey[win] = 0;
+        bk = 0;
+        bi = 0x7fffffff;
+        for (int e = threadIdx.x; e < p.E; e += kThreads)
+          if (skey[e] > bk) {
+            bk = skey[e];
+            bi = e;
+          }
+      }
+    }
+    mark(11);
+    __syncthreads();
+    mark(12);
+    // level 2: warp 0 merges the candidates
+    if (warp == 0) {
+      const int ncand = kWarps * p.K;
+      bk = 0;
+      bi = 0x7fffffff;
+      int bslot = -1;
+      for (int c = lane; c < ncand; c += 32)
+        if (ckey[c] > bk || (ckey[c] == bk && ckey[c] != 0 && cidx[c] < bi)) {
+          bk = ckey[c];
+          bi = cidx[c];
+          bslot = c;
         }
-      double l0 = 0.0, den = 0.0;
+      int mysel = 0;
       for (int k = 0; k < p.K; ++k) {
-        const uint32_t hi = static_cast<uint32_t>(bk >> 32);
-        const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
-        const uint32_t lo = (hi == mhi) ? static_cast<uint32_t>(bk) : 0u;
-        const uint32_t mlo = __reduce_max_sync(0xffffffffu, lo);
-        const unsigned long long best = (static_cast<unsigned long long>(mhi) << 32) | mlo;
-        const uint32_t cand = (bk == best) ? static_cast<uint32_t>(bi) : 0xffffffffu;
-        const int win = static_cast<int>(__reduce_min_sync(0xffffffffu, cand));
-        const double lw = slog[win];
-        if (k == 0) l0 = lw;
-        den += exp(lw - l0);
-        if (lane == 0) {
-          hdr->sel[k] = win;
-          hdr->wsl[k] = static_cast<float>(lw);  // logit for now, weight below
-        }
-        if ((win & 31) == lane) {
-          skey[win] = 0;
+        unsigned long long best;
+        int win;
+        warp_argmax(bk, bi, best, win);
+        if (lane == k) mysel = win;
+        if (win == bi && bslot >= 0 && bk == best) {
+          ckey[bslot] = 0;
           bk = 0;
           bi = 0x7fffffff;
-          for (int e = lane; e < p.E; e += 32)
-            if (skey[e] > bk) {
-              bk = skey[e];
-              bi = e;
+          bslot = -1;
+          for (int c = lane; c < ncand; c += 32)
+            if (ckey[c] > bk || (ckey[c] == bk && ckey[c] != 0 && cidx[c] < bi)) {
+              bk = ckey[c];
+              bi = cidx[c];
+              bslot = c;
             }
         }
         __syncwarp();
       }
-      if (lane == 0) {
-        for (int k = 0; k < p.K; ++k) {
-          const double wk = exp(slog[hdr->sel[k]] - l0) / den;
-          hdr->wsl[k] = static_cast<float>(wk);
-          if (blockIdx.x == 0 && p.idx_out) {
-            p.idx_out[static_cast<size_t>(t) * p.K + k] = hdr->sel[k];
-            p.w_out[static_cast<size_t>(t) * p.K + k] = static_cast<float>(wk);
-          }
+      mark(13);
+      const int sel0 = __shfl_sync(0xffffffffu, mysel, 0);
+      const double l0 = slog[sel0];
+      const double ek = lane < p.K ? exp(slog[mysel] - l0) : 0.0;
+      const double den = warp_sum_d(ek);
+      if (lane < p.K) {
+        const double wk = ek / den;
+        hdr->sel[lane] = mysel;
+        hdr->wsl[lane] = static_cast<float>(wk);
+        if (blockIdx.x == 0 && p.idx_out) {
+          p.idx_out[static_cast<size_t>(t) * p.K + lane] = mysel;
+          p.w_out[static_cast<size_t>(t) * p.K + lane] = static_cast<float>(wk);
         }
-        if (p.has_shared) {
-          const double sig = 1.0 / (1.0 + exp(-slog[p.E]));
-          hdr->wsl[p.K] = static_cast<float>(sig);
-          if (blockIdx.x == 0 && p.sig_out) p.sig_out[t] = static_cast<float>(sig);
-        }
+      }
+      if (lane == 0 && p.has_shared) {
+        const double sig = 1.0 / (1.0 + exp(-slog[p.E]));
+        hdr->wsl[p.K] = static_cast<float>(sig);
+        if (blockIdx.x == 0 && p.sig_out) p.sig_out[t] = static_cast<float>(sig);
       }
     }
     __syncthreads();
@@ -573,55 +799,63 @@ struct LayerKernel {
     int j0, j1;
     down_range(j0, j1);
     const int ndown = (j1 - j0 + p.db - 1) / p.db;
-    const uint32_t cap = static_cast<uint32_t>(p.staging_bytes);
-    // the block's gate/up chunks, one per slot its unit range touches
+    // plan: routed gate/up chunks from offset 0, down items behind them (issued once
+    // the shared expert's rows at the end of the area are consumed), h at offset 0
     GuChunk ch[kMaxChunks];
     int nc = 0, gitems = 0;
-    uint32_t gbytes = 0;
-    const uint32_t dreg = r128(g.dn_total(j1 - j0));
+    uint32_t gtotal = 0;
     int vend = v0;
     while (vend < v1 && nc < kMaxChunks) {
       const int s = vend / p.I, r = vend % p.I, n = min(v1 - vend, p.I - r);
-      ch[nc++] = GuChunk{s, r, r + n, dreg + gbytes, nitem + static_cast<uint32_t>(gitems)};
+      ch[nc++] = GuChunk{s, r, r + n, gtotal, nitem + static_cast<uint32_t>(gitems)};
       gitems += g.gu_items(n);
-      gbytes += g.gu_bytes(n);
+      gtotal = r128(gtotal + g.gu_bytes(n));
       vend += n;
     }
-    const bool prefetch = (vend >= v1) && (dreg + gbytes <= cap) && (dreg + g.h_bytes() <= cap) &&
-                          (gitems + ndown <= kMaxRoundItems);
+    const uint32_t doff = gtotal, dtotal = g.dn_total(j1 - j0);
+    const uint32_t hoff = g.h_bytes() <= doff ? 0u : r128(doff + dtotal);
+    const bool prefetch = (vend >= v1) && (!has_sc_ || gtotal <= sc_.off) && (doff + dtotal <= cap) &&
+                          (hoff + g.h_bytes() <= cap) && (gitems + ndown <= kMaxRoundItems);
     const uint32_t down_first = nitem + static_cast<uint32_t>(gitems);
     if (prefetch) {
-      // gate/up first in issue order, the down rows behind them
-      if (threadIdx.x == 0) {
-        fence_proxy_async_smem();
-        for (int k = 0; k < nc; ++k) issue_gu(ch[k]);
-      }
-      issue_down_items(j0, j1, 0, ndown, down_first, 0);
-      nitem += static_cast<uint32_t>(gitems + ndown);
+      issue_gu(ch, nc);
+      nitem += static_cast<uint32_t>(gitems);
+      if (has_sc_) gu_consume(&sc_, 1, buf);
+      __syncthreads();
+      issue_down_items(j0, j1, 0, ndown, down_first, doff);
+      nitem += static_cast<uint32_t>(ndown);
       gu_consume(ch, nc, buf);
       __syncthreads();
       if (hdr->abort_flag) return false;
     } else {
-      if (!gu_rounds(0, v0, v1, 0, cap, buf)) return false;
+      if (has_sc_) gu_consume(&sc_, 1, buf);
+      __syncthreads();
+      if (hdr->abort_flag) return false;
+      if (!gu_rounds(v0, v1, buf)) return false;
     }
-    if (!grid_sync()) return false;
+    publish(p.hflags, tok_);
+    mark(5);
     // ---- P3: stage h of every slot, then the down rows
-    const uint32_t hoff = prefetch ? dreg : 0u;
-    float* hs = reinterpret_cast<float*>(stage + hoff);
-    const int nchI = p.I / C::kCols;
+    const uint32_t hbase = prefetch ? hoff : 0u;
+    float* hs = reinterpret_cast<float*>(stage + hbase);
     const uint32_t hstride = g.padded(p.I);
     float* hsum = hs + static_cast<size_t>(nslots) * hstride;
-    const float* hb = p.hbuf + static_cast<size_t>(buf) * (p.K + 1) * p.I;
-    for (int s = 0; s < nslots; ++s)
-      stage_vec(hb + static_cast<size_t>(s) * p.I, nullptr, p.I, hs + static_cast<size_t>(s) * hstride,
-                hsum + static_cast<size_t>(s) * nchI);
+    if (!wait_all(p.hflags, tok_)) {
+      if (threadIdx.x == 0) hdr->abort_flag = 1;
+      __syncthreads();
+      return false;
+    }
+    mark(6);
+    stage_h(p.hbuf + static_cast<size_t>(buf) * (p.K + 1) * p.I, hs, hstride, hsum);
     __syncthreads();
+    mark(7);
     if (prefetch) {
       for (int k = 0; k < ndown; ++k) {
         const int ja = j0 + k * p.db, n = min(j1, ja + p.db) - ja;
-        if (!down_item(down_first + k, k * g.dn_item(p.db), ja, n, hs, hsum, resid_t, y_t)) break;
+        if (!down_item(down_first + k, doff + k * g.dn_item(p.db), ja, n, hs, hsum, resid_t, y_t)) break;
       }
       __syncthreads();
+      mark(8);
     } else {
       const uint32_t dbase = g.h_bytes();
       const int per_round = max(1, min(static_cast<int>((cap - dbase) / g.dn_item(p.db)), kMaxRoundItems));
@@ -650,36 +884,52 @@ struct LayerKernel {
       hdr->abort_flag = 0;
       hdr->skip_token = 0;
       hdr->sel[p.K] = p.E;  // the shared expert's record
+      hdr->tok_base = ld_relaxed_u32(p.tokens);
     }
+    const uint32_t err0 = ld_relaxed_u32(p.err);
     __syncthreads();
-    if (ld_relaxed_u32(p.err) != 0) return;  // sticky error from an earlier call
+    tbase_ = hdr->tok_base;
+    if (err0 != 0) return;  // sticky error from an earlier call
+    const bool route = p.mode != MODE_EXPERTS;
+    const bool do_experts = p.mode != MODE_ROUTE;
     for (int t = 0; t < p.T; ++t) {
       const int buf = t & 1;
-      const uint16_t* x_t = p.x + static_cast<size_t>(t) * p.H;
-      const bool route = p.mode != MODE_EXPERTS;
-      const bool do_experts = p.mode != MODE_ROUTE;
-      // activations: pre-scaled copy for the dequant dots, doubles for the router
-      stage_vec(nullptr, x_t, p.H, xs, xsum);
-      if (route) {
-        double* x64 = reinterpret_cast<double*>(stage);
-        for (int c = threadIdx.x; c < p.H; c += blockDim.x) x64[c] = static_cast<double>(bf16_to_f32(x_t[c]));
-      }
-      __syncthreads();
+      tok_ = t;
+      mark(0);
       if (!route) {
         given_routing(t);
         if (hdr->skip_token) continue;
       }
-      if (!phase1(buf, route, do_experts && p.has_shared)) break;
+      // weight copies first, activations while they fly
+      phase1_issue(route, do_experts && p.has_shared);
+      double2* xa = route ? reinterpret_cast<double2*>(stage) : nullptr;
+      stage_x(p.x + static_cast<size_t>(t) * p.H, xa, xa ? xa + p.H / 4 : nullptr);
+      __syncthreads();
+      mark(1);
+      if (p.hold_cta == static_cast<int>(blockIdx.x)) {  // test hook: never publish anything
+        drain();
+        return;
+      }
+      if (!phase1_consume(buf, route)) break;
+      if (route) publish(p.rflags, t);
+      mark(2);
       if (route) {
-        if (p.hold_cta == static_cast<int>(blockIdx.x)) return;  // test hook: never arrive
-        if (!grid_sync()) break;
         topk(buf, t);
+        if (hdr->abort_flag) break;
+        mark(4);
       }
       if (do_experts) {
         if (!experts(buf, p.resid + static_cast<size_t>(t) * p.H, p.y + static_cast<size_t>(t) * p.H)) break;
+        mark(9);
       }
     }
-    if (hdr->abort_flag) drain();
+    if (hdr->abort_flag) {
+      drain();
+      return;
+    }
+    // the next call's tags continue after this call's tokens (every block has read
+    // the base: block 0 could not have finished without all blocks' values)
+    if (blockIdx.x == 0 && threadIdx.x == 0) st_relaxed_u32(p.tokens, tbase_ + static_cast<uint32_t>(p.T));
   }
 };
 

@@ -24,7 +24,8 @@ DEVERR_BAD_EXPERT = 0x4
 EXPORTS = ["fmoe_record_bytes", "fmoe_workspace_bytes", "fmoe_layer_create", "fmoe_layer_destroy",
            "fmoe_layer_set_workspace", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward",
            "fmoe_rmsnorm", "fmoe_layer_get_error", "fmoe_layer_set_wait_limit",
-           "fmoe_layer_debug_hold_block", "fmoe_layer_grid_size", "fmoe_status_string"]
+           "fmoe_layer_debug_hold_block", "fmoe_layer_debug_timeline", "fmoe_layer_grid_size",
+           "fmoe_status_string"]
 
 
 class FmoeError(RuntimeError):
@@ -69,6 +70,7 @@ def lib():
         L.fmoe_layer_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.fmoe_layer_set_wait_limit.argtypes = [vp, u64]
         L.fmoe_layer_debug_hold_block.argtypes = [vp, i32]
+        L.fmoe_layer_debug_timeline.argtypes = [vp, vp, i32]
         L.fmoe_layer_grid_size.argtypes = [vp]
         L.fmoe_layer_grid_size.restype = i32
         L.fmoe_status_string.argtypes = [i32]
@@ -149,6 +151,10 @@ def fmoe_layer_set_wait_limit(handle, ns: int):
 
 def fmoe_layer_debug_hold_block(handle, cta: int):
     _check(lib().fmoe_layer_debug_hold_block(handle, cta), "fmoe_layer_debug_hold_block")
+
+
+def fmoe_layer_debug_timeline(handle, buf, token: int = 0):
+    _check(lib().fmoe_layer_debug_timeline(handle, _ptr(buf), token), "fmoe_layer_debug_timeline")
 
 
 def fmoe_layer_grid_size(handle) -> int:

@@ -313,12 +313,19 @@ def within_tolerance(gpu: np.ndarray, ref: np.ndarray, rel: float = 2e-3, out_bf
     return bool(np.all(ratio <= 1.0)), float(np.max(ratio)) if ratio.size else 0.0
 
 
-def bf16_agreement(gpu: np.ndarray, ref: np.ndarray):
+def bf16_agreement(gpu: np.ndarray, ref: np.ndarray, min_rel_rms: float = 0.0):
     """(fraction of elements equal to ref rounded to nearest-even bf16,
-    largest distance in bf16 ulps of ref's binade)."""
+    largest distance in bf16 ulps of ref's binade), over the elements with
+    |ref| >= min_rel_rms * rms(ref).  Near-zero outputs are left out with
+    min_rel_rms > 0: an fp32 sum whose terms are of size rms has an absolute
+    rounding error that can exceed the bf16 ulp of a result much smaller than rms."""
     ref = np.asarray(ref, dtype=np.float64)
     gpu = np.asarray(gpu, dtype=np.float64)
+    keep = np.abs(ref) >= min_rel_rms * math.sqrt(float(np.mean(ref * ref)))
+    ref, gpu = ref[keep], gpu[keep]
+    if ref.size == 0:
+        return 1.0, 0.0
     rb = bf16_to_f64(f64_to_bf16_bits(ref))
     ulp = 2.0 * bf16_half_ulp(ref)
     d = np.abs(gpu - rb) / np.where(ulp > 0, ulp, 1.0)
-    return float(np.mean(gpu == rb)), float(np.max(d)) if d.size else 0.0
+    return float(np.mean(gpu == rb)), float(np.max(d))

@@ -5,7 +5,9 @@ relative (fp64 softmax rounded to fp32); layer outputs per element within
 |gpu - oracle| <= 2e-3 * (|oracle| + rms(oracle)) applied before the bf16 output
 rounding (plus bf16's half-ulp), and all but max(2, 1%) of the outputs equal to
 the oracle rounded to nearest-even bf16, none more than one bf16 ulp away (an
-fp32 result within ~1e-6 of a bf16 rounding midpoint may round either way).
+fp32 result within ~1e-6 of a bf16 rounding midpoint may round either way); the
+ulp check covers outputs with |oracle| >= rms/16, where the bf16 ulp exceeds the
+fp32 sum's absolute rounding error.
 """
 import math
 
@@ -52,7 +54,7 @@ def _check_tokens(olay, xg, yg, idxg, wg, sigg, tokens, ctx=""):
         ok, ratio = oracle.within_tolerance(ys[t], r.y)
         worst = max(worst, ratio)
         assert ok, f"{ctx} token {t}: worst error/bound {ratio:.3f}"
-        same, ulps = oracle.bf16_agreement(ys[t], r.y)
+        same, ulps = oracle.bf16_agreement(ys[t], r.y, min_rel_rms=1.0 / 16)
         n_diff = round((1.0 - same) * ys.shape[1])
         assert n_diff <= max(2, 0.01 * ys.shape[1]) and ulps <= 1.0, \
             f"{ctx} token {t}: {n_diff} outputs differ from the rounded oracle, max {ulps} ulps"
