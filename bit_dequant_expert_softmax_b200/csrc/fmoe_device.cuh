@@ -109,14 +109,27 @@ __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
   return v;
 }
 
+// try_wait with a suspend-time hint: the warp is parked by the hardware until the
+// phase completes (or the hint elapses) instead of spinning on the issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for phase `parity` of `bar` to complete, for at most limit_ns.
 __device__ __noinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                                uint32_t* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
     if (global_timer_ns() - t0 > limit_ns) {
       atomicOr(err, FMOE_DEVERR_COPY_TIMEOUT);
       return false;
@@ -124,76 +137,102 @@ __device__ __noinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, u
   }
 }
 
-// ---------------------------------------------------------------- packed f32x2 FMA
-__device__ __forceinline__ void ffma2(float2& acc, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %5};\n\t"
-      "mov.b64 rc, {%0, %1};\n\t"
-      "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
-      "mov.b64 {%0, %1}, rc;\n\t}"
-      : "+f"(acc.x), "+f"(acc.y)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
 // Codes as floats without conversion instructions: a code c masked in place at bit
 // offset s (s + bits <= 24) reads, as an IEEE float, exactly c * 2^s * 2^-149 (a
 // subnormal or the first normal binade).  The activation multiplying it is stored
 // pre-scaled by 2^(kPreExp - s), so every product is code * x * 2^(kPreExp - 149)
 // exactly, and the per-chunk sum is rescaled by 2^(149 - kPreExp) once.
+//
+// Codes are taken in pairs from two adjacent words {w_a, w_b} of a 16-byte load,
+// viewed as one 64-bit register: a 64-bit AND with the same mask in both halves
+// yields, in place, the codes of position p of both words -- exactly the packed
+// operand of one fma.rn.f32x2.  Codes that sit above bit 23 are read from the pair
+// shifted right by 8 (the bits crossing from w_b into w_a's top byte are never
+// selected by the masks).  The activations are laid out so that one 64-bit shared
+// load gives the matching pair {x(word a, p), x(word b, p)}.
 constexpr int kPreExp = 100;
 constexpr float kUnscale = 562949953421312.0f;  // 2^(149 - kPreExp) = 2^49
 
-__device__ __forceinline__ float cf(uint32_t v) { return __uint_as_float(v); }
-
-// One 32-bit word of codes against its pre-scaled activations.
-//  4-bit: columns 8j..8j+7 of the word: xv[0] = cols 0..3, xv[1] = cols 4..7.
-//  2-bit: columns 16j..16j+15: xv[0..3].
-template <int BITS>
-__device__ __forceinline__ void word_fma(uint32_t w, const float4* xv, float2& acc);
-
-template <>
-__device__ __forceinline__ void word_fma<4>(uint32_t w, const float4* xv, float2& acc) {
-  const uint32_t h = w >> 16;
-  ffma2(acc, cf(w & 0xFu), cf(w & 0xF0u), xv[0].x, xv[0].y);
-  ffma2(acc, cf(w & 0xF00u), cf(w & 0xF000u), xv[0].z, xv[0].w);
-  ffma2(acc, cf(h & 0xFu), cf(h & 0xF0u), xv[1].x, xv[1].y);
-  ffma2(acc, cf(h & 0xF00u), cf(h & 0xF000u), xv[1].z, xv[1].w);
+__device__ __forceinline__ void fma2(unsigned long long& acc, unsigned long long c, unsigned long long x) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(c), "l"(x));
 }
 
-template <>
-__device__ __forceinline__ void word_fma<2>(uint32_t w, const float4* xv, float2& acc) {
-  const uint32_t h = w >> 16;
-  ffma2(acc, cf(w & 0x3u), cf(w & 0xCu), xv[0].x, xv[0].y);
-  ffma2(acc, cf(w & 0x30u), cf(w & 0xC0u), xv[0].z, xv[0].w);
-  ffma2(acc, cf(w & 0x300u), cf(w & 0xC00u), xv[1].x, xv[1].y);
-  ffma2(acc, cf(w & 0x3000u), cf(w & 0xC000u), xv[1].z, xv[1].w);
-  ffma2(acc, cf(h & 0x3u), cf(h & 0xCu), xv[2].x, xv[2].y);
-  ffma2(acc, cf(h & 0x30u), cf(h & 0xC0u), xv[2].z, xv[2].w);
-  ffma2(acc, cf(h & 0x300u), cf(h & 0xC00u), xv[3].x, xv[3].y);
-  ffma2(acc, cf(h & 0x3000u), cf(h & 0xC000u), xv[3].z, xv[3].w);
+__device__ __forceinline__ float pair_sum(unsigned long long a) {
+  return __uint_as_float(static_cast<uint32_t>(a)) + __uint_as_float(static_cast<uint32_t>(a >> 32));
 }
 
-// Chunk geometry: one chunk = 16 bytes of codes = 4 words.
+// Chunk geometry: one chunk = 16 bytes of codes = 4 words = 2 word pairs.
 template <int BITS>
 struct Chunk {
-  static constexpr int kCols = 128 / BITS;        // 32 (4-bit) or 64 (2-bit) columns
-  static constexpr int kF4 = kCols / 4;           // float4 per chunk
-  static constexpr int kF4PerWord = kF4 / 4;      // 2 or 4
-  static constexpr int kGroupsPerChunkLog = 0;
-  // shift applied to column c inside its word (where its code is masked)
-  __device__ __forceinline__ static int shift_of(int c) { return BITS == 4 ? 4 * (c & 3) : 2 * (c & 7); }
-  // index (in floats) of column c in the lane-interleaved activation layout:
-  // chunk m, float4 f of the chunk, lane slot m % 32 -> conflict-free LDS.128
-  __device__ __forceinline__ static int phys(int c) {
-    const int m = c / kCols, f = (c % kCols) >> 2, e = c & 3;
-    return ((((m >> 5) * kF4 + f) << 5) + (m & 31)) * 4 + e;
+  static constexpr int kCols = 128 / BITS;    // 32 (4-bit) or 64 (2-bit) columns
+  static constexpr int kWC = 32 / BITS;       // codes per word: 8 or 16
+  static constexpr int kF4 = kCols / 4;       // float4 of activations per chunk: 8 or 16
+  static constexpr int kF4PerPair = kWC / 2;  // float4 per word pair: 4 or 8
+  // bit offset at which position p of a word is masked (after the 8-bit shift when
+  // the code lies above bit 23)
+  __host__ __device__ static constexpr int shift_pos(int p) {
+    return BITS * p + BITS > 24 ? BITS * p - 8 : BITS * p;
   }
-  __device__ __forceinline__ static const float4* f4(const float* base, int m, int f) {
-    return reinterpret_cast<const float4*>(base) + ((((m >> 5) * kF4 + f) << 5) + (m & 31));
+  __device__ __forceinline__ static int shift_of(int c) { return shift_pos(c % kWC); }
+  // float4 k of a chunk holds, for a = 2*(k / kF4PerPair), kk = k % kF4PerPair:
+  // (word a, pos 2kk), (word a+1, pos 2kk), (word a, pos 2kk+1), (word a+1, pos 2kk+1)
+  // lane-interleaved layout: float4 k of chunk m at slot ((m/32)*kF4 + k)*32 + m%32,
+  // so a warp's lanes (consecutive chunks) read consecutive 16-byte slots
+  __device__ __forceinline__ static const ulonglong2* f4(const float* base, int m, int k) {
+    return reinterpret_cast<const ulonglong2*>(base) + ((((m >> 5) * kF4 + k) << 5) + (m & 31));
   }
   // (scale,bias) word index of chunk m within its row
   __device__ __forceinline__ static int sb_index(int m) { return BITS == 4 ? (m >> 1) : m; }
+
+  // One word pair W = {w_a, w_b} against its activation pairs (kF4PerPair float4 at
+  // xv[0], xv[32], ... in the interleaved layout), accumulated into acc.
+  template <int P>
+  __device__ __forceinline__ static void pos(unsigned long long W, unsigned long long V, unsigned long long x,
+                                             unsigned long long& acc) {
+    constexpr int s = shift_pos(P);
+    constexpr uint32_t m32 = ((1u << BITS) - 1u) << s;
+#ifdef FMOE_SCALAR_FMA
+    const unsigned long long src = (BITS * P + BITS > 24) ? V : W;
+    float lo = __uint_as_float(static_cast<uint32_t>(acc)), hi = __uint_as_float(static_cast<uint32_t>(acc >> 32));
+    lo = fmaf(__uint_as_float(static_cast<uint32_t>(src) & m32), __uint_as_float(static_cast<uint32_t>(x)), lo);
+    hi = fmaf(__uint_as_float(static_cast<uint32_t>(src >> 32) & m32), __uint_as_float(static_cast<uint32_t>(x >> 32)), hi);
+    acc = (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+#else
+    constexpr unsigned long long mask = (static_cast<unsigned long long>(m32) << 32) | m32;
+    fma2(acc, ((BITS * P + BITS > 24) ? V : W) & mask, x);
+#endif
+  }
+  // Word pairs of one or two rows against shared activation pairs.
+  template <bool TWO>
+  __device__ __forceinline__ static void word_pair2(unsigned long long Wa, unsigned long long Wb,
+                                                    const ulonglong2* xv, unsigned long long& acc_a,
+                                                    unsigned long long& acc_b) {
+    const unsigned long long Va = Wa >> 8;
+    const unsigned long long Vb = TWO ? (Wb >> 8) : 0ull;
+#pragma unroll
+    for (int k = 0; k < kF4PerPair; ++k) {
+      const ulonglong2 x = xv[k * 32];
+      // positions 2k (x.x) and 2k+1 (x.y)
+      switch (k) {
+#define FMOE_POS_CASE(K)                                  \
+  case K:                                                 \
+    pos<2 * K>(Wa, Va, x.x, acc_a);                       \
+    pos<2 * K + 1>(Wa, Va, x.y, acc_a);                   \
+    if (TWO) pos<2 * K>(Wb, Vb, x.x, acc_b);              \
+    if (TWO) pos<2 * K + 1>(Wb, Vb, x.y, acc_b);          \
+    break;
+        FMOE_POS_CASE(0)
+        FMOE_POS_CASE(1)
+        FMOE_POS_CASE(2)
+        FMOE_POS_CASE(3)
+        FMOE_POS_CASE(4)
+        FMOE_POS_CASE(5)
+        FMOE_POS_CASE(6)
+        FMOE_POS_CASE(7)
+#undef FMOE_POS_CASE
+      }
+    }
+  }
 };
 
 __device__ __forceinline__ float prescale_factor(int shift) {

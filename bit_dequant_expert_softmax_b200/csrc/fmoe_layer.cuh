@@ -163,8 +163,10 @@ struct LayerKernel {
 
   // diagnostic timestamps (token 0 only; off unless a timeline buffer is attached)
   __device__ __forceinline__ void mark(int i) const {
-    if (p.timeline != nullptr && tok_ == p.timeline_token && threadIdx.x == 0)
-      p.timeline[static_cast<size_t>(blockIdx.x) * 16 + i] = global_timer_ns();
+    if (p.timeline != nullptr && tok_ == p.timeline_token && threadIdx.x == 0) {
+      p.timeline[static_cast<size_t>(blockIdx.x) * 32 + i] = global_timer_ns();
+      p.timeline[static_cast<size_t>(blockIdx.x) * 32 + 16 + i] = static_cast<unsigned long long>(clock64());
+    }
   }
 
   // Waits (bounded) for every copy this block may still have in flight.
@@ -223,6 +225,7 @@ struct LayerKernel {
             break;
           }
         }
+        __nanosleep(32);
 #pragma unroll
         for (int i = 0; i < NF; ++i) {
           const int b = lane + 32 * i;
@@ -241,17 +244,6 @@ struct LayerKernel {
   //    arrays so the router's loads are conflict-free);
   //  transposed (thread -> consecutive float4 slots of the lane-interleaved layout):
   //    pre-scaled floats, conflict-free 16-byte stores.
-  __device__ __forceinline__ float4 prescale4(float4 v, int c0) const {
-    return make_float4(v.x * prescale_factor(C::shift_of(c0)), v.y * prescale_factor(C::shift_of(c0 + 1)),
-                       v.z * prescale_factor(C::shift_of(c0 + 2)), v.w * prescale_factor(C::shift_of(c0 + 3)));
-  }
-  // column of the first element of float4 slot `idx` of the interleaved layout (-1: padding)
-  __device__ __forceinline__ int slot_col(int idx, int nch) const {
-    const int lane_m = idx & 31, f = (idx >> 5) % C::kF4, hi = (idx >> 5) / C::kF4;
-    const int m = hi * 32 + lane_m;
-    return m < nch ? m * C::kCols + 4 * f : -1;
-  }
-
   __device__ __forceinline__ float4 bf16x4(uint2 u) const {
     return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
                        __uint_as_float(u.y & 0xFFFF0000u));
@@ -259,18 +251,14 @@ struct LayerKernel {
 
   __device__ void stage_x(const uint16_t* xt, double2* xa, double2* xb) {
     constexpr int TPC = C::kCols / 4;
-    const int n4 = p.H / 4, nch = p.H / C::kCols;
-    const int F = static_cast<int>(g.padded(p.H) / 4);
+    const int n4 = p.H / 4;
     const uint2* src = reinterpret_cast<const uint2*>(xt);
-    for (int base = 0; base < max(n4, F); base += 2 * kThreads) {
-      uint2 nat[2], tr[2];
-      int trc[2];
+    for (int base = 0; base < n4; base += 2 * kThreads) {  // block-uniform trip count
+      uint2 nat[2];
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
         nat[k] = q < n4 ? src[q] : make_uint2(0, 0);
-        trc[k] = q < F ? slot_col(q, nch) : -1;
-        tr[k] = trc[k] >= 0 ? src[trc[k] / 4] : make_uint2(0, 0);
       }
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
@@ -284,81 +272,89 @@ struct LayerKernel {
             xa[q] = make_double2(v.x, v.y);
             xb[q] = make_double2(v.z, v.w);
           }
+          const int c0 = 4 * q;
+          xs[phys(c0 + 0)] = v.x * prescale_factor(C::shift_of(c0 + 0));
+          xs[phys(c0 + 1)] = v.y * prescale_factor(C::shift_of(c0 + 1));
+          xs[phys(c0 + 2)] = v.z * prescale_factor(C::shift_of(c0 + 2));
+          xs[phys(c0 + 3)] = v.w * prescale_factor(C::shift_of(c0 + 3));
           if (q % TPC == 0) xsum[q / TPC] = sum;
-        }
-        if (q < F) {
-          const float4 w = trc[k] >= 0 ? prescale4(bf16x4(tr[k]), trc[k]) : make_float4(0.f, 0.f, 0.f, 0.f);
-          reinterpret_cast<float4*>(xs)[q] = w;
         }
       }
     }
   }
 
   // h of every slot (fp32, written by other blocks, read from L2 once every block
-  // has published): natural pass for the chunk sums, transposed pass for the
-  // conflict-free stores; all loads of a thread in flight together.
+  // has published): coalesced 16-byte loads (thread -> 4 consecutive columns), all of
+  // a thread's loads in flight together; chunk sums by shuffles over the kCols/4
+  // threads of a chunk; pre-scaled values scattered into the interleaved layout.
   __device__ void stage_h(const float* hb, float* hs, uint32_t hstride, float* hsum) {
     constexpr int TPC = C::kCols / 4;
     const int per_slot = p.I / 4, nch = p.I / C::kCols;
     const int n4 = nslots * per_slot;
-    const int F1 = static_cast<int>(hstride / 4), F = nslots * F1;
     const float4* src = reinterpret_cast<const float4*>(hb);
-    for (int base = 0; base < max(n4, F); base += 2 * kThreads) {
-      float4 nat[2], tr[2];
-      int trc[2];
+    for (int base = 0; base < n4; base += 4 * kThreads) {
+      float4 v[4];
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
+      for (int k = 0; k < 4; ++k) {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
-        nat[k] = q < n4 ? __ldcg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-        trc[k] = q < F ? slot_col(q % F1, nch) : -1;
-        tr[k] = trc[k] >= 0 ? __ldcg(src + (q / F1) * per_slot + trc[k] / 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[k] = q < n4 ? __ldcg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
+      for (int k = 0; k < 4; ++k) {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
-        float sum = (nat[k].x + nat[k].y) + (nat[k].z + nat[k].w);
+        float sum = (v[k].x + v[k].y) + (v[k].z + v[k].w);
 #pragma unroll
         for (int o = 1; o < TPC; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (q < n4 && q % TPC == 0) hsum[(q / per_slot) * nch + (q % per_slot) / TPC] = sum;
-        if (q < F) {
-          const float4 w = trc[k] >= 0 ? prescale4(tr[k], trc[k]) : make_float4(0.f, 0.f, 0.f, 0.f);
-          reinterpret_cast<float4*>(hs)[(q / F1) * (hstride / 4) + q % F1] = w;
+        if (q < n4) {
+          const int slot = q / per_slot, c0 = (q % per_slot) * 4;
+          float* d = hs + static_cast<size_t>(slot) * hstride;
+          d[phys(c0 + 0)] = v[k].x * prescale_factor(C::shift_of(c0 + 0));
+          d[phys(c0 + 1)] = v[k].y * prescale_factor(C::shift_of(c0 + 1));
+          d[phys(c0 + 2)] = v[k].z * prescale_factor(C::shift_of(c0 + 2));
+          d[phys(c0 + 3)] = v[k].w * prescale_factor(C::shift_of(c0 + 3));
+          if (q % TPC == 0) hsum[slot * nch + c0 / C::kCols] = sum;
         }
       }
+      if (base == 0) mark(14);
     }
+    mark(15);
+  }
+
+  // float index of column c in the lane-interleaved layout
+  __device__ __forceinline__ static int phys(int c) {
+    const int m = c / C::kCols, r = c % C::kCols;
+    const int word = r / C::kWC, pos = r % C::kWC;
+    // float4 k: word pair a = word & ~1, kk = pos / 2; element (pos & 1) * 2 + (word & 1)
+    const int k = (word >> 1) * C::kF4PerPair + (pos >> 1);
+    const int e = ((pos & 1) << 1) | (word & 1);
+    return ((((m >> 5) * C::kF4 + k) << 5) + (m & 31)) * 4 + e;
   }
 
   // ---------------------------------------------------------------- dot products
-  // Lane partial of sum_c W[r][c] v[c] over the lane's chunks, for up to two rows
+  // Lane partial of sum_c W[r][c] v[c] over the lane's chunks, for one or two rows
   // sharing the activation loads (W = scale*code + bias; v pre-scaled, interleaved).
-  // Two accumulator pairs per row halve the dependent FMA chains.
-  __device__ __forceinline__ void dot2(const uint8_t* q0, const uint32_t* s0, const uint8_t* q1,
-                                       const uint32_t* s1, bool two, const float* vs, const float* vsum,
-                                       int nch, float& r0, float& r1) const {
+  template <bool TWO>
+  __device__ __forceinline__ void dotn(const uint8_t* q0, const uint32_t* s0, const uint8_t* q1,
+                                       const uint32_t* s1, const float* vs, const float* vsum, int nch, float& r0,
+                                       float& r1) const {
     const int lane = threadIdx.x & 31;
 #pragma unroll 2
     for (int m = lane; m < nch; m += 32) {
-      const uint4 a4 = *reinterpret_cast<const uint4*>(q0 + 16 * m);
-      uint4 b4 = make_uint4(0, 0, 0, 0);
-      if (two) b4 = *reinterpret_cast<const uint4*>(q1 + 16 * m);
-      const uint32_t wa[4] = {a4.x, a4.y, a4.z, a4.w};
-      const uint32_t wb[4] = {b4.x, b4.y, b4.z, b4.w};
-      float2 aa0 = make_float2(0.f, 0.f), aa1 = aa0, ab0 = aa0, ab1 = aa0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float4 xv[C::kF4PerWord];
-#pragma unroll
-        for (int f = 0; f < C::kF4PerWord; ++f) xv[f] = *C::f4(vs, m, j * C::kF4PerWord + f);
-        word_fma<BITS>(wa[j], xv, j < 2 ? aa0 : aa1);
-        if (two) word_fma<BITS>(wb[j], xv, j < 2 ? ab0 : ab1);
-      }
+      const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(q0 + 16 * m);
+      ulonglong2 b = make_ulonglong2(0ull, 0ull);
+      if (TWO) b = *reinterpret_cast<const ulonglong2*>(q1 + 16 * m);
+      const ulonglong2* xv0 = C::f4(vs, m, 0);
+      const ulonglong2* xv1 = C::f4(vs, m, C::kF4PerPair);
+      unsigned long long a0 = 0ull, a1 = 0ull, b0 = 0ull, b1 = 0ull;
+      C::template word_pair2<TWO>(a.x, b.x, xv0, a0, b0);
+      C::template word_pair2<TWO>(a.y, b.y, xv1, a1, b1);
       const float vm = vsum[m];
       const uint32_t sa = s0[C::sb_index(m)];
-      r0 = fmaf(sb_scale(sa), ((aa0.x + aa0.y) + (aa1.x + aa1.y)) * kUnscale, r0);
+      r0 = fmaf(sb_scale(sa), (pair_sum(a0) + pair_sum(a1)) * kUnscale, r0);
       r0 = fmaf(sb_bias(sa), vm, r0);
-      if (two) {
+      if (TWO) {
         const uint32_t sbv = s1[C::sb_index(m)];
-        r1 = fmaf(sb_scale(sbv), ((ab0.x + ab0.y) + (ab1.x + ab1.y)) * kUnscale, r1);
+        r1 = fmaf(sb_scale(sbv), (pair_sum(b0) + pair_sum(b1)) * kUnscale, r1);
         r1 = fmaf(sb_bias(sbv), vm, r1);
       }
     }
@@ -413,7 +409,7 @@ struct LayerKernel {
     const uint32_t* sg = reinterpret_cast<const uint32_t*>(stage + c.off + g.gu_q(n) + lead) + i * 2 * (p.sh / 4);
     const uint32_t* su = sg + p.sh / 4;
     float gv = 0.f, uv = 0.f;
-    dot2(qg, sg, qu, su, true, xs, xsum, p.H / C::kCols, gv, uv);
+    dotn<true>(qg, sg, qu, su, xs, xsum, p.H / C::kCols, gv, uv);
     gv = warp_sum(gv);
     uv = warp_sum(uv);
     if ((threadIdx.x & 31) == 0) {
@@ -538,9 +534,14 @@ struct LayerKernel {
       const uint8_t* blk = stage + off + s * g.dn_slot(n);
       const uint32_t* sbase = reinterpret_cast<const uint32_t*>(blk + g.dn_q(n) + lead);
       float oa = 0.f, ob = 0.f;
-      dot2(blk + static_cast<uint32_t>(ia) * p.qi, sbase + ia * (p.si / 4), blk + static_cast<uint32_t>(ib) * p.qi,
-           sbase + ib * (p.si / 4), two, hs + static_cast<size_t>(s) * g.padded(p.I),
-           hsum + static_cast<size_t>(s) * nch, nch, oa, ob);
+      const float* hsl = hs + static_cast<size_t>(s) * g.padded(p.I);
+      const float* hsm = hsum + static_cast<size_t>(s) * nch;
+      if (two)
+        dotn<true>(blk + static_cast<uint32_t>(ia) * p.qi, sbase + ia * (p.si / 4),
+                   blk + static_cast<uint32_t>(ib) * p.qi, sbase + ib * (p.si / 4), hsl, hsm, nch, oa, ob);
+      else
+        dotn<false>(blk + static_cast<uint32_t>(ia) * p.qi, sbase + ia * (p.si / 4), nullptr, nullptr, hsl, hsm,
+                    nch, oa, ob);
       const float ws = hdr->wsl[s];
       pa = fmaf(ws, oa, pa);
       pb = fmaf(ws, ob, pb);

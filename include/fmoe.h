@@ -163,12 +163,13 @@ fmoe_status fmoe_layer_set_wait_limit(fmoe_layer_t layer, uint64_t nanoseconds);
  * runs out and FMOE_DEVERR_BARRIER_TIMEOUT is set.  -1 (default) disables it. */
 fmoe_status fmoe_layer_debug_hold_block(fmoe_layer_t layer, int cta);
 
-/* Diagnostic hook: when dev_buf != NULL (a device buffer of fmoe_layer_grid_size() * 16
- * uint64), every block of the following forward calls writes %globaltimer timestamps
- * (ns) of its phase boundaries while it processes token `token` of a call, to
- * dev_buf[block*16 + i]: 0 start, 1 activations staged, 2 router rows done, 4 top-K
- * done, 5 gate/up done, 7 h staged, 8 down rows done, 9 token done, 10 router
- * logits gathered.  NULL (default) disables it. */
+/* Diagnostic hook: when dev_buf != NULL (a device buffer of fmoe_layer_grid_size() * 32
+ * uint64), every block of the following forward calls records its phase boundaries
+ * while it processes token `token` of a call: %globaltimer (ns) in dev_buf[block*32 + i]
+ * and the SM clock counter in dev_buf[block*32 + 16 + i], for i = 0 start, 1 activations
+ * staged, 2 router rows done, 3 top-K start, 4 top-K done, 5 gate/up done, 6 h rows of
+ * all blocks visible, 7 h staged, 8 down rows done, 9 token done, 10 router logits of
+ * all blocks visible, 11..13 top-K steps.  NULL (default) disables it. */
 fmoe_status fmoe_layer_debug_timeline(fmoe_layer_t layer, uint64_t* dev_buf, int token);
 
 /* Number of thread blocks one forward launch uses (one per SM of the device). */
