@@ -132,7 +132,7 @@ fmoe_status plan(fmoe_layer* L) {
   if (p1 > sc_off || p1_items > (uint32_t)kMaxRoundItems) return FMOE_ERR_UNSUPPORTED;
   // top-K: logits, selection keys, per-warp candidates
   if ((uint64_t)r128((uint32_t)(c.n_experts + 1) * 8u) + (uint64_t)((c.n_experts + 15) & ~15) * 8u +
-          (uint64_t)kWarps * c.top_k * 12u >
+          (uint64_t)((c.n_experts + 31) / 32) * c.top_k * 12u >
       sc_off)
     return FMOE_ERR_UNSUPPORTED;
   // P2: at least one gate/up row pair per round

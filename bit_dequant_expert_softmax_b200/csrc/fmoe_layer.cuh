@@ -646,21 +646,11 @@ struct LayerKernel {
   }
 
   // ---------------------------------------------------------------- routing
-  // Every block: logits (all threads, one per expert), top-K in two levels -- each
-  // warp selects its K best, warp 0 merges the 16*K candidates -- ordered by logit
-  // descending with ties to the lower index, then the renormalised softmax weights
-  // of the K and the shared sigmoid gate.  Selection uses warp max-reductions on the
-  // order-preserving 64-bit key of each fp64 logit.
-  __device__ __forceinline__ void warp_argmax(unsigned long long bk, int bi, unsigned long long& best, int& win) const {
-    const uint32_t hi = static_cast<uint32_t>(bk >> 32);
-    const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
-    const uint32_t lo = (hi == mhi) ? static_cast<uint32_t>(bk) : 0u;
-    const uint32_t mlo = __reduce_max_sync(0xffffffffu, lo);
-    best = (static_cast<unsigned long long>(mhi) << 32) | mlo;
-    const uint32_t cand = (bk == best) ? static_cast<uint32_t>(bi) : 0xffffffffu;
-    win = static_cast<int>(__reduce_min_sync(0xffffffffu, cand));
-  }
-
+  // Every block: logits (all threads, one per expert), top-K by ranks in two levels
+  // -- within groups of 32 experts, then among the groups' K best -- ordered by logit
+  // descending with ties to the lower index (compared through the order-preserving
+  // 64-bit key of each fp64 logit), then the renormalised softmax weights of the K
+  // and the shared sigmoid gate.
   __device__ void topk(int buf, int t) {
     mark(3);
     if (!wait_all(p.rflags, t)) {
@@ -674,7 +664,7 @@ struct LayerKernel {
     double* slog = reinterpret_cast<double*>(stage);
     unsigned long long* skey = reinterpret_cast<unsigned long long*>(stage + r128(static_cast<uint32_t>(rows) * 8u));
     unsigned long long* ckey = skey + ((p.E + 15) & ~15);
-    int* cidx = reinterpret_cast<int*>(ckey + kWarps * p.K);
+    int* cidx = reinterpret_cast<int*>(ckey + ((p.E + 31) >> 5) * p.K);
     const double* lpart = p.lpart + static_cast<size_t>(buf) * rows * p.nq;
     for (int e = threadIdx.x; e < rows; e += kThreads) {
       double l = 0.0;
@@ -690,76 +680,69 @@ struct LayerKernel {
       if (e < p.E) skey[e] = dkey(l);
     }
     __syncthreads();
-    // level 1: each warp's K best of the experts its threads hold
-    unsigned long long bk = 0;
-    int bi = 0x7fffffff;
-    for (int e = threadIdx.x; e < p.E; e += kThreads)
-      if (skey[e] > bk) {
-        bk = skey[e];
-        bi = e;
+    // level 1: each expert's rank among the experts of its warp's slice (the 32
+    // consecutive experts [32w + 512j, ...) for j = 0, 1, ...): keys are read back
+    // with broadcast shared loads, ties ordered by the lower index; the warp's K best
+    // become candidates, each written to the slot of its rank.
+    for (int e = threadIdx.x; e < p.E; e += kThreads) {
+      const unsigned long long ke = skey[e];
+      const int b0 = e & ~31;
+      const int nb = min(32, p.E - b0);
+      int rank = 0;
+      if (nb == 32) {
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+          const unsigned long long kj = skey[b0 + j];
+          rank += static_cast<int>(kj > ke) | (static_cast<int>(kj == ke) & static_cast<int>(b0 + j < e));
+        }
+      } else {
+        for (int j = 0; j < nb; ++j) {
+          const unsigned long long kj = skey[b0 + j];
+          rank += static_cast<int>(kj > ke) | (static_cast<int>(kj == ke) & static_cast<int>(b0 + j < e));
+        }
       }
-    for (int k = 0; k < p.K; ++k) {
-      unsigned long long best;
-      int win;
-      warp_argmax(bk, bi, best, win);
-      if (lane == 0) {
-        ckey[warp * p.K + k] = best;
-        cidx[warp * p.K + k] = best ? win : 0x7fffffff;
+      if (rank < p.K) {
+        const int slot = (e >> 5) * p.K + rank;
+        ckey[slot] = ke;
+        cidx[slot] = e;
       }
-      if (best && win == bi) {
-        skey[win] = 0;
-        bk = 0;
-        bi = 0x7fffffff;
-        for (int e = threadIdx.x; e < p.E; e += kThreads)
-          if (skey[e] > bk) {
-            bk = skey[e];
-            bi = e;
-          }
+    }
+    const int ngroups = (p.E + 31) >> 5;
+    for (int c = threadIdx.x; c < ngroups * p.K; c += kThreads) {
+      const int gsz = min(32, p.E - (c / p.K) * 32);
+      if (c % p.K >= gsz) {  // a short last group has fewer than K members
+        ckey[c] = 0;
+        cidx[c] = 0x7fffffff;
       }
     }
     mark(11);
     __syncthreads();
     mark(12);
-    // level 2: warp 0 merges the candidates
-    if (warp == 0) {
-      const int ncand = kWarps * p.K;
-      bk = 0;
-      bi = 0x7fffffff;
-      int bslot = -1;
-      for (int c = lane; c < ncand; c += 32)
-        if (ckey[c] > bk || (ckey[c] == bk && ckey[c] != 0 && cidx[c] < bi)) {
-          bk = ckey[c];
-          bi = cidx[c];
-          bslot = c;
-        }
-      int mysel = 0;
-      for (int k = 0; k < p.K; ++k) {
-        unsigned long long best;
-        int win;
-        warp_argmax(bk, bi, best, win);
-        if (lane == k) mysel = win;
-        if (win == bi && bslot >= 0 && bk == best) {
-          ckey[bslot] = 0;
-          bk = 0;
-          bi = 0x7fffffff;
-          bslot = -1;
-          for (int c = lane; c < ncand; c += 32)
-            if (ckey[c] > bk || (ckey[c] == bk && ckey[c] != 0 && cidx[c] < bi)) {
-              bk = ckey[c];
-              bi = cidx[c];
-              bslot = c;
-            }
-        }
-        __syncwarp();
+    // level 2: every candidate's rank among all candidates; the K best are the
+    // selection, in order
+    const int ncand = ngroups * p.K;
+    for (int c = threadIdx.x; c < ncand; c += kThreads) {
+      const unsigned long long kc = ckey[c];
+      const int ic = cidx[c];
+      if (kc == 0) continue;
+      int rank = 0;
+#pragma unroll 8
+      for (int j = 0; j < ncand; ++j) {
+        const unsigned long long kj = ckey[j];
+        const int ij = cidx[j];
+        rank += static_cast<int>(kj > kc) | (static_cast<int>(kj == kc) & static_cast<int>(ij < ic));
       }
-      mark(13);
-      const int sel0 = __shfl_sync(0xffffffffu, mysel, 0);
-      const double l0 = slog[sel0];
+      if (rank < p.K) hdr->sel[rank] = ic;
+    }
+    __syncthreads();
+    mark(13);
+    if (warp == 0) {
+      const int mysel = lane < p.K ? hdr->sel[lane] : hdr->sel[0];
+      const double l0 = slog[hdr->sel[0]];
       const double ek = lane < p.K ? exp(slog[mysel] - l0) : 0.0;
       const double den = warp_sum_d(ek);
       if (lane < p.K) {
         const double wk = ek / den;
-        hdr->sel[lane] = mysel;
         hdr->wsl[lane] = static_cast<float>(wk);
         if (blockIdx.x == 0 && p.idx_out) {
           p.idx_out[static_cast<size_t>(t) * p.K + lane] = mysel;
