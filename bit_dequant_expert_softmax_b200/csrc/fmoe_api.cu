@@ -3,6 +3,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include <cuda_runtime.h>
@@ -397,8 +398,75 @@ const char* fmoe_status_string(fmoe_status s) {
     case FMOE_ERR_CUDA: return "CUDA error";
     case FMOE_ERR_NO_WORKSPACE: return "workspace missing or too small";
     case FMOE_ERR_DEVICE: return "device-side error";
+    case FMOE_ERR_SCRATCH_LIMIT:
+      return "the layer needs more scratch than fmoe_layer_forward_noalloc's fixed array (FMOE_NOALLOC_SCRATCH_BYTES)";
   }
   return "unknown status";
+}
+
+// ---------------------------------------------------------------------------
+// fmoe_layer_forward_noalloc: the same fused kernel with its scratch in a fixed
+// file-scope device array instead of a caller-provided workspace.
+}  // extern "C"
+
+namespace {
+
+__device__ __align__(256) uint8_t g_noalloc_scratch[FMOE_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the array on device `dev` (current); looked up once per device.
+// In host code the array's name is only a host-side handle, never a device address.
+fmoe_status noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (dev < 0 || dev >= kMaxDevices) return FMOE_ERR_UNSUPPORTED;
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FMOE_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FMOE_OK;
+}
+
+void set_workspace_ptrs(Params& p, const WsLayout& w, uint8_t* ws) {
+  p.err = reinterpret_cast<uint32_t*>(ws + w.err);
+  p.tokens = reinterpret_cast<uint32_t*>(ws + w.tokens);
+  p.rflags = reinterpret_cast<uint32_t*>(ws + w.rflags);
+  p.hflags = reinterpret_cast<uint32_t*>(ws + w.hflags);
+  p.lpart = reinterpret_cast<double*>(ws + w.lpart);
+  p.hbuf = reinterpret_cast<float*>(ws + w.hbuf);
+}
+
+}  // namespace
+
+extern "C" {
+
+fmoe_status fmoe_layer_forward_noalloc(fmoe_layer_t L, const uint16_t* x, const uint16_t* resid, int T, uint16_t* y,
+                                       void* stream) {
+  if (!L || T < 0) return FMOE_ERR_INVALID_ARG;
+  if (T == 0) return FMOE_OK;
+  if (!x || !resid || !y || !aligned(x, 16) || !aligned(resid, 16) || !aligned(y, 16) || y == x)
+    return FMOE_ERR_INVALID_ARG;
+  if (L->wsl.size > (size_t)FMOE_NOALLOC_SCRATCH_BYTES) return FMOE_ERR_SCRATCH_LIMIT;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FMOE_ERR_CUDA;
+  if (dev != L->device) return FMOE_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  fmoe_status st = noalloc_scratch(dev, &scratch);
+  if (st != FMOE_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  // every call starts from a clean error word, tag base and flags (the values the
+  // previous call left there would otherwise be mistaken for this call's)
+  if (cudaMemsetAsync(ws, 0, L->wsl.lpart, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FMOE_ERR_CUDA;
+  Params p = base_params(L, MODE_FULL, T);
+  set_workspace_ptrs(p, L->wsl, ws);
+  p.x = x;
+  p.resid = resid;
+  p.y = y;
+  return launch(L, p, stream);
 }
 
 }  // extern "C"

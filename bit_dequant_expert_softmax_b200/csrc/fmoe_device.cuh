@@ -189,19 +189,14 @@ struct Chunk {
   template <int P>
   __device__ __forceinline__ static void pos(unsigned long long W, unsigned long long V, unsigned long long x,
                                              unsigned long long& acc) {
-    constexpr int s = shift_pos(P);
-    constexpr uint32_t m32 = ((1u << BITS) - 1u) << s;
-#ifdef FMOE_SCALAR_FMA
-    const unsigned long long src = (BITS * P + BITS > 24) ? V : W;
-    float lo = __uint_as_float(static_cast<uint32_t>(acc)), hi = __uint_as_float(static_cast<uint32_t>(acc >> 32));
-    lo = fmaf(__uint_as_float(static_cast<uint32_t>(src) & m32), __uint_as_float(static_cast<uint32_t>(x)), lo);
-    hi = fmaf(__uint_as_float(static_cast<uint32_t>(src >> 32) & m32), __uint_as_float(static_cast<uint32_t>(x >> 32)), hi);
-    acc = (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
-#else
-    constexpr unsigned long long mask = (static_cast<unsigned long long>(m32) << 32) | m32;
-    fma2(acc, ((BITS * P + BITS > 24) ? V : W) & mask, x);
-#endif
+    if constexpr (P < kWC) {
+      constexpr int s = shift_pos(P);
+      constexpr unsigned long long m32 = ((1ull << BITS) - 1ull) << s;
+      constexpr unsigned long long mask = (m32 << 32) | m32;
+      fma2(acc, ((BITS * P + BITS > 24) ? V : W) & mask, x);
+    }
   }
+
   // Word pairs of one or two rows against shared activation pairs.
   template <bool TWO>
   __device__ __forceinline__ static void word_pair2(unsigned long long Wa, unsigned long long Wb,

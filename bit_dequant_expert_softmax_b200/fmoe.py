@@ -15,7 +15,8 @@ SO = os.path.join(HERE, "libfmoe.so")
 
 FMOE_OK = 0
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "CUDA error",
-          4: "workspace missing or too small", 5: "device-side error"}
+          4: "workspace missing or too small", 5: "device-side error", 6: "scratch limit of the no-allocation path"}
+NOALLOC_SCRATCH_BYTES = 128 * 1024
 DEVERR_BARRIER_TIMEOUT = 0x1
 DEVERR_COPY_TIMEOUT = 0x2
 DEVERR_BAD_EXPERT = 0x4
@@ -25,7 +26,7 @@ EXPORTS = ["fmoe_record_bytes", "fmoe_workspace_bytes", "fmoe_layer_create", "fm
            "fmoe_layer_set_workspace", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward",
            "fmoe_rmsnorm", "fmoe_layer_get_error", "fmoe_layer_set_wait_limit",
            "fmoe_layer_debug_hold_block", "fmoe_layer_debug_timeline", "fmoe_layer_grid_size",
-           "fmoe_status_string"]
+           "fmoe_layer_forward_noalloc", "fmoe_status_string"]
 
 
 class FmoeError(RuntimeError):
@@ -67,6 +68,7 @@ def lib():
         L.fmoe_expert_forward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp]
         L.fmoe_layer_forward.argtypes = [vp, vp, vp, i32, vp, vp]
         L.fmoe_rmsnorm.argtypes = [vp, vp, i32, i32, ctypes.c_double, vp]
+        L.fmoe_layer_forward_noalloc.argtypes = [vp, vp, vp, i32, vp, vp]
         L.fmoe_layer_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.fmoe_layer_set_wait_limit.argtypes = [vp, u64]
         L.fmoe_layer_debug_hold_block.argtypes = [vp, i32]
@@ -131,6 +133,13 @@ def fmoe_expert_forward(handle, x, resid, T, idx, w, shared_sigma, y, stream=Non
 def fmoe_layer_forward(handle, x, resid, T, y, stream=None):
     _check(lib().fmoe_layer_forward(handle, _ptr(x), _ptr(resid), T, _ptr(y), _stream(stream)),
            "fmoe_layer_forward")
+
+
+def fmoe_layer_forward_noalloc(handle, x, resid, T, y, stream=None):
+    """fmoe_layer_forward on the library's fixed scratch array (no workspace, no
+    allocation); see include/fmoe.h."""
+    _check(lib().fmoe_layer_forward_noalloc(handle, _ptr(x), _ptr(resid), T, _ptr(y), _stream(stream)),
+           "fmoe_layer_forward_noalloc")
 
 
 def fmoe_rmsnorm(h, out, T, H, eps=1e-6, stream=None):

@@ -51,7 +51,8 @@ typedef enum {
   FMOE_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels are built for    */
   FMOE_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed         */
   FMOE_ERR_NO_WORKSPACE = 4,  /* workspace missing or smaller than required          */
-  FMOE_ERR_DEVICE = 5         /* fmoe_layer_get_error found a device-side error      */
+  FMOE_ERR_DEVICE = 5,        /* fmoe_layer_get_error found a device-side error      */
+  FMOE_ERR_SCRATCH_LIMIT = 6  /* fmoe_layer_forward_noalloc: layer needs more scratch */
 } fmoe_status;
 
 /* Device-side error bits reported by fmoe_layer_get_error(). */
@@ -174,6 +175,31 @@ fmoe_status fmoe_layer_debug_timeline(fmoe_layer_t layer, uint64_t* dev_buf, int
 
 /* Number of thread blocks one forward launch uses (one per SM of the device). */
 int fmoe_layer_grid_size(fmoe_layer_t layer);
+
+/* Size in bytes of the fixed device scratch array of fmoe_layer_forward_noalloc. */
+#define FMOE_NOALLOC_SCRATCH_BYTES (128 * 1024)
+
+/* fmoe_layer_forward without any allocation, for callers that cannot allocate device
+ * memory themselves -- code running where cudaMalloc is unavailable or forbidden
+ * (inside a captured region that must not allocate, a host framework that owns all
+ * device memory, a tiny runtime without an allocator) -- and so cannot provide the
+ * workspace fmoe_layer_set_workspace expects.  The pages describing the method have
+ * no counterpart of this entry point: it exists for such callers only.
+ *
+ * Same arguments and results as fmoe_layer_forward; the layer needs no workspace.
+ * The scratch lives in one file-scope device array of FMOE_NOALLOC_SCRATCH_BYTES
+ * (128 KiB), which every GPU that loads the library keeps until the process exits.
+ * A layer whose fmoe_workspace_bytes() exceed that size is rejected with
+ * FMOE_ERR_SCRATCH_LIMIT before anything is enqueued.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress, with that device
+ * current), so make that first call before any stream capture.  Each call first
+ * clears the array's control words (an asynchronous memset on `stream`, no
+ * allocation) and nothing else allocates or frees memory.  All calls, on all layers
+ * and streams, share the one array: calls that overlap on the GPU race and must be
+ * ordered by the caller.  Device-side error bits of a call land in the array's
+ * control words, which the next call clears; they are not reported. */
+fmoe_status fmoe_layer_forward_noalloc(fmoe_layer_t layer, const uint16_t* x, const uint16_t* resid, int T,
+                                       uint16_t* y, void* stream);
 
 /* Human-readable name of a status value. */
 const char* fmoe_status_string(fmoe_status status);
