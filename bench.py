@@ -106,6 +106,30 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def profiled_traffic():
+    """DRAM bytes per launch of the layer kernel from the committed ncu summary, if
+    the kernel source is the one that was profiled (else None)."""
+    import hashlib
+    src = [os.path.join(ROOT, "bit_dequant_expert_softmax_b200", "csrc", f)
+           for f in ("fmoe_layer.cuh", "fmoe_device.cuh")]
+    h = hashlib.sha256()
+    for f in src:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    path = os.path.join(ROOT, "profiles", "fmoe_layer_kernel_layer4096.md")
+    if not os.path.exists(path):
+        return None
+    want, traffic = None, None
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if line.startswith("kernel_source_sha256:"):
+                want = line.split(":", 1)[1].strip()
+            elif line.startswith("traffic_bytes_per_launch:"):
+                traffic = int(line.split(":", 1)[1].strip())
+    return traffic if want == h.hexdigest() else None
+
+
 def layer_bytes(shape):
     """Algorithmic bytes of one single-token layer forward."""
     import fmoe_synth as synth
@@ -286,7 +310,7 @@ def main():
     achieved = (expert_b + other_b) / launch_s / 1e9
     expert_gbs = expert_b / launch_s / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": None,
+            "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
             "peak_kind": peak_kind, "kernel": "fmoe_layer_kernel<4>",
             "bytes_per_launch": expert_b + other_b, "expert_bytes_per_launch": expert_b,
             "expert_gbs": round(expert_gbs, 1), "expert_frac_of_8tbs": round(expert_gbs / HBM_NOMINAL_GBS, 4),
@@ -299,11 +323,12 @@ def main():
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "u4-dequant/f32-accum",
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic",
                 "config": {"workload": f"{args.config}: single-token decode, hidden {H}, inter {shape.inter}, "
                                        f"{shape.n_experts}+{shape.has_shared} experts, top-{shape.top_k}, "
                                        f"{shape.bits}-bit group-64",
+                           "weights": f"{shape.bits}-bit codes, bf16 scale/bias per 64-group, HBM-resident",
                            "tokens_per_step": tokens, "l2": "flushed between steps (512 MiB write)",
                            "parallelism": f"replicas x{world}"},
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": xh.numel() * 2,
