@@ -5,6 +5,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include <cuda_runtime.h>
 
@@ -343,6 +344,21 @@ fmoe_status fmoe_layer_forward(fmoe_layer_t L, const uint16_t* x, const uint16_t
   return launch(L, p, stream);
 }
 
+fmoe_status fmoe_block_forward(fmoe_layer_t L, const uint16_t* h, int T, double eps, uint16_t* h_out, void* stream) {
+  fmoe_status st = ready(L);
+  if (st != FMOE_OK) return st;
+  if (T < 0 || !(eps >= 0.0)) return FMOE_ERR_INVALID_ARG;
+  if (T == 0) return FMOE_OK;
+  if (!h || !h_out || !aligned(h, 16) || !aligned(h_out, 16)) return FMOE_ERR_INVALID_ARG;
+  Params p = base_params(L, MODE_FULL, T);
+  p.x = h;
+  p.resid = h;
+  p.y = h_out;
+  p.norm = 1;
+  p.norm_eps = eps;
+  return launch(L, p, stream);
+}
+
 fmoe_status fmoe_rmsnorm(const uint16_t* h, uint16_t* out, int T, int H, double eps, void* stream) {
   if (T < 0 || H <= 0 || !(eps >= 0.0)) return FMOE_ERR_INVALID_ARG;
   if (T == 0) return FMOE_OK;
@@ -402,6 +418,108 @@ const char* fmoe_status_string(fmoe_status s) {
       return "the layer needs more scratch than fmoe_layer_forward_noalloc's fixed array (FMOE_NOALLOC_SCRATCH_BYTES)";
   }
   return "unknown status";
+}
+
+// ---------------------------------------------------------------------------
+// Layer stacks and their CUDA graphs.
+}  // extern "C"
+
+struct fmoe_stack {
+  std::vector<fmoe_layer*> layers;
+  double eps;
+  int device;
+};
+
+struct fmoe_graph {
+  cudaGraphExec_t exec;
+};
+
+extern "C" {
+
+fmoe_status fmoe_stack_create(const fmoe_layer_t* layers, int n_layers, double eps, fmoe_stack_t* out) {
+  if (!out) return FMOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!layers || n_layers < 1 || !(eps >= 0.0)) return FMOE_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l) {
+    if (!layers[l]) return FMOE_ERR_INVALID_ARG;
+    if (!layers[l]->ws) return FMOE_ERR_NO_WORKSPACE;
+    if (layers[l]->cfg.hidden != layers[0]->cfg.hidden || layers[l]->device != layers[0]->device)
+      return FMOE_ERR_INVALID_ARG;
+  }
+  fmoe_stack* S = new (std::nothrow) fmoe_stack();
+  if (!S) return FMOE_ERR_INVALID_ARG;
+  S->layers.assign(layers, layers + n_layers);
+  S->eps = eps;
+  S->device = layers[0]->device;
+  *out = S;
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_stack_destroy(fmoe_stack_t S) {
+  delete S;
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_stack_forward(fmoe_stack_t S, uint16_t* h, int T, void* stream) {
+  if (!S || T < 0) return FMOE_ERR_INVALID_ARG;
+  if (T == 0) return FMOE_OK;
+  if (!h || !aligned(h, 16)) return FMOE_ERR_INVALID_ARG;
+  const size_t H = (size_t)S->layers[0]->cfg.hidden;
+  for (int t = 0; t < T; ++t)
+    for (fmoe_layer* L : S->layers) {
+      uint16_t* ht = h + (size_t)t * H;
+      const fmoe_status st = fmoe_block_forward(L, ht, 1, S->eps, ht, stream);
+      if (st != FMOE_OK) return st;
+    }
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_stack_graph_create(fmoe_stack_t S, uint16_t* h, int T, fmoe_graph_t* out) {
+  if (!out) return FMOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!S || T < 1 || !h || !aligned(h, 16)) return FMOE_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FMOE_ERR_CUDA;
+  if (dev != S->device) return FMOE_ERR_INVALID_ARG;
+  cudaStream_t cs = nullptr;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return FMOE_ERR_CUDA;
+  fmoe_status st = FMOE_OK;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    st = FMOE_ERR_CUDA;
+  } else {
+    st = fmoe_stack_forward(S, h, T, cs);
+    // end the capture whatever happened, so the stream is usable again
+    if (cudaStreamEndCapture(cs, &graph) != cudaSuccess && st == FMOE_OK) st = FMOE_ERR_CUDA;
+  }
+  if (st == FMOE_OK && cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) st = FMOE_ERR_CUDA;
+  if (graph) cudaGraphDestroy(graph);
+  cudaStreamDestroy(cs);
+  if (st != FMOE_OK) {
+    if (exec) cudaGraphExecDestroy(exec);
+    return st;
+  }
+  fmoe_graph* G = new (std::nothrow) fmoe_graph();
+  if (!G) {
+    cudaGraphExecDestroy(exec);
+    return FMOE_ERR_INVALID_ARG;
+  }
+  G->exec = exec;
+  *out = G;
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_graph_launch(fmoe_graph_t G, void* stream) {
+  if (!G) return FMOE_ERR_INVALID_ARG;
+  return cudaGraphLaunch(G->exec, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
+}
+
+fmoe_status fmoe_graph_destroy(fmoe_graph_t G) {
+  if (!G) return FMOE_OK;
+  const cudaError_t e = cudaGraphExecDestroy(G->exec);
+  delete G;
+  return e == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------

@@ -64,6 +64,8 @@ struct Params {
   uint32_t* hflags;  // [kMaxGrid * kFlagStride] per-block "h rows written" tags
   double* lpart;     // [2][(E+1)*nq] router partials
   float* hbuf;       // [2][(K+1)*I]  h values
+  int norm;         // 1: the input is a pre-norm block's h (RMS-normalised in the kernel)
+  double norm_eps;
   int staging_bytes;
   unsigned long long wait_ns;
   int hold_cta;
@@ -74,6 +76,7 @@ struct Params {
 // Shared-memory header (activations and the staging area follow it).
 struct alignas(128) SmemHeader {
   uint64_t bars[kNumBars];
+  double red[kWarps];    // per-warp partial sums (RMS normalisation)
   int sel[kMaxK + 1];    // expert of each slot (slot K = shared expert)
   float wsl[kMaxK + 1];  // weight of each slot (w_k; slot K = sigma)
   int abort_flag;
@@ -249,16 +252,51 @@ struct LayerKernel {
                        __uint_as_float(u.y & 0xFFFF0000u));
   }
 
+  // RMS denominator sqrt(mean(h^2) + eps) of a pre-norm block's input, in double
+  // (squares of bf16 values are exact).  Every block forms the same partial sums in
+  // the same order, so every block derives the same normalised vector.
+  __device__ double rms_of(const uint16_t* ht) {
+    const uint2* src = reinterpret_cast<const uint2*>(ht);
+    double s = 0.0;
+    for (int q = threadIdx.x; q < p.H / 4; q += kThreads) {
+      const float4 v = bf16x4(src[q]);
+      s = fma(static_cast<double>(v.x), static_cast<double>(v.x), s);
+      s = fma(static_cast<double>(v.y), static_cast<double>(v.y), s);
+      s = fma(static_cast<double>(v.z), static_cast<double>(v.z), s);
+      s = fma(static_cast<double>(v.w), static_cast<double>(v.w), s);
+    }
+    s = warp_sum_d(s);
+    if ((threadIdx.x & 31) == 0) hdr->red[threadIdx.x >> 5] = s;
+    __syncthreads();
+    double tot = 0.0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) tot += hdr->red[w];
+    return sqrt(tot / p.H + p.norm_eps);
+  }
+
+  // n = bf16(h / r) of four packed bf16 values, divided and rounded once in double
+  __device__ __forceinline__ uint2 normed(uint2 u, double r) const {
+    const float4 v = bf16x4(u);
+    const uint32_t a = f64_to_bf16(static_cast<double>(v.x) / r), b = f64_to_bf16(static_cast<double>(v.y) / r);
+    const uint32_t c = f64_to_bf16(static_cast<double>(v.z) / r), d = f64_to_bf16(static_cast<double>(v.w) / r);
+    return make_uint2(a | (b << 16), c | (d << 16));
+  }
+
   __device__ void stage_x(const uint16_t* xt, double2* xa, double2* xb) {
     constexpr int TPC = C::kCols / 4;
     const int n4 = p.H / 4;
     const uint2* src = reinterpret_cast<const uint2*>(xt);
+    const double rn = p.norm ? rms_of(xt) : 1.0;
     for (int base = 0; base < n4; base += 2 * kThreads) {  // block-uniform trip count
       uint2 nat[2];
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
         nat[k] = q < n4 ? src[q] : make_uint2(0, 0);
+      }
+      if (p.norm) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) nat[k] = normed(nat[k], rn);
       }
 #pragma unroll
       for (int k = 0; k < 2; ++k) {

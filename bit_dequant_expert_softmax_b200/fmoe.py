@@ -26,7 +26,9 @@ EXPORTS = ["fmoe_record_bytes", "fmoe_workspace_bytes", "fmoe_layer_create", "fm
            "fmoe_layer_set_workspace", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_forward",
            "fmoe_rmsnorm", "fmoe_layer_get_error", "fmoe_layer_set_wait_limit",
            "fmoe_layer_debug_hold_block", "fmoe_layer_debug_timeline", "fmoe_layer_grid_size",
-           "fmoe_layer_forward_noalloc", "fmoe_status_string"]
+           "fmoe_layer_forward_noalloc", "fmoe_status_string", "fmoe_block_forward", "fmoe_stack_create",
+           "fmoe_stack_destroy", "fmoe_stack_forward", "fmoe_stack_graph_create", "fmoe_graph_launch",
+           "fmoe_graph_destroy"]
 
 
 class FmoeError(RuntimeError):
@@ -68,6 +70,13 @@ def lib():
         L.fmoe_expert_forward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp]
         L.fmoe_layer_forward.argtypes = [vp, vp, vp, i32, vp, vp]
         L.fmoe_rmsnorm.argtypes = [vp, vp, i32, i32, ctypes.c_double, vp]
+        L.fmoe_block_forward.argtypes = [vp, vp, i32, ctypes.c_double, vp, vp]
+        L.fmoe_stack_create.argtypes = [ctypes.POINTER(vp), i32, ctypes.c_double, ctypes.POINTER(vp)]
+        L.fmoe_stack_destroy.argtypes = [vp]
+        L.fmoe_stack_forward.argtypes = [vp, vp, i32, vp]
+        L.fmoe_stack_graph_create.argtypes = [vp, vp, i32, ctypes.POINTER(vp)]
+        L.fmoe_graph_launch.argtypes = [vp, vp]
+        L.fmoe_graph_destroy.argtypes = [vp]
         L.fmoe_layer_forward_noalloc.argtypes = [vp, vp, vp, i32, vp, vp]
         L.fmoe_layer_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.fmoe_layer_set_wait_limit.argtypes = [vp, u64]
@@ -146,6 +155,39 @@ def fmoe_rmsnorm(h, out, T, H, eps=1e-6, stream=None):
     _check(lib().fmoe_rmsnorm(_ptr(h), _ptr(out), T, H, eps, _stream(stream)), "fmoe_rmsnorm")
 
 
+def fmoe_block_forward(handle, h, T, eps, h_out, stream=None):
+    _check(lib().fmoe_block_forward(handle, _ptr(h), T, eps, _ptr(h_out), _stream(stream)), "fmoe_block_forward")
+
+
+def fmoe_stack_create(handles, eps=1e-6) -> int:
+    arr = (ctypes.c_void_p * len(handles))(*handles)
+    s = ctypes.c_void_p()
+    _check(lib().fmoe_stack_create(arr, len(handles), eps, ctypes.byref(s)), "fmoe_stack_create")
+    return s.value
+
+
+def fmoe_stack_destroy(stack: int):
+    _check(lib().fmoe_stack_destroy(stack), "fmoe_stack_destroy")
+
+
+def fmoe_stack_forward(stack, h, T, stream=None):
+    _check(lib().fmoe_stack_forward(stack, _ptr(h), T, _stream(stream)), "fmoe_stack_forward")
+
+
+def fmoe_stack_graph_create(stack, h, T) -> int:
+    g = ctypes.c_void_p()
+    _check(lib().fmoe_stack_graph_create(stack, _ptr(h), T, ctypes.byref(g)), "fmoe_stack_graph_create")
+    return g.value
+
+
+def fmoe_graph_launch(graph, stream=None):
+    _check(lib().fmoe_graph_launch(graph, _stream(stream)), "fmoe_graph_launch")
+
+
+def fmoe_graph_destroy(graph):
+    _check(lib().fmoe_graph_destroy(graph), "fmoe_graph_destroy")
+
+
 def fmoe_layer_get_error(handle) -> int:
     e = ctypes.c_uint32(0)
     st = lib().fmoe_layer_get_error(handle, ctypes.byref(e))
@@ -214,10 +256,55 @@ class Layer:
         fmoe_expert_forward(self.handle, x, resid, x.shape[0], idx, w, sig, y, stream)
         return y
 
+    def block(self, h, h_out=None, eps=1e-6, stream=None):
+        """Pre-norm block h + MoE(RMSNorm(h)); h_out may be h (in place)."""
+        import torch
+        h_out = torch.empty_like(h) if h_out is None else h_out
+        fmoe_block_forward(self.handle, h, h.shape[0], eps, h_out, stream)
+        return h_out
+
     def error(self) -> int:
         return fmoe_layer_get_error(self.handle)
 
     def close(self):
         if self.handle:
             fmoe_layer_destroy(self.handle)
+            self.handle = 0
+
+
+class Stack:
+    """Layers applied as pre-norm blocks; keeps the Layer objects alive."""
+
+    def __init__(self, layers, eps=1e-6):
+        self.layers = list(layers)
+        self.eps = eps
+        self.handle = fmoe_stack_create([L.handle for L in self.layers], eps)
+
+    def forward(self, h, stream=None):
+        """Every token of h (bf16 [T, H]) through all layers, in place."""
+        fmoe_stack_forward(self.handle, h, h.shape[0], stream)
+        return h
+
+    def graph(self, h) -> "Graph":
+        return Graph(fmoe_stack_graph_create(self.handle, h, h.shape[0]), h)
+
+    def close(self):
+        if self.handle:
+            fmoe_stack_destroy(self.handle)
+            self.handle = 0
+
+
+class Graph:
+    """A captured stack decode over the buffer h (kept alive with the graph)."""
+
+    def __init__(self, handle: int, h):
+        self.handle = handle
+        self.h = h
+
+    def launch(self, stream=None):
+        fmoe_graph_launch(self.handle, stream)
+
+    def close(self):
+        if self.handle:
+            fmoe_graph_destroy(self.handle)
             self.handle = 0

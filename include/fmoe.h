@@ -149,6 +149,53 @@ fmoe_status fmoe_layer_forward(fmoe_layer_t layer, const uint16_t* x, const uint
  * computed in double and rounded once.  h, out: bf16 [T][H], may alias. */
 fmoe_status fmoe_rmsnorm(const uint16_t* h, uint16_t* out, int T, int H, double eps, void* stream);
 
+/* One pre-norm block of a layer stack, with the normalisation fused into the layer
+ * kernel: n[t] = bf16(h[t] / sqrt(mean(h[t]^2) + eps)) (as fmoe_rmsnorm computes it),
+ * then h_out[t] = h[t] + sum_k w_k o_k(n[t]) + sigma o_s(n[t]), routing on n[t], rounded
+ * once to bf16.  (hotdry.top "Metal GPU管线": RMSNorm, routing, experts and the combine
+ * with the residual run as one deferred sequence per layer; the stacks of the pages
+ * keep attention, which this library replaces by the normalisation and residual
+ * alone.)  h, h_out: bf16 [T][H], 16-byte aligned; h_out may alias h (in place).
+ * T == 0 is a no-op. */
+fmoe_status fmoe_block_forward(fmoe_layer_t layer, const uint16_t* h, int T, double eps, uint16_t* h_out,
+                               void* stream);
+
+/* A stack of layers applied as pre-norm blocks, h <- h + MoE_l(RMSNorm(h)) for
+ * l = 0 .. n_layers-1.  The stack keeps the layer handles (not owned: they must outlive
+ * it, with their workspaces attached) and eps.  All layers must have the same hidden
+ * size and live on the same device. */
+typedef struct fmoe_stack* fmoe_stack_t;
+
+/* Creates a stack over layers[0 .. n_layers-1].  Errors: INVALID_ARG (NULL handles,
+ * n_layers < 1, eps < 0, mixed hidden sizes or devices), NO_WORKSPACE (a layer without
+ * workspace).  Host memory only. */
+fmoe_status fmoe_stack_create(const fmoe_layer_t* layers, int n_layers, double eps, fmoe_stack_t* out);
+
+/* Releases the stack handle (not the layers).  NULL is accepted. */
+fmoe_status fmoe_stack_destroy(fmoe_stack_t stack);
+
+/* Single-token decode through the whole stack, in place: for t = 0 .. T-1, token t's
+ * h[t] (bf16 [H], rows of h bf16 [T][H], 16-byte aligned) passes through every block
+ * in order, one fmoe_block_forward launch per layer and token, before token t+1
+ * starts.  Asynchronous on `stream`; capturable. */
+fmoe_status fmoe_stack_forward(fmoe_stack_t stack, uint16_t* h, int T, void* stream);
+
+/* An instantiated CUDA graph of the launches fmoe_stack_forward(stack, h, T) makes
+ * (T x n_layers kernel nodes, token after token; the pages' deferred per-layer command
+ * buffer plays this role).  The graph captures the pointer h and the layers' weights
+ * and workspaces: they must stay valid and unmoved while the graph lives. */
+typedef struct fmoe_graph* fmoe_graph_t;
+
+/* Captures and instantiates the graph (on a private stream, with the stack's device
+ * current; nothing is executed).  Errors: INVALID_ARG, CUDA. */
+fmoe_status fmoe_stack_graph_create(fmoe_stack_t stack, uint16_t* h, int T, fmoe_graph_t* out);
+
+/* Replays the graph on `stream` (asynchronous). */
+fmoe_status fmoe_graph_launch(fmoe_graph_t graph, void* stream);
+
+/* Destroys the graph.  NULL is accepted. */
+fmoe_status fmoe_graph_destroy(fmoe_graph_t graph);
+
 /* Synchronises the device, returns the layer's device error bits in *device_error
  * (0 if none) and clears them (and the layer's barrier state).  Returns FMOE_OK when no
  * error was set, FMOE_ERR_DEVICE when one was. */

@@ -271,6 +271,17 @@ def rmsnorm_bf16(h: np.ndarray, eps: float = 1e-6) -> np.ndarray:
     return f64_to_bf16_bits(h / r)
 
 
+def block_forward(layer: OracleLayer, h: np.ndarray, eps: float = 1e-6) -> LayerResult:
+    """One pre-norm block of a stack: n = bf16(RMSNorm(h)); the layer runs on n with
+    the block input h as its residual, y = h + sum_k w_k o_k(n) + sigma o_s(n)
+    (hotdry.top "Metal GPU管线": normalisation, experts and the residual combine of
+    one layer; the stacks here keep no attention, so the block is norm + MoE +
+    residual).  y is returned unrounded; the stack stores it as bf16."""
+    h = np.asarray(h, dtype=np.float64)
+    n = bf16_to_f64(rmsnorm_bf16(h, eps))
+    return layer.forward(n, resid=h)
+
+
 # ----------------------------------------------------------------------------
 # synthetic layers built from the shared generator
 # ----------------------------------------------------------------------------

@@ -1,0 +1,22 @@
+"""Oracle evaluations of single pre-norm blocks of synthetic layers, in a form a
+spawned process pool can run (only numpy, the oracle and the input generator are
+imported here)."""
+import numpy as np
+
+import fmoe_synth as synth
+import oracle
+
+
+def block_case(args):
+    """(seed, layer, shape fields, h as bf16 bits) -> (idx, w, sigma, y unrounded)."""
+    seed, layer, fields, h_bits = args
+    shape = synth.LayerShape(*fields)
+    lay = oracle.synthetic_layer(seed, layer, shape, lazy=True)
+    h = oracle.bf16_to_f64(np.asarray(h_bits, dtype=np.uint16))
+    r = oracle.block_forward(lay, h)
+    return r.idx, r.w, r.sigma, r.y
+
+
+def shape_fields(shape):
+    return (shape.hidden, shape.inter, shape.n_experts, shape.top_k, shape.bits, shape.has_shared,
+            shape.router_bias)

@@ -292,6 +292,33 @@ def test_whole_layer_matches_brute_force():
         assert np.allclose(r.y, yb, rtol=1e-12, atol=1e-12)
 
 
+# ------------------------------------------------------ pre-norm block ----
+def test_block_residual_is_the_unnormalised_input():
+    """Experts whose down projections are zero add nothing: the block returns h
+    itself (not its normalised copy)."""
+    def zero_down(e, p):
+        p.down_sb[:] = 0
+    lay, H = _layer_with(zero_down)
+    h = 3.0 * _x(H)
+    r = oracle.block_forward(lay, h)
+    assert np.array_equal(r.y, h)
+
+
+def test_block_update_is_scale_invariant():
+    """With eps = 0 the normalised vector of 4h equals that of h exactly, so the
+    block's update y - h is the same for h and 4h (the experts see RMSNorm(h), not h),
+    and it differs from the update of the layer applied to h directly."""
+    lay, _ = _tiny_layer()
+    h = 0.37 * _x(128)
+    a = oracle.block_forward(lay, h, eps=0.0)
+    b = oracle.block_forward(lay, 4.0 * h, eps=0.0)
+    assert list(a.idx) == list(b.idx)
+    # equal up to the fp64 rounding of adding and removing the residual
+    assert np.allclose(a.y - h, b.y - 4.0 * h, rtol=0, atol=1e-14 * np.max(np.abs(4.0 * h)))
+    direct = lay.forward(h)
+    assert not np.allclose(direct.y - h, a.y - h, rtol=1e-3, atol=0)
+
+
 # -------------------------------------------------------------- rmsnorm ----
 def test_bf16_rounding_matches_torch():
     v = np.random.default_rng(2).standard_normal(5000).astype(np.float32).astype(np.float64)
