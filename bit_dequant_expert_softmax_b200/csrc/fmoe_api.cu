@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/fmoe.h"
+#include "fmoe_grouped.cuh"
 #include "fmoe_layer.cuh"
 
 using namespace fmoe;
@@ -64,6 +65,41 @@ WsLayout ws_layout(const fmoe_config& c) {
   return w;
 }
 
+// Workspace of the batched path for up to max_tokens tokens per call.
+struct BatchLayout {
+  size_t err, ticket, ntiles, tiles, tcost, pair_token, pidx, idx, w, sig, lpart, hbuf, obuf, xn, size;
+};
+
+int batch_max_tiles(const fmoe_config& c, int T) { return T * c.top_k + (T + kTileTok - 1) / kTileTok; }
+
+BatchLayout batch_layout(const fmoe_config& c, int T) {
+  BatchLayout b;
+  const size_t nq = (size_t)router_splits(c.hidden);
+  const size_t P = (size_t)T * (c.top_k + 1), mt = (size_t)batch_max_tiles(c, T);
+  b.err = 0;
+  b.ticket = 128;
+  b.ntiles = 256;
+  size_t o = 512;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = al256(o + bytes);
+    return at;
+  };
+  b.tiles = take(mt * sizeof(GTile));
+  b.tcost = take((mt + 1) * sizeof(long long));
+  b.pair_token = take(P * 4);
+  b.pidx = take(P * 4);
+  b.idx = take((size_t)T * c.top_k * 4);
+  b.w = take((size_t)T * c.top_k * 4);
+  b.sig = take((size_t)T * 4);
+  b.lpart = take((size_t)T * (c.n_experts + 1) * nq * 8);
+  b.hbuf = take(P * c.inter * 4);
+  b.obuf = take(P * c.hidden * 4);
+  b.xn = take((size_t)T * c.hidden * 2);
+  b.size = o;
+  return b;
+}
+
 bool config_ok(const fmoe_config* c) {
   if (!c) return false;
   RecordLayout L;
@@ -94,6 +130,12 @@ struct fmoe_layer {
   int hold_cta;
   uint64_t* timeline;
   int timeline_token;
+  // batched path
+  void* bws;
+  size_t bws_bytes;
+  int max_tokens;
+  BatchLayout bl;
+  int g_router_smem, g_topk_smem, g_gu_smem, g_dn_smem, g_db, g_ru_gu, g_ru_dn;
 };
 
 namespace {
@@ -208,6 +250,120 @@ fmoe_status launch(const fmoe_layer* L, const Params& p, void* stream) {
     e = cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<2>, p);
   return e == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
 }
+
+// Shared-memory plan of the batched kernels for up to T tokens per call.
+fmoe_status plan_batched(fmoe_layer* L, int T) {
+  const fmoe_config& c = L->cfg;
+  const int G = L->sms;
+  const int cols = c.bits == 4 ? chunk_cols<4>() : chunk_cols<2>();
+  const int rows = c.n_experts + c.has_shared;
+  // router: the block's rows plus kRouterTok token rows, all fp32
+  const size_t rsm = 128 + (size_t)((rows + G - 1) / G) * c.hidden * 4 + (size_t)kRouterTok * c.hidden * 4;
+  uint32_t tsm = 0;
+  topk_smem(c.n_experts, c.top_k, T, c.has_shared, &tsm);
+  auto act = [&](int n) {  // staged activations of a tile for rows of n columns
+    const uint32_t nch = (uint32_t)(n / cols), stride = (nch + 31) / 32 * 32 * (uint32_t)cols;
+    return (size_t)r128((uint32_t)kTileTok * (stride + nch) * 4u);
+  };
+  const int ru_gu = (int)(r16(2u * (uint32_t)L->rec.qh) + r16(2u * (uint32_t)L->rec.sh) + 16u);
+  const size_t gsm = sizeof(GHeader) + act(c.hidden) + (size_t)kWarps * kRing * ru_gu;
+  int db = 16;
+  auto ru_dn_of = [&](int d) { return (int)(r16((uint32_t)d * L->rec.qi) + r16((uint32_t)d * L->rec.si) + 16u); };
+  while (db > 1 && sizeof(GHeader) + act(c.inter) + (size_t)kWarps * kRing * ru_dn_of(db) > (size_t)kMaxSmem) db /= 2;
+  const size_t dsm = sizeof(GHeader) + act(c.inter) + (size_t)kWarps * kRing * ru_dn_of(db);
+  if (rsm > (size_t)kMaxSmem || tsm > (uint32_t)kMaxSmem || gsm > (size_t)kMaxSmem || dsm > (size_t)kMaxSmem)
+    return FMOE_ERR_UNSUPPORTED;
+  // segments a block's unit range can touch: its share of the total weight over the
+  // lightest tile, plus the partial tiles at both ends
+  const long long mt = batch_max_tiles(c, T);
+  if (mt * tile_weight(kTileTok) / ((long long)G * tile_weight(1)) + 3 > kMaxSeg) return FMOE_ERR_UNSUPPORTED;
+  L->g_router_smem = (int)rsm;
+  L->g_topk_smem = (int)tsm;
+  L->g_gu_smem = (int)gsm;
+  L->g_dn_smem = (int)dsm;
+  L->g_db = db;
+  L->g_ru_gu = ru_gu;
+  L->g_ru_dn = ru_dn_of(db);
+  return FMOE_OK;
+}
+
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+GParams batch_params(const fmoe_layer* L, int T) {
+  GParams p{};
+  const fmoe_config& c = L->cfg;
+  p.H = c.hidden;
+  p.I = c.inter;
+  p.E = c.n_experts;
+  p.K = c.top_k;
+  p.has_shared = c.has_shared;
+  p.has_rbias = c.has_router_bias;
+  p.nq = L->nq;
+  p.T = T;
+  p.experts = static_cast<const uint8_t*>(L->w.experts);
+  p.rec_bytes = L->rec.size;
+  p.o_gu_sb = L->rec.o_gu_sb;
+  p.o_d_q = L->rec.o_d_q;
+  p.o_d_sb = L->rec.o_d_sb;
+  p.qh = (int)L->rec.qh;
+  p.qi = (int)L->rec.qi;
+  p.sh = (int)L->rec.sh;
+  p.si = (int)L->rec.si;
+  p.db = L->g_db;
+  p.router = L->w.router;
+  p.rbias = L->w.router_bias;
+  p.sgate = L->w.shared_gate;
+  uint8_t* ws = static_cast<uint8_t*>(L->bws);
+  const BatchLayout& b = L->bl;
+  p.err = reinterpret_cast<uint32_t*>(ws + b.err);
+  p.ticket = reinterpret_cast<uint32_t*>(ws + b.ticket);
+  p.ntiles = reinterpret_cast<int*>(ws + b.ntiles);
+  p.tiles = reinterpret_cast<GTile*>(ws + b.tiles);
+  p.tcost = reinterpret_cast<long long*>(ws + b.tcost);
+  p.pair_token = reinterpret_cast<int*>(ws + b.pair_token);
+  p.pidx = reinterpret_cast<int*>(ws + b.pidx);
+  p.idx = reinterpret_cast<int32_t*>(ws + b.idx);
+  p.w = reinterpret_cast<float*>(ws + b.w);
+  p.sig = reinterpret_cast<float*>(ws + b.sig);
+  p.lpart = reinterpret_cast<double*>(ws + b.lpart);
+  p.hbuf = reinterpret_cast<float*>(ws + b.hbuf);
+  p.obuf = reinterpret_cast<float*>(ws + b.obuf);
+  p.wait_ns = L->wait_ns;
+  return p;
+}
+
+// router and top-K (+ grouping); then, if `experts`, gate/up, down and combine
+fmoe_status launch_batched(const fmoe_layer* L, GParams p, bool experts, cudaStream_t s) {
+  const int G = L->sms;
+  grouped_router_kernel<<<G, kThreads, L->g_router_smem, s>>>(p);
+  grouped_topk_kernel<<<p.T, kThreads, L->g_topk_smem, s>>>(p);
+  if (experts) {
+    p.ru = L->g_ru_gu;
+    if (L->cfg.bits == 4)
+      grouped_matvec_kernel<4, false><<<G, kThreads, L->g_gu_smem, s>>>(p);
+    else
+      grouped_matvec_kernel<2, false><<<G, kThreads, L->g_gu_smem, s>>>(p);
+    p.ru = L->g_ru_dn;
+    if (L->cfg.bits == 4)
+      grouped_matvec_kernel<4, true><<<G, kThreads, L->g_dn_smem, s>>>(p);
+    else
+      grouped_matvec_kernel<2, true><<<G, kThreads, L->g_dn_smem, s>>>(p);
+    grouped_combine_kernel<<<dim3((p.H + 255) / 256, p.T), 256, 0, s>>>(p);
+  }
+  return cudaGetLastError() == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
+}
+
+fmoe_status batch_ready(const fmoe_layer* L, int T) {
+  if (!L) return FMOE_ERR_INVALID_ARG;
+  if (!L->bws) return FMOE_ERR_NO_WORKSPACE;
+  if (T > L->max_tokens) return FMOE_ERR_INVALID_ARG;
+  return FMOE_OK;
+}
+
+int rmsnorm_threads(int H) { return H >= 1024 ? 1024 : ((H + 31) / 32) * 32; }
 
 fmoe_status ready(const fmoe_layer* L) {
   if (!L) return FMOE_ERR_INVALID_ARG;
@@ -359,28 +515,102 @@ fmoe_status fmoe_block_forward(fmoe_layer_t L, const uint16_t* h, int T, double 
   return launch(L, p, stream);
 }
 
+size_t fmoe_batch_workspace_bytes(const fmoe_config* cfg, int max_tokens) {
+  if (!config_ok(cfg) || max_tokens < 1 || max_tokens > kMaxBatch) return 0;
+  return batch_layout(*cfg, max_tokens).size;
+}
+
+fmoe_status fmoe_layer_set_batch_workspace(fmoe_layer_t L, void* dev_ptr, size_t bytes, int max_tokens) {
+  if (!L || !dev_ptr || !aligned(dev_ptr, 256) || max_tokens < 1 || max_tokens > kMaxBatch)
+    return FMOE_ERR_INVALID_ARG;
+  const BatchLayout bl = batch_layout(L->cfg, max_tokens);
+  if (bytes < bl.size) return FMOE_ERR_NO_WORKSPACE;
+  const fmoe_status st = plan_batched(L, max_tokens);
+  if (st != FMOE_OK) return st;
+  if (!set_smem(grouped_router_kernel, L->g_router_smem) || !set_smem(grouped_topk_kernel, L->g_topk_smem) ||
+      !set_smem(grouped_matvec_kernel<4, false>, L->g_gu_smem) ||
+      !set_smem(grouped_matvec_kernel<2, false>, L->g_gu_smem) ||
+      !set_smem(grouped_matvec_kernel<4, true>, L->g_dn_smem) || !set_smem(grouped_matvec_kernel<2, true>, L->g_dn_smem))
+    return FMOE_ERR_CUDA;
+  if (cudaMemset(dev_ptr, 0, bl.size) != cudaSuccess) return FMOE_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
+  L->bws = dev_ptr;
+  L->bws_bytes = bytes;
+  L->max_tokens = max_tokens;
+  L->bl = bl;
+  return FMOE_OK;
+}
+
+fmoe_status fmoe_route_batched(fmoe_layer_t L, const uint16_t* x, int T, int32_t* idx, float* w, float* shared_sigma,
+                               void* stream) {
+  if (T < 0) return FMOE_ERR_INVALID_ARG;
+  if (T == 0) return L ? FMOE_OK : FMOE_ERR_INVALID_ARG;
+  fmoe_status st = batch_ready(L, T);
+  if (st != FMOE_OK) return st;
+  if (!x || !aligned(x, 16) || !idx || !w) return FMOE_ERR_INVALID_ARG;
+  GParams p = batch_params(L, T);
+  p.x = x;
+  p.idx_out = idx;
+  p.w_out = w;
+  p.sig_out = shared_sigma;
+  return launch_batched(L, p, false, static_cast<cudaStream_t>(stream));
+}
+
+fmoe_status fmoe_layer_forward_batched(fmoe_layer_t L, const uint16_t* x, const uint16_t* resid, int T, uint16_t* y,
+                                       void* stream) {
+  if (T < 0) return FMOE_ERR_INVALID_ARG;
+  if (T == 0) return L ? FMOE_OK : FMOE_ERR_INVALID_ARG;
+  fmoe_status st = batch_ready(L, T);
+  if (st != FMOE_OK) return st;
+  if (!x || !resid || !y || !aligned(x, 16) || !aligned(resid, 16) || !aligned(y, 16)) return FMOE_ERR_INVALID_ARG;
+  GParams p = batch_params(L, T);
+  p.x = x;
+  p.resid = resid;
+  p.y = y;
+  return launch_batched(L, p, true, static_cast<cudaStream_t>(stream));
+}
+
+fmoe_status fmoe_block_forward_batched(fmoe_layer_t L, const uint16_t* h, int T, double eps, uint16_t* h_out,
+                                       void* stream) {
+  if (T < 0 || !(eps >= 0.0)) return FMOE_ERR_INVALID_ARG;
+  if (T == 0) return L ? FMOE_OK : FMOE_ERR_INVALID_ARG;
+  fmoe_status st = batch_ready(L, T);
+  if (st != FMOE_OK) return st;
+  if (!h || !h_out || !aligned(h, 16) || !aligned(h_out, 16)) return FMOE_ERR_INVALID_ARG;
+  GParams p = batch_params(L, T);
+  uint16_t* xn = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(L->bws) + L->bl.xn);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  fmoe_rmsnorm_kernel<<<T, rmsnorm_threads(L->cfg.hidden), 0, s>>>(h, xn, L->cfg.hidden, eps);
+  p.x = xn;
+  p.resid = h;
+  p.y = h_out;
+  return launch_batched(L, p, true, s);
+}
+
 fmoe_status fmoe_rmsnorm(const uint16_t* h, uint16_t* out, int T, int H, double eps, void* stream) {
   if (T < 0 || H <= 0 || !(eps >= 0.0)) return FMOE_ERR_INVALID_ARG;
   if (T == 0) return FMOE_OK;
   if (!h || !out) return FMOE_ERR_INVALID_ARG;
-  const int threads = H >= 1024 ? 1024 : ((H + 31) / 32) * 32;
-  fmoe_rmsnorm_kernel<<<T, threads, 0, static_cast<cudaStream_t>(stream)>>>(h, out, H, eps);
+  fmoe_rmsnorm_kernel<<<T, rmsnorm_threads(H), 0, static_cast<cudaStream_t>(stream)>>>(h, out, H, eps);
   return cudaGetLastError() == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
 }
 
 fmoe_status fmoe_layer_get_error(fmoe_layer_t L, uint32_t* device_error) {
   if (!L || !device_error) return FMOE_ERR_INVALID_ARG;
   *device_error = 0;
-  if (!L->ws) return FMOE_OK;
+  if (!L->ws && !L->bws) return FMOE_OK;
   if (cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
-  uint32_t e = 0;
+  uint32_t e = 0, eb = 0;
   uint8_t* ws = static_cast<uint8_t*>(L->ws);
-  if (cudaMemcpy(&e, ws + L->wsl.err, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return FMOE_ERR_CUDA;
-  *device_error = e;
-  if (e == 0) return FMOE_OK;
-  // clear the whole workspace: the error word, the tag base and any values an
-  // aborted launch left behind
-  if (cudaMemset(ws, 0, L->wsl.size) != cudaSuccess) return FMOE_ERR_CUDA;
+  uint8_t* bws = static_cast<uint8_t*>(L->bws);
+  if (ws && cudaMemcpy(&e, ws + L->wsl.err, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return FMOE_ERR_CUDA;
+  if (bws && cudaMemcpy(&eb, bws + L->bl.err, sizeof(eb), cudaMemcpyDeviceToHost) != cudaSuccess) return FMOE_ERR_CUDA;
+  *device_error = e | eb;
+  if ((e | eb) == 0) return FMOE_OK;
+  // clear the whole workspaces: the error words, the tag base, the grouping ticket
+  // and any values an aborted launch left behind
+  if (ws && cudaMemset(ws, 0, L->wsl.size) != cudaSuccess) return FMOE_ERR_CUDA;
+  if (bws && cudaMemset(bws, 0, L->bl.size) != cudaSuccess) return FMOE_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
   return FMOE_ERR_DEVICE;
 }
@@ -460,24 +690,30 @@ fmoe_status fmoe_stack_destroy(fmoe_stack_t S) {
   return FMOE_OK;
 }
 
-fmoe_status fmoe_stack_forward(fmoe_stack_t S, uint16_t* h, int T, void* stream) {
-  if (!S || T < 0) return FMOE_ERR_INVALID_ARG;
+fmoe_status fmoe_stack_forward(fmoe_stack_t S, uint16_t* h, int T, int batch, void* stream) {
+  if (!S || T < 0 || batch < 1) return FMOE_ERR_INVALID_ARG;
   if (T == 0) return FMOE_OK;
   if (!h || !aligned(h, 16)) return FMOE_ERR_INVALID_ARG;
   const size_t H = (size_t)S->layers[0]->cfg.hidden;
-  for (int t = 0; t < T; ++t)
+  if (batch > 1)
+    for (fmoe_layer* L : S->layers)
+      if (!L->bws || L->max_tokens < batch) return FMOE_ERR_NO_WORKSPACE;
+  for (int t0 = 0; t0 < T; t0 += batch) {
+    const int nb = T - t0 < batch ? T - t0 : batch;
+    uint16_t* ht = h + (size_t)t0 * H;
     for (fmoe_layer* L : S->layers) {
-      uint16_t* ht = h + (size_t)t * H;
-      const fmoe_status st = fmoe_block_forward(L, ht, 1, S->eps, ht, stream);
+      const fmoe_status st = batch == 1 ? fmoe_block_forward(L, ht, 1, S->eps, ht, stream)
+                                        : fmoe_block_forward_batched(L, ht, nb, S->eps, ht, stream);
       if (st != FMOE_OK) return st;
     }
+  }
   return FMOE_OK;
 }
 
-fmoe_status fmoe_stack_graph_create(fmoe_stack_t S, uint16_t* h, int T, fmoe_graph_t* out) {
+fmoe_status fmoe_stack_graph_create(fmoe_stack_t S, uint16_t* h, int T, int batch, fmoe_graph_t* out) {
   if (!out) return FMOE_ERR_INVALID_ARG;
   *out = nullptr;
-  if (!S || T < 1 || !h || !aligned(h, 16)) return FMOE_ERR_INVALID_ARG;
+  if (!S || T < 1 || batch < 1 || !h || !aligned(h, 16)) return FMOE_ERR_INVALID_ARG;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return FMOE_ERR_CUDA;
   if (dev != S->device) return FMOE_ERR_INVALID_ARG;
@@ -489,7 +725,7 @@ fmoe_status fmoe_stack_graph_create(fmoe_stack_t S, uint16_t* h, int T, fmoe_gra
   if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
     st = FMOE_ERR_CUDA;
   } else {
-    st = fmoe_stack_forward(S, h, T, cs);
+    st = fmoe_stack_forward(S, h, T, batch, cs);
     // end the capture whatever happened, so the stream is usable again
     if (cudaStreamEndCapture(cs, &graph) != cudaSuccess && st == FMOE_OK) st = FMOE_ERR_CUDA;
   }

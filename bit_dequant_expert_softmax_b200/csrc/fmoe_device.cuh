@@ -181,6 +181,15 @@ struct Chunk {
   __device__ __forceinline__ static const ulonglong2* f4(const float* base, int m, int k) {
     return reinterpret_cast<const ulonglong2*>(base) + ((((m >> 5) * kF4 + k) << 5) + (m & 31));
   }
+  // float index of column c in the lane-interleaved layout: float4 k of chunk m holds,
+  // for the word pair a = word & ~1 and kk = pos / 2, element (pos & 1) * 2 + (word & 1)
+  __device__ __forceinline__ static int phys(int c) {
+    const int m = c / kCols, r = c % kCols;
+    const int word = r / kWC, pos = r % kWC;
+    const int k = (word >> 1) * kF4PerPair + (pos >> 1);
+    const int e = ((pos & 1) << 1) | (word & 1);
+    return ((((m >> 5) * kF4 + k) << 5) + (m & 31)) * 4 + e;
+  }
   // (scale,bias) word index of chunk m within its row
   __device__ __forceinline__ static int sb_index(int m) { return BITS == 4 ? (m >> 1) : m; }
 

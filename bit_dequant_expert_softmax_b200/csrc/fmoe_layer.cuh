@@ -20,6 +20,7 @@
 #pragma once
 
 #include "fmoe_device.cuh"
+#include "fmoe_topk.cuh"
 
 namespace fmoe {
 
@@ -358,15 +359,7 @@ struct LayerKernel {
     mark(15);
   }
 
-  // float index of column c in the lane-interleaved layout
-  __device__ __forceinline__ static int phys(int c) {
-    const int m = c / C::kCols, r = c % C::kCols;
-    const int word = r / C::kWC, pos = r % C::kWC;
-    // float4 k: word pair a = word & ~1, kk = pos / 2; element (pos & 1) * 2 + (word & 1)
-    const int k = (word >> 1) * C::kF4PerPair + (pos >> 1);
-    const int e = ((pos & 1) << 1) | (word & 1);
-    return ((((m >> 5) * C::kF4 + k) << 5) + (m & 31)) * 4 + e;
-  }
+  __device__ __forceinline__ static int phys(int c) { return C::phys(c); }
 
   // ---------------------------------------------------------------- dot products
   // Lane partial of sum_c W[r][c] v[c] over the lane's chunks, for one or two rows
@@ -705,82 +698,20 @@ struct LayerKernel {
     int* cidx = reinterpret_cast<int*>(ckey + ((p.E + 31) >> 5) * p.K);
     const double* lpart = p.lpart + static_cast<size_t>(buf) * rows * p.nq;
     for (int e = threadIdx.x; e < rows; e += kThreads) {
-      double l = 0.0;
-      if (p.nq == 4) {
-        const double2 a = __ldcg(reinterpret_cast<const double2*>(lpart + static_cast<size_t>(e) * 4));
-        const double2 b = __ldcg(reinterpret_cast<const double2*>(lpart + static_cast<size_t>(e) * 4 + 2));
-        l = ((a.x + a.y) + b.x) + b.y;
-      } else {
-        for (int q = 0; q < p.nq; ++q) l += __ldcg(lpart + static_cast<size_t>(e) * p.nq + q);
-      }
+      double l = router_logit(lpart + static_cast<size_t>(e) * p.nq, p.nq);
       if (e < p.E && p.has_rbias) l += static_cast<double>(__ldg(p.rbias + e));
       slog[e] = l;
       if (e < p.E) skey[e] = dkey(l);
     }
     __syncthreads();
-    // level 1: each expert's rank among the experts of its warp's slice (the 32
-    // consecutive experts [32w + 512j, ...) for j = 0, 1, ...): keys are read back
-    // with broadcast shared loads, ties ordered by the lower index; the warp's K best
-    // become candidates, each written to the slot of its rank.
-    for (int e = threadIdx.x; e < p.E; e += kThreads) {
-      const unsigned long long ke = skey[e];
-      const int b0 = e & ~31;
-      const int nb = min(32, p.E - b0);
-      int rank = 0;
-      if (nb == 32) {
-#pragma unroll 8
-        for (int j = 0; j < 32; ++j) {
-          const unsigned long long kj = skey[b0 + j];
-          rank += static_cast<int>(kj > ke) | (static_cast<int>(kj == ke) & static_cast<int>(b0 + j < e));
-        }
-      } else {
-        for (int j = 0; j < nb; ++j) {
-          const unsigned long long kj = skey[b0 + j];
-          rank += static_cast<int>(kj > ke) | (static_cast<int>(kj == ke) & static_cast<int>(b0 + j < e));
-        }
-      }
-      if (rank < p.K) {
-        const int slot = (e >> 5) * p.K + rank;
-        ckey[slot] = ke;
-        cidx[slot] = e;
-      }
-    }
-    const int ngroups = (p.E + 31) >> 5;
-    for (int c = threadIdx.x; c < ngroups * p.K; c += kThreads) {
-      const int gsz = min(32, p.E - (c / p.K) * 32);
-      if (c % p.K >= gsz) {  // a short last group has fewer than K members
-        ckey[c] = 0;
-        cidx[c] = 0x7fffffff;
-      }
-    }
     mark(11);
-    __syncthreads();
+    rank_topk(skey, ckey, cidx, p.E, p.K, hdr->sel, kThreads);
     mark(12);
-    // level 2: every candidate's rank among all candidates; the K best are the
-    // selection, in order
-    const int ncand = ngroups * p.K;
-    for (int c = threadIdx.x; c < ncand; c += kThreads) {
-      const unsigned long long kc = ckey[c];
-      const int ic = cidx[c];
-      if (kc == 0) continue;
-      int rank = 0;
-#pragma unroll 8
-      for (int j = 0; j < ncand; ++j) {
-        const unsigned long long kj = ckey[j];
-        const int ij = cidx[j];
-        rank += static_cast<int>(kj > kc) | (static_cast<int>(kj == kc) & static_cast<int>(ij < ic));
-      }
-      if (rank < p.K) hdr->sel[rank] = ic;
-    }
-    __syncthreads();
     mark(13);
     if (warp == 0) {
-      const int mysel = lane < p.K ? hdr->sel[lane] : hdr->sel[0];
-      const double l0 = slog[hdr->sel[0]];
-      const double ek = lane < p.K ? exp(slog[mysel] - l0) : 0.0;
-      const double den = warp_sum_d(ek);
+      const double wk = topk_weight(slog, hdr->sel, p.K, lane);
       if (lane < p.K) {
-        const double wk = ek / den;
+        const int mysel = hdr->sel[lane];
         hdr->wsl[lane] = static_cast<float>(wk);
         if (blockIdx.x == 0 && p.idx_out) {
           p.idx_out[static_cast<size_t>(t) * p.K + lane] = mysel;

@@ -20,6 +20,8 @@ NOALLOC_SCRATCH_BYTES = 128 * 1024
 DEVERR_BARRIER_TIMEOUT = 0x1
 DEVERR_COPY_TIMEOUT = 0x2
 DEVERR_BAD_EXPERT = 0x4
+DEVERR_PLAN = 0x8
+MAX_BATCH = 64
 
 # every symbol include/fmoe.h declares
 EXPORTS = ["fmoe_record_bytes", "fmoe_workspace_bytes", "fmoe_layer_create", "fmoe_layer_destroy",
@@ -28,7 +30,8 @@ EXPORTS = ["fmoe_record_bytes", "fmoe_workspace_bytes", "fmoe_layer_create", "fm
            "fmoe_layer_debug_hold_block", "fmoe_layer_debug_timeline", "fmoe_layer_grid_size",
            "fmoe_layer_forward_noalloc", "fmoe_status_string", "fmoe_block_forward", "fmoe_stack_create",
            "fmoe_stack_destroy", "fmoe_stack_forward", "fmoe_stack_graph_create", "fmoe_graph_launch",
-           "fmoe_graph_destroy"]
+           "fmoe_graph_destroy", "fmoe_batch_workspace_bytes", "fmoe_layer_set_batch_workspace",
+           "fmoe_route_batched", "fmoe_layer_forward_batched", "fmoe_block_forward_batched"]
 
 
 class FmoeError(RuntimeError):
@@ -73,8 +76,14 @@ def lib():
         L.fmoe_block_forward.argtypes = [vp, vp, i32, ctypes.c_double, vp, vp]
         L.fmoe_stack_create.argtypes = [ctypes.POINTER(vp), i32, ctypes.c_double, ctypes.POINTER(vp)]
         L.fmoe_stack_destroy.argtypes = [vp]
-        L.fmoe_stack_forward.argtypes = [vp, vp, i32, vp]
-        L.fmoe_stack_graph_create.argtypes = [vp, vp, i32, ctypes.POINTER(vp)]
+        L.fmoe_stack_forward.argtypes = [vp, vp, i32, i32, vp]
+        L.fmoe_stack_graph_create.argtypes = [vp, vp, i32, i32, ctypes.POINTER(vp)]
+        L.fmoe_batch_workspace_bytes.restype = sz
+        L.fmoe_batch_workspace_bytes.argtypes = [ctypes.POINTER(fmoe_config), i32]
+        L.fmoe_layer_set_batch_workspace.argtypes = [vp, vp, sz, i32]
+        L.fmoe_route_batched.argtypes = [vp, vp, i32, vp, vp, vp, vp]
+        L.fmoe_layer_forward_batched.argtypes = [vp, vp, vp, i32, vp, vp]
+        L.fmoe_block_forward_batched.argtypes = [vp, vp, i32, ctypes.c_double, vp, vp]
         L.fmoe_graph_launch.argtypes = [vp, vp]
         L.fmoe_graph_destroy.argtypes = [vp]
         L.fmoe_layer_forward_noalloc.argtypes = [vp, vp, vp, i32, vp, vp]
@@ -170,14 +179,38 @@ def fmoe_stack_destroy(stack: int):
     _check(lib().fmoe_stack_destroy(stack), "fmoe_stack_destroy")
 
 
-def fmoe_stack_forward(stack, h, T, stream=None):
-    _check(lib().fmoe_stack_forward(stack, _ptr(h), T, _stream(stream)), "fmoe_stack_forward")
+def fmoe_stack_forward(stack, h, T, batch=1, stream=None):
+    _check(lib().fmoe_stack_forward(stack, _ptr(h), T, batch, _stream(stream)), "fmoe_stack_forward")
 
 
-def fmoe_stack_graph_create(stack, h, T) -> int:
+def fmoe_stack_graph_create(stack, h, T, batch=1) -> int:
     g = ctypes.c_void_p()
-    _check(lib().fmoe_stack_graph_create(stack, _ptr(h), T, ctypes.byref(g)), "fmoe_stack_graph_create")
+    _check(lib().fmoe_stack_graph_create(stack, _ptr(h), T, batch, ctypes.byref(g)), "fmoe_stack_graph_create")
     return g.value
+
+
+def fmoe_batch_workspace_bytes(cfg: fmoe_config, max_tokens: int) -> int:
+    return lib().fmoe_batch_workspace_bytes(ctypes.byref(cfg), max_tokens)
+
+
+def fmoe_layer_set_batch_workspace(handle, ws, max_tokens: int):
+    _check(lib().fmoe_layer_set_batch_workspace(handle, ws.data_ptr(), ws.numel() * ws.element_size(), max_tokens),
+           "fmoe_layer_set_batch_workspace")
+
+
+def fmoe_route_batched(handle, x, T, idx, w, shared_sigma=None, stream=None):
+    _check(lib().fmoe_route_batched(handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(shared_sigma), _stream(stream)),
+           "fmoe_route_batched")
+
+
+def fmoe_layer_forward_batched(handle, x, resid, T, y, stream=None):
+    _check(lib().fmoe_layer_forward_batched(handle, _ptr(x), _ptr(resid), T, _ptr(y), _stream(stream)),
+           "fmoe_layer_forward_batched")
+
+
+def fmoe_block_forward_batched(handle, h, T, eps, h_out, stream=None):
+    _check(lib().fmoe_block_forward_batched(handle, _ptr(h), T, eps, _ptr(h_out), _stream(stream)),
+           "fmoe_block_forward_batched")
 
 
 def fmoe_graph_launch(graph, stream=None):
@@ -223,6 +256,7 @@ class Layer:
     router_bias: object
     shared_gate: object
     workspace: object
+    batch_workspace: object = None
 
     @staticmethod
     def create(cfg: fmoe_config, experts, router, router_bias=None, shared_gate=None) -> "Layer":
@@ -263,6 +297,39 @@ class Layer:
         fmoe_block_forward(self.handle, h, h.shape[0], eps, h_out, stream)
         return h_out
 
+    def attach_batch(self, max_tokens: int):
+        """Allocates and attaches the batched-path workspace for up to max_tokens tokens."""
+        import torch
+        n = fmoe_batch_workspace_bytes(self.cfg, max_tokens)
+        if n == 0:
+            raise FmoeError(1, "fmoe_batch_workspace_bytes")
+        ws = torch.empty(n, dtype=torch.uint8, device=self.experts.device)
+        fmoe_layer_set_batch_workspace(self.handle, ws, max_tokens)
+        self.batch_workspace = ws
+        return self
+
+    def forward_batched(self, x, resid=None, y=None, stream=None):
+        import torch
+        resid = x if resid is None else resid
+        y = torch.empty_like(x) if y is None else y
+        fmoe_layer_forward_batched(self.handle, x, resid, x.shape[0], y, stream)
+        return y
+
+    def route_batched(self, x, stream=None):
+        import torch
+        T, K = x.shape[0], self.cfg.top_k
+        idx = torch.empty(T, K, dtype=torch.int32, device=x.device)
+        w = torch.empty(T, K, dtype=torch.float32, device=x.device)
+        sig = torch.empty(T, dtype=torch.float32, device=x.device)
+        fmoe_route_batched(self.handle, x, T, idx, w, sig, stream)
+        return idx, w, sig
+
+    def block_batched(self, h, h_out=None, eps=1e-6, stream=None):
+        import torch
+        h_out = torch.empty_like(h) if h_out is None else h_out
+        fmoe_block_forward_batched(self.handle, h, h.shape[0], eps, h_out, stream)
+        return h_out
+
     def error(self) -> int:
         return fmoe_layer_get_error(self.handle)
 
@@ -280,13 +347,14 @@ class Stack:
         self.eps = eps
         self.handle = fmoe_stack_create([L.handle for L in self.layers], eps)
 
-    def forward(self, h, stream=None):
-        """Every token of h (bf16 [T, H]) through all layers, in place."""
-        fmoe_stack_forward(self.handle, h, h.shape[0], stream)
+    def forward(self, h, batch=1, stream=None):
+        """Every token of h (bf16 [T, H]) through all layers, in place; batch > 1 runs
+        steps of `batch` tokens on the batched path."""
+        fmoe_stack_forward(self.handle, h, h.shape[0], batch, stream)
         return h
 
-    def graph(self, h) -> "Graph":
-        return Graph(fmoe_stack_graph_create(self.handle, h, h.shape[0]), h)
+    def graph(self, h, batch=1) -> "Graph":
+        return Graph(fmoe_stack_graph_create(self.handle, h, h.shape[0], batch), h)
 
     def close(self):
         if self.handle:

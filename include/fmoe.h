@@ -59,6 +59,8 @@ typedef enum {
 #define FMOE_DEVERR_BARRIER_TIMEOUT 0x1u  /* a grid-wide wait ran past its time limit  */
 #define FMOE_DEVERR_COPY_TIMEOUT    0x2u  /* a wait for a bulk copy ran past the limit */
 #define FMOE_DEVERR_BAD_EXPERT      0x4u  /* fmoe_expert_forward got idx out of range  */
+#define FMOE_DEVERR_PLAN            0x8u  /* a batched launch's work split overran the
+                                             limits its plan was checked against     */
 
 /* Layer geometry.  hidden (H) and inter (I) are multiples of 64; bits is 4 or 2;
  * 1 <= top_k (K) <= n_experts (E); has_shared and has_router_bias are 0 or 1. */
@@ -160,6 +162,44 @@ fmoe_status fmoe_rmsnorm(const uint16_t* h, uint16_t* out, int T, int H, double 
 fmoe_status fmoe_block_forward(fmoe_layer_t layer, const uint16_t* h, int T, double eps, uint16_t* h_out,
                                void* stream);
 
+/* ---- Batched decode: T tokens per call, grouped by expert --------------------------
+ * The same per-token results as the single-token entry points (routing identical bit
+ * for bit; outputs within the same tolerance of the fp64 definition), computed in
+ * another order: the T*K (token, slot) pairs are grouped by expert, so each active
+ * expert's weights stream from HBM once for all of its tokens.  The pages decode one
+ * token at a time; grouping several tokens' pairs by expert is this library's
+ * addition for batched decode, kept to the same arithmetic per (token, expert).
+ * Launch sequence per call: router (fp64, all tokens in one pass over the router),
+ * top-K per token plus the grouping, grouped gate/up + SwiGLU, grouped down, combine. */
+
+/* Bytes of the batched-path workspace for up to max_tokens (1..64) tokens per call (0
+ * for an invalid config or max_tokens). */
+size_t fmoe_batch_workspace_bytes(const fmoe_config* cfg, int max_tokens);
+
+/* Attaches a caller-owned device workspace for the batched entry points (separate from
+ * the single-token workspace), 256-byte aligned, of at least
+ * fmoe_batch_workspace_bytes(cfg, max_tokens) bytes, and zeroes it (synchronously).
+ * Errors: INVALID_ARG, NO_WORKSPACE (too small), UNSUPPORTED (shapes the batched
+ * kernels' shared-memory plan cannot hold), CUDA. */
+fmoe_status fmoe_layer_set_batch_workspace(fmoe_layer_t layer, void* dev_ptr, size_t bytes, int max_tokens);
+
+/* Routing of T <= max_tokens tokens in one batched pass: idx int32 [T][K], w fp32 [T][K],
+ * shared_sigma fp32 [T] (may be NULL), as fmoe_route computes them. */
+fmoe_status fmoe_route_batched(fmoe_layer_t layer, const uint16_t* x, int T, int32_t* idx, float* w,
+                               float* shared_sigma, void* stream);
+
+/* The whole layer for T <= max_tokens tokens, grouped by expert:
+ * y[t] = resid[t] + sum_k w_k o_k(x[t]) + sigma o_s(x[t]).  x, resid, y: bf16 [T][H],
+ * 16-byte aligned; y may alias x or resid. */
+fmoe_status fmoe_layer_forward_batched(fmoe_layer_t layer, const uint16_t* x, const uint16_t* resid, int T,
+                                       uint16_t* y, void* stream);
+
+/* fmoe_block_forward for T <= max_tokens tokens on the batched path: the normalised
+ * input n = bf16(h / sqrt(mean(h^2) + eps)) is written to the batch workspace, then
+ * h_out = h + MoE(n).  h_out may alias h. */
+fmoe_status fmoe_block_forward_batched(fmoe_layer_t layer, const uint16_t* h, int T, double eps, uint16_t* h_out,
+                                       void* stream);
+
 /* A stack of layers applied as pre-norm blocks, h <- h + MoE_l(RMSNorm(h)) for
  * l = 0 .. n_layers-1.  The stack keeps the layer handles (not owned: they must outlive
  * it, with their workspaces attached) and eps.  All layers must have the same hidden
@@ -174,21 +214,22 @@ fmoe_status fmoe_stack_create(const fmoe_layer_t* layers, int n_layers, double e
 /* Releases the stack handle (not the layers).  NULL is accepted. */
 fmoe_status fmoe_stack_destroy(fmoe_stack_t stack);
 
-/* Single-token decode through the whole stack, in place: for t = 0 .. T-1, token t's
- * h[t] (bf16 [H], rows of h bf16 [T][H], 16-byte aligned) passes through every block
- * in order, one fmoe_block_forward launch per layer and token, before token t+1
- * starts.  Asynchronous on `stream`; capturable. */
-fmoe_status fmoe_stack_forward(fmoe_stack_t stack, uint16_t* h, int T, void* stream);
+/* Decode through the whole stack, in place, on h bf16 [T][H] (16-byte aligned).
+ * batch == 1: token after token, each through every block (one fmoe_block_forward
+ * launch per layer and token) before the next starts.  batch > 1: steps of `batch`
+ * tokens (the last step may be shorter), each step through every block on the batched
+ * path (fmoe_block_forward_batched; every layer needs a batch workspace with
+ * max_tokens >= batch, else NO_WORKSPACE).  Asynchronous on `stream`; capturable. */
+fmoe_status fmoe_stack_forward(fmoe_stack_t stack, uint16_t* h, int T, int batch, void* stream);
 
-/* An instantiated CUDA graph of the launches fmoe_stack_forward(stack, h, T) makes
- * (T x n_layers kernel nodes, token after token; the pages' deferred per-layer command
- * buffer plays this role).  The graph captures the pointer h and the layers' weights
+/* An instantiated CUDA graph of the launches fmoe_stack_forward(stack, h, T, batch)
+ * makes (the pages' deferred per-layer command buffer plays this role).  The graph captures the pointer h and the layers' weights
  * and workspaces: they must stay valid and unmoved while the graph lives. */
 typedef struct fmoe_graph* fmoe_graph_t;
 
 /* Captures and instantiates the graph (on a private stream, with the stack's device
  * current; nothing is executed).  Errors: INVALID_ARG, CUDA. */
-fmoe_status fmoe_stack_graph_create(fmoe_stack_t stack, uint16_t* h, int T, fmoe_graph_t* out);
+fmoe_status fmoe_stack_graph_create(fmoe_stack_t stack, uint16_t* h, int T, int batch, fmoe_graph_t* out);
 
 /* Replays the graph on `stream` (asynchronous). */
 fmoe_status fmoe_graph_launch(fmoe_graph_t graph, void* stream);
