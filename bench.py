@@ -199,6 +199,140 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def bench_stack(args, world, rank):
+    """A layer stack (pre-norm blocks) decoding its token set through the captured
+    graph: token after token (batch 1) or in steps of `batch` tokens on the batched
+    path.  One step = every token of the set through every layer."""
+    import torch
+    import torch.distributed as dist
+
+    import fmoe_synth as synth
+    from bit_dequant_expert_softmax_b200 import fmoe
+    from fmoe_synth.torch_layer import make_device_layer, make_device_x
+
+    cfg_d = synth.CONFIGS[args.config]
+    shape, NL, B = cfg_d["shape"], cfg_d["layers"], cfg_d["batch"]
+    tokens = args.tokens or cfg_d["tokens"]
+    H = shape.hidden
+    cfg = fmoe.fmoe_config(H, shape.inter, shape.n_experts, shape.top_k, shape.bits, shape.has_shared,
+                           shape.router_bias)
+    layers = []
+    for l in range(NL):
+        w = make_device_layer(shape, 0, l)
+        L = fmoe.Layer.create(cfg, w.experts, w.router, w.router_bias, w.shared_gate)
+        if B > 1:
+            L.attach_batch(B)
+        layers.append(L)
+    stack = fmoe.Stack(layers, 1e-6)
+    h0 = make_device_x(0, rank * tokens, tokens, H)
+    h = h0.clone()
+    graph = stack.graph(h, batch=B)
+    stream = torch.cuda.Stream()
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            h.copy_(h0)
+            graph.launch(stream)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            h.copy_(h0)           # every step decodes the same token set
+            flush.fill_(i & 0xFF)  # L2 flush (outside the timed events)
+            starts[i].record(stream)
+            graph.launch(stream)
+            ends[i].record(stream)
+    barrier()
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    t = torch.tensor([sum(step_ms)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    errs = [L.error() for L in layers]
+    if any(errs):
+        raise RuntimeError(f"device-side error bits {errs} during the benchmark")
+    # end to end: the token set from pinned host memory, the result back
+    hh = h0.cpu().pin_memory()
+    ho = torch.empty_like(hh).pin_memory()
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with torch.cuda.stream(stream):
+        e_s.record(stream)
+        for i in range(args.steps):
+            h.copy_(hh, non_blocking=True)
+            graph.launch(stream)
+            ho.copy_(h, non_blocking=True)
+        e_e.record(stream)
+    barrier()
+    te = torch.tensor([e_s.elapsed_time(e_e)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+
+    rb = synth.record_bytes(H, shape.inter, shape.bits)
+    router_b = shape.n_experts * H * 4 + (H * 4 if shape.has_shared else 0)
+    if B > 1:
+        # distinct routed experts per layer-step, counted on the first step's routing
+        hs = h0[:B].clone()
+        uniq = []
+        for L in layers:
+            n = torch.empty_like(hs)
+            fmoe.fmoe_rmsnorm(hs, n, B, H, 1e-6)
+            idx, _, _ = L.route_batched(n)
+            uniq.append(int(torch.unique(idx).numel()))
+            L.block_batched(hs, h_out=hs)
+        mean_u = sum(uniq) / len(uniq)
+        step_bytes = (tokens / B) * NL * ((mean_u + shape.has_shared) * rb + router_b)
+        expert_bytes = (tokens / B) * NL * (mean_u + shape.has_shared) * rb
+    else:
+        mean_u = None
+        step_bytes = tokens * NL * ((shape.top_k + shape.has_shared) * rb + router_b)
+        expert_bytes = tokens * NL * (shape.top_k + shape.has_shared) * rb
+    peak, peak_kind = measured_peaks()
+    step_s = total_ms / 1e3 / args.steps
+    achieved = step_bytes / step_s / 1e9
+    value = tokens * args.steps * world / (total_ms / 1e3)
+    if rank == 0:
+        launches_per_layer = 1 if B == 1 else 6
+        line = {"metric": f"{NL}-layer stack decode tokens/s", "value": value, "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic",
+                "config": {"workload": f"{args.config}: {NL} pre-norm layers, hidden {H}, inter {shape.inter}, "
+                                       f"{shape.n_experts}+{shape.has_shared} experts, top-{shape.top_k}, "
+                                       f"{shape.bits}-bit, {tokens} tokens "
+                                       + ("one at a time" if B == 1 else f"in steps of {B} grouped by expert"),
+                           "tokens_per_step": tokens, "l2": "flushed between steps (512 MiB write)",
+                           "parallelism": f"replicas x{world}"},
+                "e2e": {"value": tokens * args.steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": hh.numel() * 2, "d2h_bytes_per_step": ho.numel() * 2},
+                "gpu_launches": args.steps * NL * (tokens if B == 1 else -(-tokens // B) * launches_per_layer),
+                "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                             "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                             "kernel": "whole step (all kernels)", "bytes_per_step": step_bytes,
+                             "expert_gbs": round(expert_bytes / step_s / 1e9, 1),
+                             "mean_distinct_experts_per_layer_step": mean_u},
+                "cpu_baseline": None, "clocks": clocks,
+                "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)}}
+        print(json.dumps(line), flush=True)
+    graph.close()
+    stack.close()
+    for L in layers:
+        L.close()
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -221,6 +355,11 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
+    if synth.CONFIGS[args.config]["layers"] > 1:
+        bench_stack(args, world, rank)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     shape = synth.CONFIGS[args.config]["shape"]
     tokens = args.tokens or synth.CONFIGS[args.config]["tokens"]
     H = shape.hidden

@@ -140,6 +140,11 @@ struct fmoe_layer {
 
 namespace {
 
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
 template <int BITS>
 int chunk_cols() {
   return Chunk<BITS>::kCols;
@@ -245,9 +250,11 @@ fmoe_status launch(const fmoe_layer* L, const Params& p, void* stream) {
   cfg.numAttrs = 1;
   cudaError_t e;
   if (L->cfg.bits == 4)
-    e = cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<4>, p);
+    e = p.norm ? cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<4, true>, p)
+               : cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<4, false>, p);
   else
-    e = cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<2>, p);
+    e = p.norm ? cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<2, true>, p)
+               : cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<2, false>, p);
   return e == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
 }
 
@@ -285,11 +292,6 @@ fmoe_status plan_batched(fmoe_layer* L, int T) {
   L->g_ru_gu = ru_gu;
   L->g_ru_dn = ru_dn_of(db);
   return FMOE_OK;
-}
-
-template <typename K>
-bool set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
 GParams batch_params(const fmoe_layer* L, int T) {
@@ -415,15 +417,13 @@ fmoe_status fmoe_layer_create(const fmoe_config* cfg, const fmoe_weights* w, fmo
     delete L;
     return st;
   }
-  if (cudaFuncSetAttribute(fmoe_layer_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, L->smem_bytes) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(fmoe_layer_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, L->smem_bytes) !=
-          cudaSuccess) {
+  if (!set_smem(fmoe_layer_kernel<4, false>, L->smem_bytes) || !set_smem(fmoe_layer_kernel<2, false>, L->smem_bytes) ||
+      !set_smem(fmoe_layer_kernel<4, true>, L->smem_bytes) || !set_smem(fmoe_layer_kernel<2, true>, L->smem_bytes)) {
     delete L;
     return FMOE_ERR_CUDA;
   }
   int nb = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fmoe_layer_kernel<4>, kThreads, L->smem_bytes) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fmoe_layer_kernel<4, false>, kThreads, L->smem_bytes) !=
           cudaSuccess ||
       nb < 1) {
     delete L;

@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_topk_kernel(const __grid_
     if (e < p.E) skey[e] = dkey(l);
   }
   __syncthreads();
-  rank_topk(skey, ckey, cidx, p.E, p.K, sel, kThreads);
+  rank_topk<kThreads>(skey, ckey, cidx, p.E, p.K, sel);
   if (warp == 0) {
     const double wk = topk_weight(slog, sel, p.K, lane);
     if (lane < p.K) {

@@ -65,7 +65,7 @@ struct Params {
   uint32_t* hflags;  // [kMaxGrid * kFlagStride] per-block "h rows written" tags
   double* lpart;     // [2][(E+1)*nq] router partials
   float* hbuf;       // [2][(K+1)*I]  h values
-  int norm;         // 1: the input is a pre-norm block's h (RMS-normalised in the kernel)
+  int norm;         // 1: the input is a pre-norm block's h (the NORM kernel variant)
   double norm_eps;
   int staging_bytes;
   unsigned long long wait_ns;
@@ -127,7 +127,8 @@ struct GuChunk {
   uint32_t off, first;
 };
 
-template <int BITS>
+// NORM: the input is a pre-norm block's h, RMS-normalised while it is staged.
+template <int BITS, bool NORM>
 struct LayerKernel {
   using C = Chunk<BITS>;
 
@@ -287,7 +288,7 @@ struct LayerKernel {
     constexpr int TPC = C::kCols / 4;
     const int n4 = p.H / 4;
     const uint2* src = reinterpret_cast<const uint2*>(xt);
-    const double rn = p.norm ? rms_of(xt) : 1.0;
+    const double rn = NORM ? rms_of(xt) : 1.0;
     for (int base = 0; base < n4; base += 2 * kThreads) {  // block-uniform trip count
       uint2 nat[2];
 #pragma unroll
@@ -295,7 +296,7 @@ struct LayerKernel {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
         nat[k] = q < n4 ? src[q] : make_uint2(0, 0);
       }
-      if (p.norm) {
+      if (NORM) {
 #pragma unroll
         for (int k = 0; k < 2; ++k) nat[k] = normed(nat[k], rn);
       }
@@ -705,7 +706,7 @@ struct LayerKernel {
     }
     __syncthreads();
     mark(11);
-    rank_topk(skey, ckey, cidx, p.E, p.K, hdr->sel, kThreads);
+    rank_topk<kThreads>(skey, ckey, cidx, p.E, p.K, hdr->sel);
     mark(12);
     mark(13);
     if (warp == 0) {
@@ -886,10 +887,10 @@ struct LayerKernel {
   }
 };
 
-template <int BITS>
+template <int BITS, bool NORM>
 __global__ void __launch_bounds__(kThreads, 1) fmoe_layer_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  LayerKernel<BITS> L(p, smem);
+  LayerKernel<BITS, NORM> L(p, smem);
   L.run();
 }
 

@@ -26,11 +26,12 @@ __device__ __forceinline__ double router_logit(const double* lp, int nq) {
 }
 
 // skey[e], e < E: keys of the logits.  ckey / cidx: scratch of ceil(E/32)*K entries.
-// Writes sel[0..K).  Called by every thread of a block of `nthreads` threads; ends
+// Writes sel[0..K).  Called by every thread of a block of NTHREADS threads; ends
 // synchronised.
+template <int NTHREADS>
 __device__ __forceinline__ void rank_topk(const unsigned long long* skey, unsigned long long* ckey, int* cidx,
-                                          int E, int K, int* sel, int nthreads) {
-  for (int e = threadIdx.x; e < E; e += nthreads) {
+                                          int E, int K, int* sel) {
+  for (int e = threadIdx.x; e < E; e += NTHREADS) {
     const unsigned long long ke = skey[e];
     const int b0 = e & ~31;
     const int nb = min(32, E - b0);
@@ -54,7 +55,7 @@ __device__ __forceinline__ void rank_topk(const unsigned long long* skey, unsign
     }
   }
   const int ngroups = (E + 31) >> 5;
-  for (int c = threadIdx.x; c < ngroups * K; c += nthreads) {
+  for (int c = threadIdx.x; c < ngroups * K; c += NTHREADS) {
     const int gsz = min(32, E - (c / K) * 32);
     if (c % K >= gsz) {  // a short last group has fewer than K members
       ckey[c] = 0;
@@ -63,7 +64,7 @@ __device__ __forceinline__ void rank_topk(const unsigned long long* skey, unsign
   }
   __syncthreads();
   const int ncand = ngroups * K;
-  for (int c = threadIdx.x; c < ncand; c += nthreads) {
+  for (int c = threadIdx.x; c < ncand; c += NTHREADS) {
     const unsigned long long kc = ckey[c];
     const int ic = cidx[c];
     if (kc == 0) continue;
