@@ -135,7 +135,7 @@ struct fmoe_layer {
   size_t bws_bytes;
   int max_tokens;
   BatchLayout bl;
-  int g_router_smem, g_topk_smem, g_gu_smem, g_dn_smem, g_db, g_ru_gu, g_ru_dn;
+  int g_router_smem, g_topk_smem, g_gu_smem, g_dn_smem;
 };
 
 namespace {
@@ -262,22 +262,19 @@ fmoe_status launch(const fmoe_layer* L, const Params& p, void* stream) {
 fmoe_status plan_batched(fmoe_layer* L, int T) {
   const fmoe_config& c = L->cfg;
   const int G = L->sms;
-  const int cols = c.bits == 4 ? chunk_cols<4>() : chunk_cols<2>();
   const int rows = c.n_experts + c.has_shared;
-  // router: the block's rows plus kRouterTok token rows, all fp32
-  const size_t rsm = 128 + (size_t)((rows + G - 1) / G) * c.hidden * 4 + (size_t)kRouterTok * c.hidden * 4;
+  // router: the block's router slices (fp32) plus kRouterTok token rows of the column
+  // splits it touches (fp64)
+  const int nq = router_splits(c.hidden), hc = c.hidden / nq;
+  const size_t rsm = 128 + r128((uint32_t)(((long long)rows * nq + G - 1) / G) * hc * 4u) +
+                     (size_t)kRouterTok * router_splits_touched(rows, nq, G) * hc * 8;
   uint32_t tsm = 0;
   topk_smem(c.n_experts, c.top_k, T, c.has_shared, &tsm);
-  auto act = [&](int n) {  // staged activations of a tile for rows of n columns
-    const uint32_t nch = (uint32_t)(n / cols), stride = (nch + 31) / 32 * 32 * (uint32_t)cols;
-    return (size_t)r128((uint32_t)kTileTok * (stride + nch) * 4u);
+  auto mv_smem = [&](bool down) {
+    const MvGeom g = mv_geom(down, c.hidden, c.inter, c.bits);
+    return sizeof(GHeader) + (size_t)g.frag_bytes + (size_t)g.sum_bytes + (size_t)kGWarps * kRing * g.piece_bytes;
   };
-  const int ru_gu = (int)(r16(2u * (uint32_t)L->rec.qh) + r16(2u * (uint32_t)L->rec.sh) + 16u);
-  const size_t gsm = sizeof(GHeader) + act(c.hidden) + (size_t)kWarps * kRing * ru_gu;
-  int db = 16;
-  auto ru_dn_of = [&](int d) { return (int)(r16((uint32_t)d * L->rec.qi) + r16((uint32_t)d * L->rec.si) + 16u); };
-  while (db > 1 && sizeof(GHeader) + act(c.inter) + (size_t)kWarps * kRing * ru_dn_of(db) > (size_t)kMaxSmem) db /= 2;
-  const size_t dsm = sizeof(GHeader) + act(c.inter) + (size_t)kWarps * kRing * ru_dn_of(db);
+  const size_t gsm = mv_smem(false), dsm = mv_smem(true);
   if (rsm > (size_t)kMaxSmem || tsm > (uint32_t)kMaxSmem || gsm > (size_t)kMaxSmem || dsm > (size_t)kMaxSmem)
     return FMOE_ERR_UNSUPPORTED;
   // segments a block's unit range can touch: its share of the total weight over the
@@ -288,9 +285,6 @@ fmoe_status plan_batched(fmoe_layer* L, int T) {
   L->g_topk_smem = (int)tsm;
   L->g_gu_smem = (int)gsm;
   L->g_dn_smem = (int)dsm;
-  L->g_db = db;
-  L->g_ru_gu = ru_gu;
-  L->g_ru_dn = ru_dn_of(db);
   return FMOE_OK;
 }
 
@@ -314,7 +308,6 @@ GParams batch_params(const fmoe_layer* L, int T) {
   p.qi = (int)L->rec.qi;
   p.sh = (int)L->rec.sh;
   p.si = (int)L->rec.si;
-  p.db = L->g_db;
   p.router = L->w.router;
   p.rbias = L->w.router_bias;
   p.sgate = L->w.shared_gate;
@@ -343,16 +336,14 @@ fmoe_status launch_batched(const fmoe_layer* L, GParams p, bool experts, cudaStr
   grouped_router_kernel<<<G, kThreads, L->g_router_smem, s>>>(p);
   grouped_topk_kernel<<<p.T, kThreads, L->g_topk_smem, s>>>(p);
   if (experts) {
-    p.ru = L->g_ru_gu;
     if (L->cfg.bits == 4)
-      grouped_matvec_kernel<4, false><<<G, kThreads, L->g_gu_smem, s>>>(p);
+      grouped_matvec_kernel<4, false><<<G, kGThreads, L->g_gu_smem, s>>>(p);
     else
-      grouped_matvec_kernel<2, false><<<G, kThreads, L->g_gu_smem, s>>>(p);
-    p.ru = L->g_ru_dn;
+      grouped_matvec_kernel<2, false><<<G, kGThreads, L->g_gu_smem, s>>>(p);
     if (L->cfg.bits == 4)
-      grouped_matvec_kernel<4, true><<<G, kThreads, L->g_dn_smem, s>>>(p);
+      grouped_matvec_kernel<4, true><<<G, kGThreads, L->g_dn_smem, s>>>(p);
     else
-      grouped_matvec_kernel<2, true><<<G, kThreads, L->g_dn_smem, s>>>(p);
+      grouped_matvec_kernel<2, true><<<G, kGThreads, L->g_dn_smem, s>>>(p);
     grouped_combine_kernel<<<dim3((p.H + 255) / 256, p.T), 256, 0, s>>>(p);
   }
   return cudaGetLastError() == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;

@@ -28,7 +28,7 @@
 
 namespace fmoe {
 
-constexpr int kTileTok = 4;    // pairs whose activations are staged together
+constexpr int kTileTok = 8;    // pairs of one expert whose activations are staged together (MMA N)
 constexpr int kRouterTok = 8;  // tokens per pass of the batched router
 constexpr int kMaxBatch = 64;  // tokens one batched call may have
 constexpr int kMaxSeg = 64;    // tiles one block's unit range may touch
@@ -38,17 +38,15 @@ struct GTile {
   int expert, p0, n, pad;
 };
 
-// Work weight of one unit of a tile of n pairs (relative): the bytes of a unit are
-// the same for every tile; the dot-product work grows with n.
-__host__ __device__ constexpr int tile_weight(int n) { return 11 + 9 * n > 24 ? 11 + 9 * n : 24; }
+// Work weight of one unit of a tile of n pairs (relative).  Every unit moves the same
+// bytes and, on the tensor cores, does the same work whatever n is.
+__host__ __device__ constexpr int tile_weight(int n) { return n > 0 ? 1 : 0; }
 
 struct GParams {
   int H, I, E, K, has_shared, has_rbias, nq, T;
   const uint8_t* experts;
   unsigned long long rec_bytes, o_gu_sb, o_d_q, o_d_sb;
   int qh, qi, sh, si;
-  int db;      // output rows per down unit
-  int ru;      // bytes of one ring slot
   const float* router;
   const float* rbias;
   const float* sgate;
@@ -75,23 +73,34 @@ struct GParams {
 };
 
 // ---------------------------------------------------------------- router
-// Block b: router rows [r0, r1) (the shared gate vector is row E), staged whole by
-// bulk copies; x of kRouterTok tokens at a time as floats.  Unit (row, split q) is a
-// warp; every lane accumulates its columns of each token in the single-token
+// Units are (row, column split q) in split-major order (u = q * rows + row; the shared
+// gate vector is row E), so a block's contiguous range of units touches at most a
+// couple of column splits.  Block b stages its units' router slices by bulk copies and,
+// kRouterTok tokens at a time, the activations of those splits as doubles (all loads
+// in flight); a warp per unit, every lane accumulating each token in the single-token
 // kernel's order, so the logits are bit-identical to that path.
+__host__ __device__ inline int router_splits_touched(int rows, int nq, int G) {
+  const int per = (rows * nq + G - 1) / G;  // units of the largest block
+  return min(nq, (per + rows - 1) / rows + 1);
+}
+
 __global__ void __launch_bounds__(kThreads, 1) grouped_router_kernel(const __grid_constant__ GParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   if (ld_relaxed_u32(p.err) != 0) return;
   const int rows = p.E + (p.has_shared ? 1 : 0);
   const int G = gridDim.x, b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r0 = static_cast<int>(static_cast<long long>(rows) * b / G);
-  const int r1 = static_cast<int>(static_cast<long long>(rows) * (b + 1) / G);
-  const int nr = r1 - r0;
+  const int U = rows * p.nq;
+  const int u0 = static_cast<int>(static_cast<long long>(U) * b / G);
+  const int u1 = static_cast<int>(static_cast<long long>(U) * (b + 1) / G);
+  const int nu = u1 - u0;
   const int H = p.H, hc = H / p.nq;
+  const int q0 = nu > 0 ? u0 / rows : 0;
+  const int nqs = nu > 0 ? (u1 - 1) / rows - q0 + 1 : 0;  // splits touched
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
-  float* wr = reinterpret_cast<float*>(smem + 128);
-  float* xt = wr + static_cast<size_t>(nr) * H;
+  float* wr = reinterpret_cast<float*>(smem + 128);               // [nu][hc]
+  double* xd = reinterpret_cast<double*>(smem + 128 + r128(static_cast<uint32_t>(nu) * hc * 4u));
+  // xd: [kRouterTok][nqs * hc] doubles of the touched splits
   __shared__ int fail;
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
@@ -99,55 +108,98 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_router_kernel(const __gri
     fail = 0;
   }
   __syncthreads();
-  if (threadIdx.x == 0 && nr > 0) {
+  if (nu == 0) return;
+  if (threadIdx.x == 0) {
     fence_proxy_async_smem();
-    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nr) * H * 4u);
-    for (int r = r0; r < r1; ++r)
-      bulk_g2s(wr + static_cast<size_t>(r - r0) * H, r < p.E ? p.router + static_cast<size_t>(r) * H : p.sgate,
-               static_cast<uint32_t>(H) * 4u, bar);
-    if (!mbar_wait_bounded(bar, 0, p.wait_ns, p.err)) fail = 1;
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nu) * hc * 4u);
+    for (int u = u0; u < u1; ++u) {
+      const int q = u / rows, r = u % rows;
+      const float* src = (r < p.E ? p.router + static_cast<size_t>(r) * H : p.sgate) + static_cast<size_t>(q) * hc;
+      bulk_g2s(wr + static_cast<size_t>(u - u0) * hc, src, static_cast<uint32_t>(hc) * 4u, bar);
+    }
   }
-  __syncthreads();
-  if (fail) return;
-  const int n4 = H / 4;
+  const int xw = nqs * hc / 2;  // double2 per staged token row in each of the two arrays
+  const int n4 = nqs * hc / 4;
+  // xa[t][k] = (x[4k], x[4k+1]), xb[t][k] = (x[4k+2], x[4k+3]) of the touched splits:
+  // a warp's 16-byte loads of consecutive k are conflict-free
+  double2* xa = reinterpret_cast<double2*>(xd);
+  double2* xb = xa + static_cast<size_t>(kRouterTok) * (xw / 2);
+  constexpr int KU = 8;
   for (int tg = 0; tg < p.T; tg += kRouterTok) {
     const int nt = min(kRouterTok, p.T - tg);
-    for (int i = threadIdx.x; i < nt * n4; i += kThreads) {
-      const int t = i / n4, q = i % n4;
-      const uint2 u = reinterpret_cast<const uint2*>(p.x + static_cast<size_t>(tg + t) * H)[q];
-      reinterpret_cast<float4*>(xt + static_cast<size_t>(t) * H)[q] =
-          make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
-                      __uint_as_float(u.y & 0xFFFF0000u));
-    }
-    __syncthreads();
-    for (int u = warp; u < nr * p.nq; u += kWarps) {
-      const int rl = u / p.nq, qq = u % p.nq;
-      const float4* wrow = reinterpret_cast<const float4*>(wr + static_cast<size_t>(rl) * H) + qq * (hc / 4);
-      double acc0[kRouterTok], acc1[kRouterTok];
+    if (tg > 0) __syncthreads();  // the previous group's activations are no longer read
+    for (int base = 0; base < nt * n4; base += KU * kThreads) {
+      uint2 v[KU];
 #pragma unroll
-      for (int t = 0; t < kRouterTok; ++t) acc0[t] = acc1[t] = 0.0;
+      for (int k = 0; k < KU; ++k) {
+        const int i = base + static_cast<int>(threadIdx.x) + k * kThreads;
+        v[k] = make_uint2(0u, 0u);
+        if (i < nt * n4) {
+          const int t = i / n4, c4 = i % n4;
+          v[k] = reinterpret_cast<const uint2*>(p.x + static_cast<size_t>(tg + t) * H + static_cast<size_t>(q0) * hc)[c4];
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < KU; ++k) {
+        const int i = base + static_cast<int>(threadIdx.x) + k * kThreads;
+        if (i < nt * n4) {
+          const int t = i / n4, c4 = i % n4;
+          xa[static_cast<size_t>(t) * n4 + c4] =
+              make_double2(__uint_as_float(v[k].x << 16), __uint_as_float(v[k].x & 0xFFFF0000u));
+          xb[static_cast<size_t>(t) * n4 + c4] =
+              make_double2(__uint_as_float(v[k].y << 16), __uint_as_float(v[k].y & 0xFFFF0000u));
+        }
+      }
+    }
+    if (tg == 0 && threadIdx.x == 0 && !mbar_wait_bounded(bar, 0, p.wait_ns, p.err)) fail = 1;
+    __syncthreads();
+    if (fail) return;
+    // a warp takes two units at a time (the same activation loads serve both rows)
+    for (int u = u0 + 2 * warp; u < u1; u += 2 * kWarps) {
+      const bool two = u + 1 < u1;
+      const int qa = u / rows, ra = u % rows;
+      const int ub = two ? u + 1 : u;
+      const int qb = ub / rows, rb = ub % rows;
+      const float4* wa = reinterpret_cast<const float4*>(wr + static_cast<size_t>(u - u0) * hc);
+      const float4* wb = reinterpret_cast<const float4*>(wr + static_cast<size_t>(ub - u0) * hc);
+      const int ka = (qa - q0) * (hc / 4), kb = (qb - q0) * (hc / 4);
+      double a0[kRouterTok], a1[kRouterTok], b0[kRouterTok], b1[kRouterTok];
+#pragma unroll
+      for (int t = 0; t < kRouterTok; ++t) a0[t] = a1[t] = b0[t] = b1[t] = 0.0;
       for (int k = lane; k < hc / 4; k += 32) {
-        const float4 wv = wrow[k];
+        const float4 va = wa[k];
+        const float4 vb = wb[k];
 #pragma unroll
         for (int t = 0; t < kRouterTok; ++t) {
           if (t < nt) {
-            const float4 xv = reinterpret_cast<const float4*>(xt + static_cast<size_t>(t) * H)[qq * (hc / 4) + k];
-            acc0[t] = fma(static_cast<double>(wv.x), static_cast<double>(xv.x), acc0[t]);
-            acc1[t] = fma(static_cast<double>(wv.y), static_cast<double>(xv.y), acc1[t]);
-            acc0[t] = fma(static_cast<double>(wv.z), static_cast<double>(xv.z), acc0[t]);
-            acc1[t] = fma(static_cast<double>(wv.w), static_cast<double>(xv.w), acc1[t]);
+            const double2 xa0 = xa[static_cast<size_t>(t) * n4 + ka + k];
+            const double2 xb0 = xb[static_cast<size_t>(t) * n4 + ka + k];
+            a0[t] = fma(static_cast<double>(va.x), xa0.x, a0[t]);
+            a1[t] = fma(static_cast<double>(va.y), xa0.y, a1[t]);
+            a0[t] = fma(static_cast<double>(va.z), xb0.x, a0[t]);
+            a1[t] = fma(static_cast<double>(va.w), xb0.y, a1[t]);
+            // the second unit usually shares the split (and so the loads)
+            const double2 xa1 = kb == ka ? xa0 : xa[static_cast<size_t>(t) * n4 + kb + k];
+            const double2 xb1 = kb == ka ? xb0 : xb[static_cast<size_t>(t) * n4 + kb + k];
+            b0[t] = fma(static_cast<double>(vb.x), xa1.x, b0[t]);
+            b1[t] = fma(static_cast<double>(vb.y), xa1.y, b1[t]);
+            b0[t] = fma(static_cast<double>(vb.z), xb1.x, b0[t]);
+            b1[t] = fma(static_cast<double>(vb.w), xb1.y, b1[t]);
           }
         }
       }
 #pragma unroll
       for (int t = 0; t < kRouterTok; ++t) {
         if (t < nt) {
-          const double l = warp_sum_d(acc0[t] + acc1[t]);
-          if (lane == 0) p.lpart[(static_cast<size_t>(tg + t) * rows + r0 + rl) * p.nq + qq] = l;
+          const double la = warp_sum_d(a0[t] + a1[t]);
+          const double lb = warp_sum_d(b0[t] + b1[t]);
+          if (lane == 0) {
+            p.lpart[(static_cast<size_t>(tg + t) * rows + ra) * p.nq + qa] = la;
+            if (two) p.lpart[(static_cast<size_t>(tg + t) * rows + rb) * p.nq + qb] = lb;
+          }
         }
       }
     }
-    __syncthreads();
   }
 }
 
@@ -183,7 +235,7 @@ __device__ __forceinline__ long long block_scan_excl(long long v, long long* wsu
 // ---------------------------------------------------------------- top-K + grouping
 struct TopkSmem {
   // byte offsets inside the dynamic shared memory
-  uint32_t slog, skey, ckey, cidx, sel, sidx, cnt, tn, wsum, misc;
+  uint32_t slog, skey, ckey, cidx, sel, sidx, mask, off, tn, wsum, misc;
 };
 
 __host__ __device__ inline TopkSmem topk_smem(int E, int K, int T, int has_shared, uint32_t* total) {
@@ -198,7 +250,8 @@ __host__ __device__ inline TopkSmem topk_smem(int E, int K, int T, int has_share
   s.cidx = o; o = r128(o + ngroups * K * 4u);
   s.sel = o; o = r128(o + (kMaxK + 1) * 4u);
   s.sidx = o; o = r128(o + T * K * 4u);
-  s.cnt = o; o = r128(o + E * 4u);
+  s.mask = o; o = r128(o + E * 8u);
+  s.off = o; o = r128(o + E * 4u);
   s.tn = o; o = r128(o + max_tiles * 4u);
   s.wsum = o; o = r128(o + (kWarps + 1) * 8u);
   s.misc = o; o = r128(o + 64u);
@@ -208,23 +261,30 @@ __host__ __device__ inline TopkSmem topk_smem(int E, int K, int T, int has_share
 
 // The last block: pairs grouped by expert (experts ascending, tokens ascending within
 // an expert, then the shared expert's pair of every token), tiles of <= kTileTok
-// pairs and the prefix sums of their work weights.
+// pairs and the prefix sums of their work weights.  A 64-bit token mask per expert
+// gives every pair its place without any serial scan: the pair (t, e) is number
+// popcount(mask[e] & ((1 << t) - 1)) of expert e.
 __device__ void build_groups(const GParams& p, uint8_t* smem, const TopkSmem& L) {
   const int E = p.E, K = p.K, T = p.T;
   int* sidx = reinterpret_cast<int*>(smem + L.sidx);
-  int* cnt = reinterpret_cast<int*>(smem + L.cnt);
+  unsigned long long* mask = reinterpret_cast<unsigned long long*>(smem + L.mask);
+  int* off = reinterpret_cast<int*>(smem + L.off);
   int* tn = reinterpret_cast<int*>(smem + L.tn);
   long long* wsum = reinterpret_cast<long long*>(smem + L.wsum);
-  for (int i = threadIdx.x; i < T * K; i += kThreads) sidx[i] = __ldcg(p.idx + i);
+  for (int e = threadIdx.x; e < E; e += kThreads) mask[e] = 0ull;
   __syncthreads();
-  // per-thread experts: a contiguous run of ceil(E / kThreads)
+  for (int i = threadIdx.x; i < T * K; i += kThreads) {
+    const int e = __ldcg(p.idx + i);
+    sidx[i] = e;
+    atomicOr(&mask[e], 1ull << (i / K));
+  }
+  __syncthreads();
+  // per-thread runs of ceil(E / kThreads) experts: pair and tile offsets
   const int per = (E + kThreads - 1) / kThreads;
   const int e0 = min(E, static_cast<int>(threadIdx.x) * per), e1 = min(E, e0 + per);
   long long npairs = 0, ntl = 0;
   for (int e = e0; e < e1; ++e) {
-    int c = 0;
-    for (int i = 0; i < T * K; ++i) c += sidx[i] == e;
-    cnt[e] = c;
+    const int c = __popcll(mask[e]);
     npairs += c;
     ntl += (c + kTileTok - 1) / kTileTok;
   }
@@ -234,18 +294,8 @@ __device__ void build_groups(const GParams& p, uint8_t* smem, const TopkSmem& L)
   {
     long long po = poff, to = toff0;
     for (int e = e0; e < e1; ++e) {
-      const int c = cnt[e];
-      // the pairs of expert e, tokens ascending
-      int j = 0;
-      for (int i = 0; i < T * K && j < c; ++i) {
-        if (sidx[i] == e) {
-          const int t = i / K, k = i % K;
-          const int pr = static_cast<int>(po) + j;
-          p.pair_token[pr] = t;
-          p.pidx[t * (K + 1) + k] = pr;
-          ++j;
-        }
-      }
+      const int c = __popcll(mask[e]);
+      off[e] = static_cast<int>(po);
       for (int i = 0; i * kTileTok < c; ++i) {
         const int n = min(kTileTok, c - i * kTileTok);
         p.tiles[to + i] = GTile{e, static_cast<int>(po) + i * kTileTok, n, 0};
@@ -254,6 +304,13 @@ __device__ void build_groups(const GParams& p, uint8_t* smem, const TopkSmem& L)
       po += c;
       to += (c + kTileTok - 1) / kTileTok;
     }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < T * K; i += kThreads) {
+    const int e = sidx[i], t = i / K, k = i % K;
+    const int pr = off[e] + __popcll(mask[e] & ((1ull << t) - 1ull));
+    p.pair_token[pr] = t;
+    p.pidx[t * (K + 1) + k] = pr;
   }
   const int routed_tiles = static_cast<int>(tot_tiles);
   const int PR = T * K;  // the shared expert's pairs follow the routed ones
@@ -343,11 +400,79 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_topk_kernel(const __grid_
 }
 
 // ---------------------------------------------------------------- grouped matvecs
+// Tensor-core (mma.sync m16n8k16, bf16 in, fp32 accumulate) dequantising matvecs of a
+// tile: M = 16 weight rows, N = 8 pairs of the tile, K = the row's columns.
+//
+// Exactness.  A code c enters the MMA as the bf16 value 1 + c/2^b' (b' = 4 for 4-bit
+// codes, 2 for 2-bit: the code placed in the top mantissa bits by one rotate and one
+// LOP3, no conversion), the activations as exact bf16 (x is bf16; h, fp32, is split
+// into hi = bf16(h) and lo = bf16(h - hi) and both are multiplied).  Every product is
+// exact in fp32.  Per 64-column group g the accumulator D_g = X_g + sum_c c*x_c/2^b'
+// (X_g = sum of the group's activations) is folded with the group's scale s and bias
+// b:  sum_c (s*c + b) x_c = (2^b' s) D_g + (b - 2^b' s) X_g, both coefficients exact.
+//
+// The K order inside each 16-column step is permuted (the same way for A and B) so
+// that one rotate of a code word yields the pair of codes a fragment register holds:
+// 4-bit, step columns c0..c0+15 (words w0 = c0..c0+7, w1 = c0+8..c0+15):
+//   k = 2q+j      <-> column c0 + q + 4j         (from w0)
+//   k = 8 + 2q+j  <-> column c0 + 8 + q + 4j     (from w1)
+// 2-bit, one word w = c0..c0+15:
+//   k = 2q+j      <-> column c0 + q + 8j
+//   k = 8 + 2q+j  <-> column c0 + q + 4 + 8j
+// where q = lane % 4 and j in {0, 1}.
+constexpr int kGWarps = 8;  // warps of a grouped matvec block
+constexpr int kGThreads = kGWarps * 32;
+constexpr int kPieceCols = 1024;  // columns of one staged piece of a unit's 16 rows
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The register holding codes (q, q+4) of a 4-bit word (low, high half) as bf16 1+c/16.
+__device__ __forceinline__ uint32_t codes4_bf16(uint32_t w, int q) {
+  return (__funnelshift_r(w, w, (4 * q - 3) & 31) & 0x00780078u) | 0x3F803F80u;
+}
+// Codes (q + 4h, q + 4h + 8) of a 2-bit word as bf16 1+c/4 (h = 0 or 1).
+__device__ __forceinline__ uint32_t codes2_bf16(uint32_t w, int q, int h) {
+  return (__funnelshift_r(w, w, (2 * q + 8 * h - 5) & 31) & 0x00600060u) | 0x3F803F80u;
+}
+
+// Shared-memory geometry of one grouped matvec phase (host and device).
+struct MvGeom {
+  int ncol;         // columns of a weight row
+  int kc;           // columns per piece
+  int npiece;       // pieces per unit
+  int R;            // units per tile
+  int code_stride;  // bytes per staged code row (padded: rows fall in different banks)
+  int sb_stride;    // bytes per staged (scale,bias) row (padded)
+  int piece_bytes;  // 16 rows of codes and (scale,bias)
+  int frag_bytes;   // staged activations in fragment order (hi and lo for down)
+  int sum_bytes;    // per-group activation sums
+};
+
+__host__ __device__ inline MvGeom mv_geom(bool down, int H, int I, int bits) {
+  MvGeom g;
+  g.ncol = down ? I : H;
+  g.kc = g.ncol < kPieceCols ? g.ncol : kPieceCols;
+  g.npiece = (g.ncol + g.kc - 1) / g.kc;
+  g.R = down ? H / 16 : I / 8;
+  g.code_stride = static_cast<int>(r16(static_cast<uint32_t>(g.kc * bits / 8))) + 16;
+  g.sb_stride = static_cast<int>(r16(static_cast<uint32_t>(g.kc / 64 * 4))) + 16;
+  g.piece_bytes = 16 * (g.code_stride + g.sb_stride);
+  g.frag_bytes = (down ? 2 : 1) * (g.ncol / 16) * 32 * 8;
+  g.sum_bytes = static_cast<int>(r128(static_cast<uint32_t>(g.ncol / 64 * kTileTok * 4)));
+  return g;
+}
+
 // Units of a phase: unit (tile i, row block r) of R row blocks per tile carries the
 // tile's work weight; block b takes the units whose position falls in its equal share
 // [b, b+1) * total / G of the weighted sequence.
 struct alignas(128) GHeader {
-  uint64_t bars[kWarps][kRing];
+  uint64_t bars[kGWarps][kRing];
   int seg_tile[kMaxSeg];
   int seg_ra[kMaxSeg];
   int seg_rb[kMaxSeg];
@@ -359,51 +484,45 @@ struct alignas(128) GHeader {
 
 template <int BITS, bool DOWN>
 struct GroupedKernel {
-  using C = Chunk<BITS>;
   const GParams& p;
+  MvGeom G;
   GHeader* hdr;
-  float* xs;    // [kTileTok][xstride] pre-scaled interleaved activations
-  float* xsum;  // [kTileTok][nch] chunk sums
+  uint32_t* frag;  // [ncol/16][32] uint2 (and the lo half after it for down)
+  float* xsum;     // [ncol/64][kTileTok]
   uint8_t* ring;
-  int ncol;     // columns of a row: H (gate/up) or I (down)
-  int nch;      // chunks of a row
-  uint32_t xstride;
-  int R;        // row blocks per tile
   int warp, lane;
 
   __device__ GroupedKernel(const GParams& pp, uint8_t* smem) : p(pp) {
     warp = threadIdx.x >> 5;
     lane = threadIdx.x & 31;
-    ncol = DOWN ? p.I : p.H;
-    nch = ncol / C::kCols;
-    xstride = static_cast<uint32_t>((nch + 31) / 32) * 32u * C::kCols;
-    R = DOWN ? (p.H + p.db - 1) / p.db : p.I;
+    G = mv_geom(DOWN, p.H, p.I, BITS);
     hdr = reinterpret_cast<GHeader*>(smem);
-    xs = reinterpret_cast<float*>(smem + sizeof(GHeader));
-    xsum = xs + kTileTok * xstride;
-    ring = smem + sizeof(GHeader) + r128(static_cast<uint32_t>(kTileTok) * (xstride + nch) * 4u);
+    frag = reinterpret_cast<uint32_t*>(smem + sizeof(GHeader));
+    xsum = reinterpret_cast<float*>(smem + sizeof(GHeader) + G.frag_bytes);
+    ring = smem + sizeof(GHeader) + G.frag_bytes + G.sum_bytes;
   }
 
   // ---- the block's segments: (tile, [ra, rb)) in tile order
   __device__ void plan_segments() {
     const int nt = __ldcg(p.ntiles);
     const long long Ctot = __ldcg(p.tcost + nt);
-    const int G = gridDim.x, b = blockIdx.x;
-    const long long X0 = Ctot * R * b / G, X1 = Ctot * R * (b + 1) / G;
+    const int NB = gridDim.x, b = blockIdx.x;
+    const long long R = G.R;
+    const long long X0 = Ctot * R * b / NB, X1 = Ctot * R * (b + 1) / NB;
     if (threadIdx.x == 0) {
       hdr->nseg = 0;
       hdr->first = 0;
       hdr->abort_flag = 0;
     }
     __syncthreads();
-    // rows of tile i at positions tcost[i]*R + r*w_i, r in [0, R)
+    // units of tile i at positions tcost[i]*R + r*w_i, r in [0, R)
     auto range = [&](int i, int& ra, int& rb) {
       const long long c0 = __ldcg(p.tcost + i) * R;
       const long long wi = __ldcg(p.tcost + i + 1) - __ldcg(p.tcost + i);
-      ra = X0 <= c0 ? 0 : static_cast<int>(min(static_cast<long long>(R), (X0 - c0 + wi - 1) / wi));
-      rb = X1 <= c0 ? 0 : static_cast<int>(min(static_cast<long long>(R), (X1 - c0 + wi - 1) / wi));
+      ra = X0 <= c0 ? 0 : static_cast<int>(min(R, (X0 - c0 + wi - 1) / wi));
+      rb = X1 <= c0 ? 0 : static_cast<int>(min(R, (X1 - c0 + wi - 1) / wi));
     };
-    for (int i = threadIdx.x; i < nt; i += kThreads) {
+    for (int i = threadIdx.x; i < nt; i += kGThreads) {
       int ra, rb;
       range(i, ra, rb);
       if (rb > ra) {
@@ -423,7 +542,7 @@ struct GroupedKernel {
       __syncthreads();
       return;
     }
-    for (int s = threadIdx.x; s < nseg; s += kThreads) {
+    for (int s = threadIdx.x; s < nseg; s += kGThreads) {
       int ra, rb;
       range(first + s, ra, rb);
       hdr->seg_tile[s] = first + s;
@@ -433,83 +552,113 @@ struct GroupedKernel {
     __syncthreads();
   }
 
-  // ---- this warp's units in order: segment s, row blocks ra + warp, ra + warp + kWarps, ...
+  // ---- this warp's pieces in order: segment s, units ra + warp, ra + warp + kGWarps, ...,
+  // pieces 0 .. npiece-1 of each
   struct It {
-    int s, r;
+    int s, u, pc;
   };
   __device__ __forceinline__ It norm(It it) const {
-    while (it.s < hdr->nseg && it.r >= hdr->seg_rb[it.s]) {
+    while (it.s < hdr->nseg && it.u >= hdr->seg_rb[it.s]) {
       ++it.s;
-      if (it.s < hdr->nseg) it.r = hdr->seg_ra[it.s] + warp;
+      if (it.s < hdr->nseg) it.u = hdr->seg_ra[it.s] + warp;
     }
     return it;
   }
-  __device__ __forceinline__ It first_unit() const {
-    return hdr->nseg > 0 ? norm(It{0, hdr->seg_ra[0] + warp}) : It{0, 0};
+  __device__ __forceinline__ It first_piece() const {
+    return hdr->nseg > 0 ? norm(It{0, hdr->seg_ra[0] + warp, 0}) : It{0, 0, 0};
   }
-  __device__ __forceinline__ It next_unit(It it) const { return norm(It{it.s, it.r + kWarps}); }
+  __device__ __forceinline__ It next_piece(It it) const {
+    if (it.pc + 1 < G.npiece) return It{it.s, it.u, it.pc + 1};
+    return norm(It{it.s, it.u + kGWarps, 0});
+  }
   __device__ __forceinline__ bool valid(It it) const { return it.s < hdr->nseg; }
 
   __device__ __forceinline__ uint8_t* slot_ptr(int slot) const {
-    return ring + (static_cast<uint32_t>(warp) * kRing + slot) * static_cast<uint32_t>(p.ru);
+    return ring + (static_cast<uint32_t>(warp) * kRing + slot) * static_cast<uint32_t>(G.piece_bytes);
   }
 
-  // bytes [src, src + n) as the 16-byte-aligned cover; returns the lead offset
-  __device__ __forceinline__ uint32_t cover(const uint8_t* base, unsigned long long off, uint32_t n,
-                                            const uint8_t** src, uint32_t* bytes) const {
-    const unsigned long long a = off & ~15ull;
-    const unsigned long long e = (off + n + 15ull) & ~15ull;
-    *src = base + a;
-    *bytes = static_cast<uint32_t>(e - a);
-    return static_cast<uint32_t>(off - a);
+  // staged row i (0..15) of unit u: source offsets of its code row piece and its
+  // (scale, bias) row piece inside the expert record
+  __device__ __forceinline__ void row_src(int u, int i, int pc, unsigned long long* qoff, unsigned long long* soff,
+                                          uint32_t* qbytes, uint32_t* sbytes) const {
+    const int c0 = pc * G.kc, cols = min(G.kc, G.ncol - c0);
+    *qbytes = static_cast<uint32_t>(cols * BITS / 8);
+    *sbytes = static_cast<uint32_t>(cols / 64 * 4);
+    if (DOWN) {
+      const unsigned long long j = static_cast<unsigned long long>(16 * u + i);
+      *qoff = p.o_d_q + j * p.qi + static_cast<unsigned long long>(c0 * BITS / 8);
+      *soff = p.o_d_sb + j * p.si + static_cast<unsigned long long>(c0 / 64 * 4);
+    } else {  // rows 0..7: gate rows 8u..8u+7, rows 8..15: the up rows of the same r
+      const unsigned long long r = static_cast<unsigned long long>(8 * u + (i & 7));
+      const unsigned long long up = i >= 8 ? 1ull : 0ull;
+      *qoff = r * 2u * p.qh + up * p.qh + static_cast<unsigned long long>(c0 * BITS / 8);
+      *soff = p.o_gu_sb + r * 2u * p.sh + up * p.sh + static_cast<unsigned long long>(c0 / 64 * 4);
+    }
   }
 
-  // lane 0: bulk copies of unit `it` into ring slot `slot`
+  // the whole warp: bulk copies of piece `it` into ring slot `slot` (lanes 0..15 the
+  // code rows, lanes 16..31 the 16-byte covers of the (scale, bias) rows)
   __device__ void issue(It it, int slot) {
     const GTile tl = p.tiles[hdr->seg_tile[it.s]];
     const uint8_t* rec = p.experts + static_cast<unsigned long long>(tl.expert) * p.rec_bytes;
     uint8_t* dst = slot_ptr(slot);
     uint64_t* bar = &hdr->bars[warp][slot];
-    const uint8_t* qsrc;
-    const uint8_t* ssrc;
-    uint32_t qb, sbb;
-    if (DOWN) {
-      const int j0 = it.r * p.db, n = min(p.H, j0 + p.db) - j0;
-      qsrc = rec + p.o_d_q + static_cast<unsigned long long>(j0) * p.qi;
-      qb = static_cast<uint32_t>(n) * p.qi;
-      cover(rec, p.o_d_sb + static_cast<unsigned long long>(j0) * p.si, static_cast<uint32_t>(n) * p.si, &ssrc, &sbb);
-    } else {
-      qsrc = rec + static_cast<unsigned long long>(it.r) * 2u * p.qh;
-      qb = 2u * p.qh;
-      cover(rec, p.o_gu_sb + static_cast<unsigned long long>(it.r) * 2u * p.sh, 2u * p.sh, &ssrc, &sbb);
-    }
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(bar, qb + sbb);
-    bulk_g2s(dst, qsrc, qb, bar);
-    bulk_g2s(dst + r16(qb), ssrc, sbb, bar);
+    const int i = lane & 15;
+    unsigned long long qoff, soff;
+    uint32_t qb, sb;
+    row_src(it.u, i, it.pc, &qoff, &soff, &qb, &sb);
+    const unsigned long long a = soff & ~15ull, e = (soff + sb + 15ull) & ~15ull;
+    const uint32_t bytes = lane < 16 ? qb : static_cast<uint32_t>(e - a);
+    const uint32_t total = __reduce_add_sync(0xffffffffu, bytes);
+    if (lane == 0) mbar_arrive_expect_tx(bar, total);
+    __syncwarp();
+    fence_proxy_async_smem();  // this lane's earlier reads of the slot before the copy
+    if (lane < 16)
+      bulk_g2s(dst + i * G.code_stride, rec + qoff, qb, bar);
+    else
+      bulk_g2s(dst + 16 * G.code_stride + i * G.sb_stride, rec + a, bytes, bar);
   }
 
-  // ---- activations of a tile: n rows (x rows of the tile's tokens, or h rows of its
-  // pairs), every load of the tile issued before any is used; pre-scaled values
-  // scattered into the interleaved layout, chunk sums by shuffles over the threads of
-  // a chunk (the single-token kernel's staging pattern)
+  // ---- activations of a tile in fragment order, every load issued before any use:
+  // x rows of the tile's tokens (bf16) or h rows of its pairs (fp32, split hi + lo);
+  // per-group sums by shuffles over the 16 threads of a 64-column group.  Pairs
+  // beyond the tile's count are zeros.
+  __device__ __forceinline__ uint32_t frag_half(int c, int n) const {
+    // 16-bit index of column c of pair n in the fragment array
+    const int ks = c >> 4, cc = c & 15;
+    int q, reg, j;
+    if (BITS == 4) {
+      reg = cc >> 3;
+      const int pos = cc & 7;
+      q = pos & 3;
+      j = pos >> 2;
+    } else {
+      j = cc >> 3;
+      const int r = cc & 7;
+      q = r & 3;
+      reg = r >> 2;
+    }
+    return static_cast<uint32_t>((((ks * 32 + 4 * n + q) * 2 + reg) * 2) + j);
+  }
+
   __device__ void stage_tile(const GTile& tl) {
-    constexpr int TPC = C::kCols / 4;
     constexpr int KU = 8;
-    const int n4 = ncol / 4;
-    const int total = tl.n * n4;
-    for (int base = 0; base < total; base += KU * kThreads) {  // block-uniform trip count
+    const int n4 = G.ncol / 4;
+    const int total = kTileTok * n4;
+    uint16_t* f16 = reinterpret_cast<uint16_t*>(frag);
+    uint16_t* f16lo = f16 + (G.ncol / 16) * 32 * 4;
+    for (int base = 0; base < total; base += KU * kGThreads) {  // block-uniform trip count
       float4 v[KU];
 #pragma unroll
       for (int k = 0; k < KU; ++k) {
-        const int i = base + static_cast<int>(threadIdx.x) + k * kThreads;
+        const int i = base + static_cast<int>(threadIdx.x) + k * kGThreads;
         v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i < total) {
-          const int j = i / n4, q = i % n4;
+        const int n = i / n4, q4 = i % n4;
+        if (i < total && n < tl.n) {
           if (DOWN) {
-            v[k] = __ldcg(reinterpret_cast<const float4*>(p.hbuf + static_cast<size_t>(tl.p0 + j) * p.I) + q);
+            v[k] = __ldcg(reinterpret_cast<const float4*>(p.hbuf + static_cast<size_t>(tl.p0 + n) * p.I) + q4);
           } else {
-            const uint2 u = reinterpret_cast<const uint2*>(p.x + static_cast<size_t>(hdr->tok[j]) * p.H)[q];
+            const uint2 u = reinterpret_cast<const uint2*>(p.x + static_cast<size_t>(hdr->tok[n]) * p.H)[q4];
             v[k] = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
                                __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
           }
@@ -517,125 +666,134 @@ struct GroupedKernel {
       }
 #pragma unroll
       for (int k = 0; k < KU; ++k) {
-        const int i = base + static_cast<int>(threadIdx.x) + k * kThreads;
+        const int i = base + static_cast<int>(threadIdx.x) + k * kGThreads;
         float sum = (v[k].x + v[k].y) + (v[k].z + v[k].w);
 #pragma unroll
-        for (int o = 1; o < TPC; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        for (int o = 1; o < 16; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         if (i < total) {
-          const int j = i / n4, q = i % n4, c0 = 4 * q;
-          float* d = xs + static_cast<size_t>(j) * xstride;
-          d[C::phys(c0 + 0)] = v[k].x * prescale_factor(C::shift_of(c0 + 0));
-          d[C::phys(c0 + 1)] = v[k].y * prescale_factor(C::shift_of(c0 + 1));
-          d[C::phys(c0 + 2)] = v[k].z * prescale_factor(C::shift_of(c0 + 2));
-          d[C::phys(c0 + 3)] = v[k].w * prescale_factor(C::shift_of(c0 + 3));
-          if (q % TPC == 0) xsum[j * nch + q / TPC] = sum;
-        }
-      }
-    }
-  }
-
-  // ---- per-lane partial sums of rows qa (and qb) against the n activation rows
-  template <bool TWO>
-  __device__ __forceinline__ void dot_tile(const uint8_t* qa, const uint32_t* sa, const uint8_t* qb,
-                                           const uint32_t* sb, int n, float (&ra)[kTileTok],
-                                           float (&rb)[kTileTok]) const {
+          const int n = i / n4, c = 4 * (i % n4);
+          const float vv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
-    for (int j = 0; j < kTileTok; ++j) ra[j] = rb[j] = 0.f;
-#pragma unroll 1
-    for (int m = lane; m < nch; m += 32) {
-      const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(qa + 16 * m);
-      ulonglong2 bq = make_ulonglong2(0ull, 0ull);
-      if (TWO) bq = *reinterpret_cast<const ulonglong2*>(qb + 16 * m);
-      const uint32_t swa = sa[C::sb_index(m)];
-      const uint32_t swb = TWO ? sb[C::sb_index(m)] : 0u;
-#pragma unroll
-      for (int j = 0; j < kTileTok; ++j) {
-        if (j < n) {
-          const float* vs = xs + static_cast<size_t>(j) * xstride;
-          const ulonglong2* xv0 = C::f4(vs, m, 0);
-          const ulonglong2* xv1 = C::f4(vs, m, C::kF4PerPair);
-          unsigned long long a0 = 0ull, a1 = 0ull, b0 = 0ull, b1 = 0ull;
-          C::template word_pair2<TWO>(a.x, bq.x, xv0, a0, b0);
-          C::template word_pair2<TWO>(a.y, bq.y, xv1, a1, b1);
-          const float vm = xsum[j * nch + m];
-          ra[j] = fmaf(sb_scale(swa), (pair_sum(a0) + pair_sum(a1)) * kUnscale, ra[j]);
-          ra[j] = fmaf(sb_bias(swa), vm, ra[j]);
-          if (TWO) {
-            rb[j] = fmaf(sb_scale(swb), (pair_sum(b0) + pair_sum(b1)) * kUnscale, rb[j]);
-            rb[j] = fmaf(sb_bias(swb), vm, rb[j]);
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t fi = frag_half(c + e, n);
+            const uint16_t hi = f32_to_bf16(vv[e]);
+            f16[fi] = hi;
+            if (DOWN) f16lo[fi] = f32_to_bf16(vv[e] - bf16_to_f32(hi));
           }
+          if ((i & 15) == 0) xsum[(c >> 6) * kTileTok + n] = sum;
         }
       }
     }
   }
 
-  // ---- consume unit `it` from ring slot `slot`
-  __device__ void consume(It it, int slot) {
-    const GTile tl = p.tiles[hdr->seg_tile[it.s]];
-    const uint8_t* sl = slot_ptr(slot);
-    float ra[kTileTok], rb[kTileTok];
-    if (DOWN) {
-      const int j0 = it.r * p.db, nrows = min(p.H, j0 + p.db) - j0;
-      const uint32_t qb = static_cast<uint32_t>(nrows) * p.qi;
-      const uint32_t lead = static_cast<uint32_t>((p.o_d_sb + static_cast<unsigned long long>(j0) * p.si) & 15ull);
-      const uint32_t* sbase = reinterpret_cast<const uint32_t*>(sl + r16(qb) + lead);
-      for (int i = 0; i < nrows; i += 2) {
-        const bool two = i + 1 < nrows;
-        if (two)
-          dot_tile<true>(sl + static_cast<uint32_t>(i) * p.qi, sbase + i * (p.si / 4),
-                         sl + static_cast<uint32_t>(i + 1) * p.qi, sbase + (i + 1) * (p.si / 4), tl.n, ra, rb);
-        else
-          dot_tile<false>(sl + static_cast<uint32_t>(i) * p.qi, sbase + i * (p.si / 4), nullptr, nullptr, tl.n, ra,
-                          rb);
+  // ---- one piece: 16 rows x the piece's columns against the tile's pairs, folded
+  // per group into acc (rows g and g+8 of the unit, pairs 2q and 2q+1)
+  __device__ __forceinline__ void piece(const uint8_t* sl, int u, int pc, float (&acc)[4]) const {
+    const int g = lane >> 2, q = lane & 3;
+    const int c0 = pc * G.kc, cols = min(G.kc, G.ncol - c0);
+    const uint8_t* ra = sl + g * G.code_stride;
+    const uint8_t* rb = sl + (g + 8) * G.code_stride;
+    unsigned long long qo, so;
+    uint32_t qb, sbb;
+    row_src(u, g, pc, &qo, &so, &qb, &sbb);
+    const uint32_t* sa = reinterpret_cast<const uint32_t*>(sl + 16 * G.code_stride + g * G.sb_stride + (so & 15ull));
+    row_src(u, g + 8, pc, &qo, &so, &qb, &sbb);
+    const uint32_t* sb = reinterpret_cast<const uint32_t*>(sl + 16 * G.code_stride + (g + 8) * G.sb_stride + (so & 15ull));
+    const uint2* fr = reinterpret_cast<const uint2*>(frag);
+    const uint2* frlo = fr + (G.ncol / 16) * 32;
+    constexpr float kScaleMul = BITS == 4 ? 16.0f : 4.0f;
+#pragma unroll 2
+    for (int grp = 0; grp < cols / 64; ++grp) {
+      // a group is 32 bytes of a 4-bit row (two 16-byte loads) or 16 of a 2-bit row
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      float e[4] = {0.f, 0.f, 0.f, 0.f};
+      const int ks0 = (c0 >> 4) + grp * 4;
+      if (BITS == 4) {
 #pragma unroll
-        for (int j = 0; j < kTileTok; ++j) {
-          if (j < tl.n) {
-            const float oa = warp_sum(ra[j]);
-            const float ob = two ? warp_sum(rb[j]) : 0.f;
-            if (lane == 0) {
-              float* o = p.obuf + static_cast<size_t>(tl.p0 + j) * p.H + j0 + i;
-              o[0] = oa;
-              if (two) o[1] = ob;
+        for (int half = 0; half < 2; ++half) {
+          const uint4 wa = *reinterpret_cast<const uint4*>(ra + grp * 32 + half * 16);
+          const uint4 wb = *reinterpret_cast<const uint4*>(rb + grp * 32 + half * 16);
+#pragma unroll
+          for (int st = 0; st < 2; ++st) {
+            const uint32_t a[4] = {codes4_bf16(st ? wa.z : wa.x, q), codes4_bf16(st ? wb.z : wb.x, q),
+                                   codes4_bf16(st ? wa.w : wa.y, q), codes4_bf16(st ? wb.w : wb.y, q)};
+            const int ks = ks0 + half * 2 + st;
+            const uint2 bh = fr[ks * 32 + lane];
+            float(&dd)[4] = (st == 0) ? d : e;
+            mma_bf16_16816(dd, a, bh.x, bh.y);
+            if (DOWN) {
+              const uint2 bl = frlo[ks * 32 + lane];
+              mma_bf16_16816(dd, a, bl.x, bl.y);
             }
           }
         }
-      }
-    } else {
-      const uint32_t lead =
-          static_cast<uint32_t>((p.o_gu_sb + static_cast<unsigned long long>(it.r) * 2u * p.sh) & 15ull);
-      const uint32_t* sg = reinterpret_cast<const uint32_t*>(sl + r16(2u * p.qh) + lead);
-      dot_tile<true>(sl, sg, sl + p.qh, sg + p.sh / 4, tl.n, ra, rb);
+      } else {
+        const uint4 wa = *reinterpret_cast<const uint4*>(ra + grp * 16);
+        const uint4 wb = *reinterpret_cast<const uint4*>(rb + grp * 16);
 #pragma unroll
-      for (int j = 0; j < kTileTok; ++j) {
-        if (j < tl.n) {
-          const float gv = warp_sum(ra[j]);
-          const float uv = warp_sum(rb[j]);
-          if (lane == 0) p.hbuf[static_cast<size_t>(tl.p0 + j) * p.I + it.r] = (gv / (1.0f + expf(-gv))) * uv;
+        for (int st = 0; st < 4; ++st) {
+          const uint32_t xa = st == 0 ? wa.x : st == 1 ? wa.y : st == 2 ? wa.z : wa.w;
+          const uint32_t xb = st == 0 ? wb.x : st == 1 ? wb.y : st == 2 ? wb.z : wb.w;
+          const uint32_t a[4] = {codes2_bf16(xa, q, 0), codes2_bf16(xb, q, 0), codes2_bf16(xa, q, 1),
+                                 codes2_bf16(xb, q, 1)};
+          const int ks = ks0 + st;
+          const uint2 bh = fr[ks * 32 + lane];
+          float(&dd)[4] = (st & 1) ? e : d;
+          mma_bf16_16816(dd, a, bh.x, bh.y);
+          if (DOWN) {
+            const uint2 bl = frlo[ks * 32 + lane];
+            mma_bf16_16816(dd, a, bl.x, bl.y);
+          }
         }
+      }
+      const float2 X = *reinterpret_cast<const float2*>(xsum + ((c0 >> 6) + grp) * kTileTok + 2 * q);
+      const uint32_t wsa = sa[grp], wsb = sb[grp];
+      const float s16a = kScaleMul * sb_scale(wsa), s16b = kScaleMul * sb_scale(wsb);
+      const float cba = sb_bias(wsa) - s16a, cbb = sb_bias(wsb) - s16b;
+      acc[0] = fmaf(s16a, d[0] + e[0], fmaf(cba, X.x, acc[0]));
+      acc[1] = fmaf(s16a, d[1] + e[1], fmaf(cba, X.y, acc[1]));
+      acc[2] = fmaf(s16b, d[2] + e[2], fmaf(cbb, X.x, acc[2]));
+      acc[3] = fmaf(s16b, d[3] + e[3], fmaf(cbb, X.y, acc[3]));
+    }
+  }
+
+  __device__ __forceinline__ void epilogue(const GTile& tl, int u, const float (&acc)[4]) const {
+    const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int n = 2 * q + j;
+      if (n >= tl.n) continue;
+      if (DOWN) {
+        float* o = p.obuf + static_cast<size_t>(tl.p0 + n) * p.H + 16 * u + g;
+        o[0] = acc[j];
+        o[8] = acc[2 + j];
+      } else {
+        const float gv = acc[j], uv = acc[2 + j];
+        p.hbuf[static_cast<size_t>(tl.p0 + n) * p.I + 8 * u + g] = (gv / (1.0f + expf(-gv))) * uv;
       }
     }
   }
 
   __device__ void run() {
     if (threadIdx.x == 0) {
-      for (int w = 0; w < kWarps; ++w)
+      for (int w = 0; w < kGWarps; ++w)
         for (int s = 0; s < kRing; ++s) mbar_init(&hdr->bars[w][s], 1);
       mbar_init_fence();
     }
     __syncthreads();
     plan_segments();
     if (hdr->abort_flag) return;
-    // prologue: the warp's first kRing units in flight
-    It pre = first_unit();
-    uint32_t issued = 0;  // units this warp has requested
+    // prologue: the warp's first kRing pieces in flight
+    It pre = first_piece();
+    uint32_t issued = 0;  // pieces this warp has requested
     for (int s = 0; s < kRing; ++s) {
       if (valid(pre)) {
-        if (lane == 0) issue(pre, s);
-        pre = next_unit(pre);
+        issue(pre, s);
+        pre = next_piece(pre);
         ++issued;
       }
     }
-    uint32_t k = 0;  // units this warp has consumed
+    uint32_t k = 0;  // pieces this warp has consumed
     bool ok = true;
     for (int s = 0; s < hdr->nseg; ++s) {
       const GTile tl = p.tiles[hdr->seg_tile[s]];
@@ -645,21 +803,25 @@ struct GroupedKernel {
       stage_tile(tl);
       __syncthreads();
       if (!ok) continue;
-      for (int r = hdr->seg_ra[s] + warp; r < hdr->seg_rb[s]; r += kWarps) {
-        const int slot = static_cast<int>(k % kRing);
-        const bool arrived = mbar_wait_bounded(&hdr->bars[warp][slot], (k / kRing) & 1u, p.wait_ns, p.err);
-        if (!__all_sync(0xffffffffu, arrived)) {
-          ok = false;
-          break;
+      for (int u = hdr->seg_ra[s] + warp; u < hdr->seg_rb[s] && ok; u += kGWarps) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int pc = 0; pc < G.npiece; ++pc) {
+          const int slot = static_cast<int>(k % kRing);
+          const bool arrived = mbar_wait_bounded(&hdr->bars[warp][slot], (k / kRing) & 1u, p.wait_ns, p.err);
+          if (!__all_sync(0xffffffffu, arrived)) {
+            ok = false;
+            break;
+          }
+          piece(slot_ptr(slot), u, pc, acc);
+          ++k;
+          __syncwarp();
+          if (valid(pre)) {
+            issue(pre, slot);
+            pre = next_piece(pre);
+            ++issued;
+          }
         }
-        consume(It{s, r}, slot);
-        ++k;
-        __syncwarp();
-        if (valid(pre)) {
-          if (lane == 0) issue(pre, slot);
-          pre = next_unit(pre);
-          ++issued;
-        }
+        if (ok) epilogue(tl, u, acc);
       }
     }
     // a warp that stopped early waits for the copies it still has in flight
@@ -671,27 +833,39 @@ struct GroupedKernel {
 };
 
 template <int BITS, bool DOWN>
-__global__ void __launch_bounds__(kThreads, 1) grouped_matvec_kernel(const __grid_constant__ GParams p) {
+__global__ void __launch_bounds__(kGThreads, 1) grouped_matvec_kernel(const __grid_constant__ GParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   if (ld_relaxed_u32(p.err) != 0) return;
   GroupedKernel<BITS, DOWN> G(p, smem);
   G.run();
 }
 
-// y[t][j] = resid[t][j] + sum_k w[t][k] o[pair(t, k)][j] + sigma_t o[pair(t, shared)][j]
+// y[t][j] = resid[t][j] + sum_k w[t][k] o[pair(t, k)][j] + sigma_t o[pair(t, shared)][j]:
+// block (column chunk, token) stages the token's pairs and weights once, then every
+// thread's K+1 output loads are independent.
 __global__ void grouped_combine_kernel(const __grid_constant__ GParams p) {
+  __shared__ int spi[kMaxK + 1];
+  __shared__ float sw[kMaxK + 1];
   if (ld_relaxed_u32(p.err) != 0) return;
   const int t = blockIdx.y;
+  const int ns = p.K + (p.has_shared ? 1 : 0);
+  if (threadIdx.x < ns) {
+    spi[threadIdx.x] = __ldcg(p.pidx + static_cast<size_t>(t) * (p.K + 1) + threadIdx.x);
+    sw[threadIdx.x] = threadIdx.x < p.K ? __ldcg(p.w + static_cast<size_t>(t) * p.K + threadIdx.x) : __ldcg(p.sig + t);
+  }
+  __syncthreads();
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= p.H) return;
-  const int* pi = p.pidx + static_cast<size_t>(t) * (p.K + 1);
+  float o[kMaxK + 1];
+#pragma unroll
+  for (int s = 0; s <= kMaxK; ++s)
+    if (s < ns) o[s] = __ldcg(p.obuf + static_cast<size_t>(spi[s]) * p.H + j);
   float pa = 0.f;
-  for (int k = 0; k < p.K; ++k)
-    pa = fmaf(__ldcg(p.w + static_cast<size_t>(t) * p.K + k), __ldcg(p.obuf + static_cast<size_t>(__ldcg(pi + k)) * p.H + j),
-              pa);
-  if (p.has_shared) pa = fmaf(__ldcg(p.sig + t), __ldcg(p.obuf + static_cast<size_t>(__ldcg(pi + p.K)) * p.H + j), pa);
-  const size_t o = static_cast<size_t>(t) * p.H + j;
-  p.y[o] = f32_to_bf16(bf16_to_f32(p.resid[o]) + pa);
+#pragma unroll
+  for (int s = 0; s <= kMaxK; ++s)
+    if (s < ns) pa = fmaf(sw[s], o[s], pa);
+  const size_t oi = static_cast<size_t>(t) * p.H + j;
+  p.y[oi] = f32_to_bf16(bf16_to_f32(p.resid[oi]) + pa);
 }
 
 }  // namespace fmoe
