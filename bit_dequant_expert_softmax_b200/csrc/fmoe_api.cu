@@ -1,5 +1,6 @@
 // Host side of libfmoe.so: validation, the layer handle, workspace layout and
 // kernel launches for the C ABI declared in include/fmoe.h.
+#include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -169,8 +170,9 @@ fmoe_status plan(fmoe_layer* L) {
   const uint32_t staging = (uint32_t)kMaxSmem - fixed;
   const int G = L->sms;
   // P1: x in doubles and the router rows a block touches from the start of the
-  // staging area, its shared gate/up rows at the end; top-K's logits and
-  // candidates must not reach the shared rows either (they are consumed after it)
+  // staging area, its shared gate/up rows at the end (both in flight together); the
+  // shared rows are consumed before top-K, whose logits and candidates then may use
+  // the whole area
   const long long U = (long long)(c.n_experts + c.has_shared) * L->nq;
   const uint32_t rows_touched = (uint32_t)(((U + G - 1) / G + L->nq - 1) / L->nq + 1);
   const int shared_rows = (c.inter + G - 1) / G;
@@ -182,7 +184,7 @@ fmoe_status plan(fmoe_layer* L) {
   // top-K: logits, selection keys, per-warp candidates
   if ((uint64_t)r128((uint32_t)(c.n_experts + 1) * 8u) + (uint64_t)((c.n_experts + 15) & ~15) * 8u +
           (uint64_t)((c.n_experts + 31) / 32) * c.top_k * 12u >
-      sc_off)
+      staging)
     return FMOE_ERR_UNSUPPORTED;
   // P2: at least one gate/up row pair per round
   if (g.gu_bytes(1) > staging) return FMOE_ERR_UNSUPPORTED;
@@ -237,24 +239,44 @@ Params base_params(const fmoe_layer* L, int mode, int T) {
   return p;
 }
 
+// Programmatic dependent launch with the cooperative launch: the next layer call is
+// launched while this one runs and its blocks start as SMs free up (each waits for the
+// previous grid's completion before touching any data).  Dropped for the rest of the
+// process if the runtime refuses the combination.
+std::atomic<int> g_pdl_ok{1};
+
 fmoe_status launch(const fmoe_layer* L, const Params& p, void* stream) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(L->sms);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = L->smem_bytes;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e;
-  if (L->cfg.bits == 4)
-    e = p.norm ? cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<4, true>, p)
-               : cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<4, false>, p);
-  else
-    e = p.norm ? cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<2, true>, p)
-               : cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<2, false>, p);
+  auto go = [&]() {
+    if (L->cfg.bits == 4)
+      return p.norm ? cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<4, true>, p)
+                    : cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<4, false>, p);
+    return p.norm ? cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<2, true>, p)
+                  : cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<2, false>, p);
+  };
+  cudaError_t e = cudaErrorNotSupported;
+  if (g_pdl_ok.load(std::memory_order_relaxed)) {
+    cfg.numAttrs = 2;
+    e = go();
+    if (e != cudaSuccess) {
+      cudaGetLastError();  // clear the launch error and fall back for good
+      g_pdl_ok.store(0, std::memory_order_relaxed);
+    }
+  }
+  if (e != cudaSuccess) {
+    cfg.numAttrs = 1;
+    e = go();
+  }
   return e == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
 }
 

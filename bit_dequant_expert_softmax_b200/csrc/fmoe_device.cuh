@@ -123,13 +123,18 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Waits for phase `parity` of `bar` to complete, for at most limit_ns.
+// Waits for phase `parity` of `bar` to complete, for at most limit_ns.  Between polls
+// the warp sleeps, so that waiting warps leave the issue slots to computing ones.
+#ifndef FMOE_WAIT_SLEEP_NS
+#define FMOE_WAIT_SLEEP_NS 64
+#endif
 __device__ __noinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                                uint32_t* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    __nanosleep(FMOE_WAIT_SLEEP_NS);
+    if (mbar_try_wait(bar, parity)) return true;
     if (global_timer_ns() - t0 > limit_ns) {
       atomicOr(err, FMOE_DEVERR_COPY_TIMEOUT);
       return false;

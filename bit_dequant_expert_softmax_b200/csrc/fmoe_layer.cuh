@@ -74,15 +74,32 @@ struct Params {
   int timeline_token;
 };
 
+// Rows [ra, rb) of expert slot `slot`, staged at `off`, copy items from `first`.
+struct GuChunk {
+  int slot, ra, rb;
+  uint32_t off, first;
+};
+
+// The block's share of a token's expert work (the same for every token of a launch):
+// routed gate/up chunks (item numbers relative to the token's first routed item), the
+// down rows, and where the down rows and h are staged.
+struct ExpertPlan {
+  GuChunk ch[kMaxChunks];
+  int nc, gitems, ndown, j0, j1, v0, v1, prefetch;
+  uint32_t doff, hoff;
+};
+
 // Shared-memory header (activations and the staging area follow it).
 struct alignas(128) SmemHeader {
   uint64_t bars[kNumBars];
   double red[kWarps];    // per-warp partial sums (RMS normalisation)
+  double selog[kMaxK + 1];  // logits of the selection in rank order; slot K: shared gate
   int sel[kMaxK + 1];    // expert of each slot (slot K = shared expert)
   float wsl[kMaxK + 1];  // weight of each slot (w_k; slot K = sigma)
   int abort_flag;
   int skip_token;
   uint32_t tok_base;
+  ExpertPlan plan;
 };
 
 __host__ __device__ constexpr uint32_t r16(uint32_t n) { return (n + 15u) & ~15u; }
@@ -121,11 +138,6 @@ struct Geometry {
   __host__ __device__ uint32_t router_item() const { return static_cast<uint32_t>(H) * 4u; }
 };
 
-// Rows [ra, rb) of expert slot `slot`, staged at `off`, copy items from `first`.
-struct GuChunk {
-  int slot, ra, rb;
-  uint32_t off, first;
-};
 
 // NORM: the input is a pre-norm block's h, RMS-normalised while it is staged.
 template <int BITS, bool NORM>
@@ -417,15 +429,16 @@ struct LayerKernel {
   }
 
   // Warp 0: issue every item of `nc` chunks, one lane per item.
+  // Thread 0: every item of `nc` chunks, one after another in the order the warps
+  // consume them (copies requested in one instruction by many lanes are served
+  // interleaved and all complete late; requested in sequence, the first ones land
+  // first).
   __device__ void issue_gu(const GuChunk* ch, int nc) {
-    if (threadIdx.x >= 32) return;
+    if (threadIdx.x != 0) return;
     fence_proxy_async_smem();
-    int base = 0;
     for (int k = 0; k < nc; ++k) {
       const int items = g.gu_items(ch[k].rb - ch[k].ra);
-      for (int i = static_cast<int>(threadIdx.x) - base; i < items; i += 32)
-        if (i >= 0) issue_gu_item(ch[k], i);
-      base = (base + items) % 32;
+      for (int i = 0; i < items; ++i) issue_gu_item(ch[k], i);
     }
   }
 
@@ -451,15 +464,19 @@ struct LayerKernel {
     return true;
   }
 
-  // Consume every row pair of `nc` chunks, spread over the warps (unit u -> warp u % kWarps).
-  __device__ void gu_consume(const GuChunk* ch, int nc, int buf) {
+  // Consume every row pair of `nc` chunks, spread over warps w0 .. kWarps-1 (unit u ->
+  // warp w0 + u % (kWarps - w0)); w0 = 1 keeps warp 0, which issues the copies and
+  // computes the routing weights meanwhile, out of the routed rows.
+  __device__ void gu_consume(const GuChunk* ch, int nc, int buf, int w0 = 0) {
     const int warp = threadIdx.x >> 5;
+    if (warp < w0) return;
+    const int nw = kWarps - w0;
     int base = 0;
     for (int k = 0; k < nc; ++k) {
       const int n = ch[k].rb - ch[k].ra;
-      int first = (warp - base) % kWarps;
-      if (first < 0) first += kWarps;
-      for (int i = first; i < n; i += kWarps) {
+      int first = (warp - w0 - base) % nw;
+      if (first < 0) first += nw;
+      for (int i = first; i < n; i += nw) {
         if (!gu_unit(ch[k], ch[k].ra + i, buf)) {
           hdr->abort_flag = 1;
           return;
@@ -540,9 +557,9 @@ struct LayerKernel {
 
   // Warp 0: items [ka, kb) of the block's rows [j0, j1) from staging offset `base`.
   __device__ void issue_down_items(int j0, int j1, int ka, int kb, uint32_t first, uint32_t base) {
-    if (threadIdx.x >= 32) return;
+    if (threadIdx.x != 0) return;
     fence_proxy_async_smem();
-    for (int k = ka + static_cast<int>(threadIdx.x); k < kb; k += 32) {
+    for (int k = ka; k < kb; ++k) {
       const int ja = j0 + k * p.db, n = min(j1, ja + p.db) - ja;
       issue_down(first + (k - ka), base + (k - ka) * g.dn_item(p.db), ja, n);
     }
@@ -692,7 +709,6 @@ struct LayerKernel {
     }
     mark(10);
     const int rows = p.E + (p.has_shared ? 1 : 0);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     double* slog = reinterpret_cast<double*>(stage);
     unsigned long long* skey = reinterpret_cast<unsigned long long*>(stage + r128(static_cast<uint32_t>(rows) * 8u));
     unsigned long long* ckey = skey + ((p.E + 15) & ~15);
@@ -709,23 +725,31 @@ struct LayerKernel {
     rank_topk<kThreads>(skey, ckey, cidx, p.E, p.K, hdr->sel);
     mark(12);
     mark(13);
-    if (warp == 0) {
-      const double wk = topk_weight(slog, hdr->sel, p.K, lane);
-      if (lane < p.K) {
-        const int mysel = hdr->sel[lane];
-        hdr->wsl[lane] = static_cast<float>(wk);
-        if (blockIdx.x == 0 && p.idx_out) {
-          p.idx_out[static_cast<size_t>(t) * p.K + lane] = mysel;
-          p.w_out[static_cast<size_t>(t) * p.K + lane] = static_cast<float>(wk);
-        }
-      }
-      if (lane == 0 && p.has_shared) {
-        const double sig = 1.0 / (1.0 + exp(-slog[p.E]));
-        hdr->wsl[p.K] = static_cast<float>(sig);
-        if (blockIdx.x == 0 && p.sig_out) p.sig_out[t] = static_cast<float>(sig);
+    // keep the selection's logits: the staging area is about to receive the rows
+    if (threadIdx.x <= p.K)
+      hdr->selog[threadIdx.x] =
+          threadIdx.x < p.K ? slog[hdr->sel[threadIdx.x]] : (p.has_shared ? slog[p.E] : 0.0);
+    __syncthreads();
+  }
+
+  // Warp 0: the renormalised softmax weights of the selection and the shared sigmoid
+  // gate (needed only by the combine, so computed while the selected rows fly).
+  __device__ void route_weights(int t) {
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    const double wk = topk_weight_sorted(hdr->selog, p.K, lane);
+    if (lane < p.K) {
+      hdr->wsl[lane] = static_cast<float>(wk);
+      if (blockIdx.x == 0 && p.idx_out) {
+        p.idx_out[static_cast<size_t>(t) * p.K + lane] = hdr->sel[lane];
+        p.w_out[static_cast<size_t>(t) * p.K + lane] = static_cast<float>(wk);
       }
     }
-    __syncthreads();
+    if (lane == 0 && p.has_shared) {
+      const double sig = 1.0 / (1.0 + exp(-hdr->selog[p.K]));
+      hdr->wsl[p.K] = static_cast<float>(sig);
+      if (blockIdx.x == 0 && p.sig_out) p.sig_out[t] = static_cast<float>(sig);
+    }
   }
 
   // Routing given by the caller (expert-forward entry point).
@@ -746,46 +770,57 @@ struct LayerKernel {
   }
 
   // ---------------------------------------------------------------- P2 + P3
-  __device__ bool experts(int buf, const uint16_t* resid_t, uint16_t* y_t) {
+  // The block's expert work plan: the same for every token, computed once per launch.
+  __device__ void plan_experts() {
+    ExpertPlan& pl = hdr->plan;
     const int G = gridDim.x, b = blockIdx.x;
-    const int v0 = static_cast<int>(static_cast<long long>(p.K) * p.I * b / G);
-    const int v1 = static_cast<int>(static_cast<long long>(p.K) * p.I * (b + 1) / G);
-    int j0, j1;
-    down_range(j0, j1);
-    const int ndown = (j1 - j0 + p.db - 1) / p.db;
-    // plan: routed gate/up chunks from offset 0, down items behind them (issued once
-    // the shared expert's rows at the end of the area are consumed), h at offset 0
-    GuChunk ch[kMaxChunks];
+    pl.v0 = static_cast<int>(static_cast<long long>(p.K) * p.I * b / G);
+    pl.v1 = static_cast<int>(static_cast<long long>(p.K) * p.I * (b + 1) / G);
+    down_range(pl.j0, pl.j1);
+    pl.ndown = (pl.j1 - pl.j0 + p.db - 1) / p.db;
+    // routed gate/up chunks from offset 0, down items behind them, h at offset 0 (the
+    // whole staging area is free: the shared expert's rows are consumed before top-K)
     int nc = 0, gitems = 0;
     uint32_t gtotal = 0;
-    int vend = v0;
-    while (vend < v1 && nc < kMaxChunks) {
-      const int s = vend / p.I, r = vend % p.I, n = min(v1 - vend, p.I - r);
-      ch[nc++] = GuChunk{s, r, r + n, gtotal, nitem + static_cast<uint32_t>(gitems)};
+    int vend = pl.v0;
+    while (vend < pl.v1 && nc < kMaxChunks) {
+      const int s = vend / p.I, r = vend % p.I, n = min(pl.v1 - vend, p.I - r);
+      pl.ch[nc++] = GuChunk{s, r, r + n, gtotal, static_cast<uint32_t>(gitems)};
       gitems += g.gu_items(n);
       gtotal = r128(gtotal + g.gu_bytes(n));
       vend += n;
     }
-    const uint32_t doff = gtotal, dtotal = g.dn_total(j1 - j0);
-    const uint32_t hoff = g.h_bytes() <= doff ? 0u : r128(doff + dtotal);
-    const bool prefetch = (vend >= v1) && (!has_sc_ || gtotal <= sc_.off) && (doff + dtotal <= cap) &&
-                          (hoff + g.h_bytes() <= cap) && (gitems + ndown <= kMaxRoundItems);
-    const uint32_t down_first = nitem + static_cast<uint32_t>(gitems);
+    pl.nc = nc;
+    pl.gitems = gitems;
+    pl.doff = gtotal;
+    const uint32_t dtotal = g.dn_total(pl.j1 - pl.j0);
+    pl.hoff = g.h_bytes() <= pl.doff ? 0u : r128(pl.doff + dtotal);
+    pl.prefetch = (vend >= pl.v1) && (pl.doff + dtotal <= cap) && (pl.hoff + g.h_bytes() <= cap) &&
+                  (gitems + pl.ndown <= kMaxRoundItems);
+  }
+
+  __device__ bool experts(int buf, bool route, const uint16_t* resid_t, uint16_t* y_t) {
+    const ExpertPlan& pl = hdr->plan;
+    const int j0 = pl.j0, j1 = pl.j1, ndown = pl.ndown;
+    const bool prefetch = pl.prefetch != 0;
+    const uint32_t doff = pl.doff, hoff = pl.hoff;
+    const uint32_t down_first = nitem + static_cast<uint32_t>(pl.gitems);
     if (prefetch) {
-      issue_gu(ch, nc);
-      nitem += static_cast<uint32_t>(gitems);
-      if (has_sc_) gu_consume(&sc_, 1, buf);
-      __syncthreads();
+      GuChunk ch[kMaxChunks];
+      for (int k = 0; k < pl.nc; ++k) {
+        ch[k] = pl.ch[k];
+        ch[k].first += nitem;
+      }
+      issue_gu(ch, pl.nc);
       issue_down_items(j0, j1, 0, ndown, down_first, doff);
-      nitem += static_cast<uint32_t>(ndown);
-      gu_consume(ch, nc, buf);
+      nitem += static_cast<uint32_t>(pl.gitems + ndown);
+      if (route) route_weights(tok_);
+      gu_consume(ch, pl.nc, buf, 1);
       __syncthreads();
       if (hdr->abort_flag) return false;
     } else {
-      if (has_sc_) gu_consume(&sc_, 1, buf);
-      __syncthreads();
-      if (hdr->abort_flag) return false;
-      if (!gu_rounds(v0, v1, buf)) return false;
+      if (route) route_weights(tok_);
+      if (!gu_rounds(pl.v0, pl.v1, buf)) return false;
     }
     publish(p.hflags, tok_);
     mark(5);
@@ -832,13 +867,17 @@ struct LayerKernel {
 
   // ---------------------------------------------------------------- driver
   __device__ void run() {
-    if (threadIdx.x == 0) {
-      for (int i = 0; i < kNumBars; ++i) mbar_init(&hdr->bars[i], 1);
+    if (threadIdx.x < 32) {  // warp 0: barriers; warp 1 meanwhile: the expert plan
+      for (int i = static_cast<int>(threadIdx.x); i < kNumBars; i += 32) mbar_init(&hdr->bars[i], 1);
       mbar_init_fence();
-      hdr->abort_flag = 0;
-      hdr->skip_token = 0;
-      hdr->sel[p.K] = p.E;  // the shared expert's record
-      hdr->tok_base = ld_relaxed_u32(p.tokens);
+      if (threadIdx.x == 0) {
+        hdr->abort_flag = 0;
+        hdr->skip_token = 0;
+        hdr->sel[p.K] = p.E;  // the shared expert's record
+        hdr->tok_base = ld_relaxed_u32(p.tokens);
+      }
+    } else if (threadIdx.x == 32 && p.mode != MODE_ROUTE) {
+      plan_experts();
     }
     const uint32_t err0 = ld_relaxed_u32(p.err);
     __syncthreads();
@@ -867,13 +906,20 @@ struct LayerKernel {
       if (!phase1_consume(buf, route)) break;
       if (route) publish(p.rflags, t);
       mark(2);
+      if (has_sc_) {  // the shared expert does not depend on the routing: its gate/up
+        gu_consume(&sc_, 1, buf);  // rows are consumed while the router partials travel
+        __syncthreads();
+        if (hdr->abort_flag) break;
+      }
       if (route) {
         topk(buf, t);
         if (hdr->abort_flag) break;
+        if (!do_experts) route_weights(t);  // otherwise computed while the rows fly
         mark(4);
       }
       if (do_experts) {
-        if (!experts(buf, p.resid + static_cast<size_t>(t) * p.H, p.y + static_cast<size_t>(t) * p.H)) break;
+        if (!experts(buf, route, p.resid + static_cast<size_t>(t) * p.H, p.y + static_cast<size_t>(t) * p.H))
+          break;
         mark(9);
       }
     }
@@ -890,6 +936,11 @@ struct LayerKernel {
 template <int BITS, bool NORM>
 __global__ void __launch_bounds__(kThreads, 1) fmoe_layer_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
+  // launched with programmatic stream serialization: let the next call's launch begin
+  // now, and wait until the previous grid has completed (its outputs and this layer's
+  // workspace) before reading anything (both are no-ops otherwise)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   LayerKernel<BITS, NORM> L(p, smem);
   L.run();
 }

@@ -90,4 +90,11 @@ __device__ __forceinline__ double topk_weight(const double* slog, const int* sel
   return ek / den;
 }
 
+// The same weight from the selection's logits already in rank order (l[0] largest).
+__device__ __forceinline__ double topk_weight_sorted(const double* l, int K, int lane) {
+  const double ek = lane < K ? exp(l[lane] - l[0]) : 0.0;
+  const double den = warp_sum_d(ek);
+  return ek / den;
+}
+
 }  // namespace fmoe
