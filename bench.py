@@ -355,7 +355,7 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
-    if synth.CONFIGS[args.config]["layers"] > 1:
+    if synth.CONFIGS[args.config]["layers"] > 1 or synth.CONFIGS[args.config]["batch"] > 1:
         bench_stack(args, world, rank)
         if world > 1:
             dist.destroy_process_group()

@@ -354,4 +354,6 @@ CONFIGS = {
     "stack24_4bit": dict(shape=LayerShape(4096, 1024, 512, 4, 4, 1, 0), layers=24, tokens=256, batch=1),
     "stack60_2bit": dict(shape=LayerShape(4096, 1024, 512, 4, 2, 1, 0), layers=60, tokens=128, batch=1),
     "stack16_batched": dict(shape=LayerShape(4096, 1024, 512, 10, 4, 1, 1), layers=16, tokens=2048, batch=32),
+    # one layer of the batched stack, one 32-token step (a profiling case of the batched path)
+    "batched_layer_k10": dict(shape=LayerShape(4096, 1024, 512, 10, 4, 1, 1), layers=1, tokens=32, batch=32),
 }
