@@ -111,7 +111,7 @@ def profiled_traffic():
     the kernel source is the one that was profiled (else None)."""
     import hashlib
     src = [os.path.join(ROOT, "bit_dequant_expert_softmax_b200", "csrc", f)
-           for f in ("fmoe_layer.cuh", "fmoe_device.cuh")]
+           for f in ("fmoe_layer.cuh", "fmoe_device.cuh", "fmoe_topk.cuh")]
     h = hashlib.sha256()
     for f in src:
         with open(f, "rb") as fh:

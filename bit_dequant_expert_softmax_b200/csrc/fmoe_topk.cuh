@@ -63,19 +63,27 @@ __device__ __forceinline__ void rank_topk(const unsigned long long* skey, unsign
     }
   }
   __syncthreads();
+  // every candidate's rank is counted by kStripe consecutive lanes, each over every
+  // kStripe-th candidate, and summed by shuffles
+  constexpr int kStripe = 8;
   const int ncand = ngroups * K;
-  for (int c = threadIdx.x; c < ncand; c += NTHREADS) {
-    const unsigned long long kc = ckey[c];
-    const int ic = cidx[c];
-    if (kc == 0) continue;
-    int rank = 0;
-#pragma unroll 8
-    for (int j = 0; j < ncand; ++j) {
-      const unsigned long long kj = ckey[j];
-      const int ij = cidx[j];
-      rank += static_cast<int>(kj > kc) | (static_cast<int>(kj == kc) & static_cast<int>(ij < ic));
+  for (int base = 0; base < ncand * kStripe; base += NTHREADS) {  // block-uniform trip count
+    const int i = base + static_cast<int>(threadIdx.x);
+    const int c = i / kStripe, part = i % kStripe;
+    unsigned long long kc = 0;
+    int ic = 0, rank = 0;
+    if (c < ncand) {
+      kc = ckey[c];
+      ic = cidx[c];
+      for (int j = part; j < ncand; j += kStripe) {
+        const unsigned long long kj = ckey[j];
+        const int ij = cidx[j];
+        rank += static_cast<int>(kj > kc) | (static_cast<int>(kj == kc) & static_cast<int>(ij < ic));
+      }
     }
-    if (rank < K) sel[rank] = ic;
+#pragma unroll
+    for (int o = 1; o < kStripe; o <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+    if (c < ncand && part == 0 && kc != 0 && rank < K) sel[rank] = ic;
   }
   __syncthreads();
 }
