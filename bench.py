@@ -130,6 +130,23 @@ def profiled_traffic():
     return traffic if want == h.hexdigest() else None
 
 
+def max_over_ranks(value: float, world: int, device="cuda") -> float:
+    """The largest of every rank's `value` (the timed region of a multi-rank run is the
+    slowest rank's); every rank must call it, in the same order."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: float, world: int, slowest_ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (slowest_ms / 1e3)
+
+
 def layer_bytes(shape):
     """Algorithmic bytes of one single-token layer forward."""
     import fmoe_synth as synth
@@ -256,10 +273,7 @@ def bench_stack(args, world, rank):
     barrier()
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
-    t = torch.tensor([sum(step_ms)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world)
     errs = [L.error() for L in layers]
     if any(errs):
         raise RuntimeError(f"device-side error bits {errs} during the benchmark")
@@ -276,10 +290,7 @@ def bench_stack(args, world, rank):
             ho.copy_(h, non_blocking=True)
         e_e.record(stream)
     barrier()
-    te = torch.tensor([e_s.elapsed_time(e_e)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), world)
 
     rb = synth.record_bytes(H, shape.inter, shape.bits)
     router_b = shape.n_experts * H * 4 + (H * 4 if shape.has_shared else 0)
@@ -303,7 +314,7 @@ def bench_stack(args, world, rank):
     peak, peak_kind = measured_peaks()
     step_s = total_ms / 1e3 / args.steps
     achieved = step_bytes / step_s / 1e9
-    value = tokens * args.steps * world / (total_ms / 1e3)
+    value = job_rate(tokens * args.steps, world, total_ms)
     if rank == 0:
         launches_per_layer = 1 if B == 1 else 6
         line = {"metric": f"{NL}-layer stack decode tokens/s", "value": value, "unit": "tokens/s",
@@ -316,7 +327,7 @@ def bench_stack(args, world, rank):
                                        + ("one at a time" if B == 1 else f"in steps of {B} grouped by expert"),
                            "tokens_per_step": tokens, "l2": "flushed between steps (512 MiB write)",
                            "parallelism": f"replicas x{world}"},
-                "e2e": {"value": tokens * args.steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                "e2e": {"value": job_rate(tokens * args.steps, world, e2e_ms), "unit": "tokens/s",
                         "h2d_bytes_per_step": hh.numel() * 2, "d2h_bytes_per_step": ho.numel() * 2},
                 "gpu_launches": args.steps * NL * (tokens if B == 1 else -(-tokens // B) * launches_per_layer),
                 "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -412,10 +423,7 @@ def main():
     clocks = sampler.stop()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world)
     err = L.error()
     if err:
         raise RuntimeError(f"device-side error bits {err:#x} during the benchmark")
@@ -434,15 +442,10 @@ def main():
             yh.copy_(y, non_blocking=True)
         e_e.record(stream)
     barrier()
-    e2e_ms = e_s.elapsed_time(e_e)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), world)
 
-    total_tokens = tokens * args.steps * world
-    value = total_tokens / (total_ms / 1e3)
-    e2e_value = total_tokens / (e2e_ms / 1e3)
+    value = job_rate(tokens * args.steps, world, total_ms)
+    e2e_value = job_rate(tokens * args.steps, world, e2e_ms)
     expert_b, other_b = layer_bytes(shape)
     launch_s = (total_ms / 1e3) / (tokens * args.steps)
     peak, peak_kind = measured_peaks()

@@ -154,8 +154,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_router_kernel(const __gri
     if (tg == 0 && threadIdx.x == 0 && !mbar_wait_bounded(bar, 0, p.wait_ns, p.err)) fail = 1;
     __syncthreads();
     if (fail) return;
-    // a warp takes two units at a time (the same activation loads serve both rows)
-    for (int u = u0 + 2 * warp; u < u1; u += 2 * kWarps) {
+    // tiles of two units x four tokens, spread over all warps (one activation load
+    // serves both rows; enough tiles to keep every warp's loads in flight)
+    constexpr int kTT = 4;
+    const int nup = (nu + 1) / 2, nth = (nt + kTT - 1) / kTT;
+    for (int tile = warp; tile < nup * nth; tile += kWarps) {
+      const int u = u0 + 2 * (tile / nth), t0 = kTT * (tile % nth);
       const bool two = u + 1 < u1;
       const int qa = u / rows, ra = u % rows;
       const int ub = two ? u + 1 : u;
@@ -163,39 +167,42 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_router_kernel(const __gri
       const float4* wa = reinterpret_cast<const float4*>(wr + static_cast<size_t>(u - u0) * hc);
       const float4* wb = reinterpret_cast<const float4*>(wr + static_cast<size_t>(ub - u0) * hc);
       const int ka = (qa - q0) * (hc / 4), kb = (qb - q0) * (hc / 4);
-      double a0[kRouterTok], a1[kRouterTok], b0[kRouterTok], b1[kRouterTok];
+      double a0[kTT], a1[kTT], b0[kTT], b1[kTT];
 #pragma unroll
-      for (int t = 0; t < kRouterTok; ++t) a0[t] = a1[t] = b0[t] = b1[t] = 0.0;
+      for (int t = 0; t < kTT; ++t) a0[t] = a1[t] = b0[t] = b1[t] = 0.0;
       for (int k = lane; k < hc / 4; k += 32) {
         const float4 va = wa[k];
         const float4 vb = wb[k];
+        const double wa0 = va.x, wa1 = va.y, wa2 = va.z, wa3 = va.w;
+        const double wb0 = vb.x, wb1 = vb.y, wb2 = vb.z, wb3 = vb.w;
 #pragma unroll
-        for (int t = 0; t < kRouterTok; ++t) {
-          if (t < nt) {
-            const double2 xa0 = xa[static_cast<size_t>(t) * n4 + ka + k];
-            const double2 xb0 = xb[static_cast<size_t>(t) * n4 + ka + k];
-            a0[t] = fma(static_cast<double>(va.x), xa0.x, a0[t]);
-            a1[t] = fma(static_cast<double>(va.y), xa0.y, a1[t]);
-            a0[t] = fma(static_cast<double>(va.z), xb0.x, a0[t]);
-            a1[t] = fma(static_cast<double>(va.w), xb0.y, a1[t]);
+        for (int t = 0; t < kTT; ++t) {
+          if (t0 + t < nt) {
+            const size_t xt = static_cast<size_t>(t0 + t) * n4 + k;
+            const double2 xa0 = xa[xt + ka];
+            const double2 xb0 = xb[xt + ka];
+            a0[t] = fma(wa0, xa0.x, a0[t]);
+            a1[t] = fma(wa1, xa0.y, a1[t]);
+            a0[t] = fma(wa2, xb0.x, a0[t]);
+            a1[t] = fma(wa3, xb0.y, a1[t]);
             // the second unit usually shares the split (and so the loads)
-            const double2 xa1 = kb == ka ? xa0 : xa[static_cast<size_t>(t) * n4 + kb + k];
-            const double2 xb1 = kb == ka ? xb0 : xb[static_cast<size_t>(t) * n4 + kb + k];
-            b0[t] = fma(static_cast<double>(vb.x), xa1.x, b0[t]);
-            b1[t] = fma(static_cast<double>(vb.y), xa1.y, b1[t]);
-            b0[t] = fma(static_cast<double>(vb.z), xb1.x, b0[t]);
-            b1[t] = fma(static_cast<double>(vb.w), xb1.y, b1[t]);
+            const double2 xa1 = kb == ka ? xa0 : xa[xt + kb];
+            const double2 xb1 = kb == ka ? xb0 : xb[xt + kb];
+            b0[t] = fma(wb0, xa1.x, b0[t]);
+            b1[t] = fma(wb1, xa1.y, b1[t]);
+            b0[t] = fma(wb2, xb1.x, b0[t]);
+            b1[t] = fma(wb3, xb1.y, b1[t]);
           }
         }
       }
 #pragma unroll
-      for (int t = 0; t < kRouterTok; ++t) {
-        if (t < nt) {
+      for (int t = 0; t < kTT; ++t) {
+        if (t0 + t < nt) {
           const double la = warp_sum_d(a0[t] + a1[t]);
           const double lb = warp_sum_d(b0[t] + b1[t]);
           if (lane == 0) {
-            p.lpart[(static_cast<size_t>(tg + t) * rows + ra) * p.nq + qa] = la;
-            if (two) p.lpart[(static_cast<size_t>(tg + t) * rows + rb) * p.nq + qb] = lb;
+            p.lpart[(static_cast<size_t>(tg + t0 + t) * rows + ra) * p.nq + qa] = la;
+            if (two) p.lpart[(static_cast<size_t>(tg + t0 + t) * rows + rb) * p.nq + qb] = lb;
           }
         }
       }

@@ -54,3 +54,27 @@ def test_workspace_and_argument_checks(lib):
     assert L.fmoe_layer_forward(None, None, None, 1, None, None) == 1
     assert L.fmoe_rmsnorm(None, None, 1, 64, -1.0, None) == 1
     assert L.fmoe_status_string(4) == b"workspace missing or too small"
+
+
+def test_stack_and_batch_argument_checks(lib):
+    """Host-side checks of the stack, graph and batched entry points (no device work)."""
+    L = lib.lib()
+    cfg = lib.fmoe_config(4096, 1024, 512, 10, 4, 1, 1)
+    b32 = lib.fmoe_batch_workspace_bytes(cfg, 32)
+    assert b32 > lib.fmoe_batch_workspace_bytes(cfg, 1) > 0
+    assert lib.fmoe_batch_workspace_bytes(cfg, 0) == 0
+    assert lib.fmoe_batch_workspace_bytes(cfg, 65) == 0
+    s = ctypes.c_void_p()
+    assert L.fmoe_stack_create(None, 1, 1e-6, ctypes.byref(s)) == 1
+    arr = (ctypes.c_void_p * 1)(None)
+    assert L.fmoe_stack_create(arr, 1, 1e-6, ctypes.byref(s)) == 1
+    assert L.fmoe_stack_create(arr, 0, 1e-6, ctypes.byref(s)) == 1
+    assert L.fmoe_stack_forward(None, None, 1, 1, None) == 1
+    assert L.fmoe_stack_graph_create(None, None, 1, 1, ctypes.byref(s)) == 1
+    assert L.fmoe_graph_launch(None, None) == 1
+    assert L.fmoe_graph_destroy(None) == 0
+    assert L.fmoe_stack_destroy(None) == 0
+    assert L.fmoe_block_forward(None, None, 1, 1e-6, None, None) == 1
+    assert L.fmoe_layer_forward_batched(None, None, None, 1, None, None) == 1
+    assert L.fmoe_block_forward_batched(None, None, 1, 1e-6, None, None) == 1
+    assert L.fmoe_route_batched(None, None, 1, None, None, None, None) == 1

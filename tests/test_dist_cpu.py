@@ -1,0 +1,50 @@
+"""The multi-rank plumbing of bench.py on CPU (gloo, world size 2): the timed region of
+a run is the slowest rank's, and the job rate counts the units of every rank."""
+import datetime
+import multiprocessing as mp
+import os
+import socket
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        ms = 10.0 + 5.0 * rank  # rank 1 is the slow one
+        slowest = bench.max_over_ranks(ms, world, device="cpu")
+        rate = bench.job_rate(100, world, slowest)
+        dist.barrier()
+        q.put((rank, slowest, rate))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_slowest_rank_and_job_rate_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = sorted(q.get(timeout=10) for _ in procs)
+    for rank, slowest, rate in res:
+        assert slowest == 15.0
+        assert abs(rate - 200 / 0.015) < 1e-6
+
+
+def test_single_rank_needs_no_process_group():
+    import bench
+    assert bench.max_over_ranks(12.5, 1) == 12.5
+    assert bench.job_rate(1000, 1, 20.0) == 50000.0
