@@ -21,6 +21,10 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Waits until the grid this one depends on (programmatic dependent launch) has
+// completed and its memory operations are visible; a no-op without such a dependency.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }

@@ -874,11 +874,14 @@ struct LayerKernel {
         hdr->abort_flag = 0;
         hdr->skip_token = 0;
         hdr->sel[p.K] = p.E;  // the shared expert's record
-        hdr->tok_base = ld_relaxed_u32(p.tokens);
       }
     } else if (threadIdx.x == 32 && p.mode != MODE_ROUTE) {
       plan_experts();
     }
+    // everything above touches only shared memory and the parameters; from here on
+    // the kernel reads what the previous grid may have written
+    grid_dependency_wait();
+    if (threadIdx.x == 0) hdr->tok_base = ld_relaxed_u32(p.tokens);
     const uint32_t err0 = ld_relaxed_u32(p.err);
     __syncthreads();
     tbase_ = hdr->tok_base;
@@ -937,10 +940,9 @@ template <int BITS, bool NORM>
 __global__ void __launch_bounds__(kThreads, 1) fmoe_layer_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   // launched with programmatic stream serialization: let the next call's launch begin
-  // now, and wait until the previous grid has completed (its outputs and this layer's
-  // workspace) before reading anything (both are no-ops otherwise)
+  // now (a no-op otherwise); the kernel waits for the previous grid before it reads
+  // anything that grid may have written
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   LayerKernel<BITS, NORM> L(p, smem);
   L.run();
 }
