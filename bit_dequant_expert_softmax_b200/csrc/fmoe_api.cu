@@ -245,7 +245,7 @@ Params base_params(const fmoe_layer* L, int mode, int T) {
 // process if the runtime refuses the combination.
 std::atomic<int> g_pdl_ok{1};
 
-fmoe_status launch(const fmoe_layer* L, const Params& p, void* stream) {
+fmoe_status launch(const fmoe_layer* L, const Params& p, void* stream, bool allow_pdl = true) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(L->sms);
   cfg.blockDim = dim3(kThreads);
@@ -265,7 +265,7 @@ fmoe_status launch(const fmoe_layer* L, const Params& p, void* stream) {
                   : cudaLaunchKernelEx(&cfg, fmoe_layer_kernel<2, false>, p);
   };
   cudaError_t e = cudaErrorNotSupported;
-  if (g_pdl_ok.load(std::memory_order_relaxed)) {
+  if (allow_pdl && g_pdl_ok.load(std::memory_order_relaxed)) {
     cfg.numAttrs = 2;
     e = go();
     if (e != cudaSuccess) {
@@ -352,23 +352,44 @@ GParams batch_params(const fmoe_layer* L, int T) {
   return p;
 }
 
+// One launch, with programmatic stream serialization when the runtime allows it (the
+// kernels wait for their predecessor before reading anything).
+template <typename... A>
+cudaError_t launch_pdl(void (*kernel)(A...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, const GParams& p) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_pdl_ok.load(std::memory_order_relaxed) ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, p);
+  if (e != cudaSuccess && cfg.numAttrs == 1) {
+    cudaGetLastError();
+    g_pdl_ok.store(0, std::memory_order_relaxed);
+    cfg.numAttrs = 0;
+    e = cudaLaunchKernelEx(&cfg, kernel, p);
+  }
+  return e;
+}
+
 // router and top-K (+ grouping); then, if `experts`, gate/up, down and combine
 fmoe_status launch_batched(const fmoe_layer* L, GParams p, bool experts, cudaStream_t s) {
   const int G = L->sms;
-  grouped_router_kernel<<<G, kThreads, L->g_router_smem, s>>>(p);
-  grouped_topk_kernel<<<p.T, kThreads, L->g_topk_smem, s>>>(p);
-  if (experts) {
-    if (L->cfg.bits == 4)
-      grouped_matvec_kernel<4, false><<<G, kGThreads, L->g_gu_smem, s>>>(p);
-    else
-      grouped_matvec_kernel<2, false><<<G, kGThreads, L->g_gu_smem, s>>>(p);
-    if (L->cfg.bits == 4)
-      grouped_matvec_kernel<4, true><<<G, kGThreads, L->g_dn_smem, s>>>(p);
-    else
-      grouped_matvec_kernel<2, true><<<G, kGThreads, L->g_dn_smem, s>>>(p);
-    grouped_combine_kernel<<<dim3((p.H + 255) / 256, p.T), 256, 0, s>>>(p);
-  }
-  return cudaGetLastError() == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
+  cudaError_t e = launch_pdl(grouped_router_kernel, dim3(G), dim3(kThreads), L->g_router_smem, s, p);
+  if (e == cudaSuccess) e = launch_pdl(grouped_topk_kernel, dim3(p.T), dim3(kThreads), L->g_topk_smem, s, p);
+  if (experts && e == cudaSuccess)
+    e = launch_pdl(L->cfg.bits == 4 ? grouped_matvec_kernel<4, false> : grouped_matvec_kernel<2, false>, dim3(G),
+                   dim3(kGThreads), L->g_gu_smem, s, p);
+  if (experts && e == cudaSuccess)
+    e = launch_pdl(L->cfg.bits == 4 ? grouped_matvec_kernel<4, true> : grouped_matvec_kernel<2, true>, dim3(G),
+                   dim3(kGThreads), L->g_dn_smem, s, p);
+  if (experts && e == cudaSuccess)
+    e = launch_pdl(grouped_combine_kernel, dim3((p.H + 255) / 256, p.T), dim3(256), 0, s, p);
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
 }
 
 fmoe_status batch_ready(const fmoe_layer* L, int T) {
@@ -504,7 +525,6 @@ fmoe_status fmoe_layer_forward(fmoe_layer_t L, const uint16_t* x, const uint16_t
   if (T < 0) return FMOE_ERR_INVALID_ARG;
   if (T == 0) return FMOE_OK;
   if (!x || !resid || !y || !aligned(x, 16) || !aligned(resid, 16) || !aligned(y, 16)) return FMOE_ERR_INVALID_ARG;
-  if (y == x && resid != x) return FMOE_ERR_INVALID_ARG;
   if (y == x) return FMOE_ERR_INVALID_ARG;
   Params p = base_params(L, MODE_FULL, T);
   p.x = x;
@@ -833,7 +853,8 @@ fmoe_status fmoe_layer_forward_noalloc(fmoe_layer_t L, const uint16_t* x, const 
   p.x = x;
   p.resid = resid;
   p.y = y;
-  return launch(L, p, stream);
+  // the memset above precedes the launch: no programmatic overlap with it
+  return launch(L, p, stream, false);
 }
 
 }  // extern "C"

@@ -25,6 +25,10 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // completed and its memory operations are visible; a no-op without such a dependency.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Lets the grid launched after this one (with programmatic serialization) start its
+// launch now; a no-op otherwise.
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }

@@ -86,6 +86,8 @@ __host__ __device__ inline int router_splits_touched(int rows, int nq, int G) {
 
 __global__ void __launch_bounds__(kThreads, 1) grouped_router_kernel(const __grid_constant__ GParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
+  grid_launch_dependents();
+  grid_dependency_wait();
   if (ld_relaxed_u32(p.err) != 0) return;
   const int rows = p.E + (p.has_shared ? 1 : 0);
   const int G = gridDim.x, b = blockIdx.x;
@@ -358,6 +360,8 @@ __device__ void build_groups(const GParams& p, uint8_t* smem, const TopkSmem& L)
 // renormalised weights and the shared gate; then the grouping by the last block.
 __global__ void __launch_bounds__(kThreads, 1) grouped_topk_kernel(const __grid_constant__ GParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
+  grid_launch_dependents();
+  grid_dependency_wait();
   if (ld_relaxed_u32(p.err) != 0) return;
   uint32_t total;
   const TopkSmem L = topk_smem(p.E, p.K, p.T, p.has_shared, &total);
@@ -842,6 +846,8 @@ struct GroupedKernel {
 template <int BITS, bool DOWN>
 __global__ void __launch_bounds__(kGThreads, 1) grouped_matvec_kernel(const __grid_constant__ GParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
+  grid_launch_dependents();
+  grid_dependency_wait();
   if (ld_relaxed_u32(p.err) != 0) return;
   GroupedKernel<BITS, DOWN> G(p, smem);
   G.run();
@@ -853,6 +859,8 @@ __global__ void __launch_bounds__(kGThreads, 1) grouped_matvec_kernel(const __gr
 __global__ void grouped_combine_kernel(const __grid_constant__ GParams p) {
   __shared__ int spi[kMaxK + 1];
   __shared__ float sw[kMaxK + 1];
+  grid_launch_dependents();
+  grid_dependency_wait();
   if (ld_relaxed_u32(p.err) != 0) return;
   const int t = blockIdx.y;
   const int ns = p.K + (p.has_shared ? 1 : 0);

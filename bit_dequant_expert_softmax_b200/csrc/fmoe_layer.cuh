@@ -724,7 +724,6 @@ struct LayerKernel {
     mark(11);
     rank_topk<kThreads>(skey, ckey, cidx, p.E, p.K, hdr->sel);
     mark(12);
-    mark(13);
     // keep the selection's logits: the staging area is about to receive the rows
     if (threadIdx.x <= p.K)
       hdr->selog[threadIdx.x] =
@@ -942,7 +941,7 @@ __global__ void __launch_bounds__(kThreads, 1) fmoe_layer_kernel(const __grid_co
   // launched with programmatic stream serialization: let the next call's launch begin
   // now (a no-op otherwise); the kernel waits for the previous grid before it reads
   // anything that grid may have written
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  grid_launch_dependents();
   LayerKernel<BITS, NORM> L(p, smem);
   L.run();
 }
@@ -951,6 +950,8 @@ __global__ void __launch_bounds__(kThreads, 1) fmoe_layer_kernel(const __grid_co
 // of bf16 values), then out = bf16(h / sqrt(mean + eps)) rounded once from double.
 __global__ void fmoe_rmsnorm_kernel(const uint16_t* h, uint16_t* out, int H, double eps) {
   __shared__ double part[32];
+  grid_launch_dependents();
+  grid_dependency_wait();
   const uint16_t* ht = h + static_cast<size_t>(blockIdx.x) * H;
   uint16_t* ot = out + static_cast<size_t>(blockIdx.x) * H;
   double s = 0.0;

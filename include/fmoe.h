@@ -256,9 +256,10 @@ fmoe_status fmoe_layer_debug_hold_block(fmoe_layer_t layer, int cta);
  * uint64), every block of the following forward calls records its phase boundaries
  * while it processes token `token` of a call: %globaltimer (ns) in dev_buf[block*32 + i]
  * and the SM clock counter in dev_buf[block*32 + 16 + i], for i = 0 start, 1 activations
- * staged, 2 router rows done, 3 top-K start, 4 top-K done, 5 gate/up done, 6 h rows of
- * all blocks visible, 7 h staged, 8 down rows done, 9 token done, 10 router logits of
- * all blocks visible, 11..13 top-K steps.  NULL (default) disables it. */
+ * staged, 2 router rows done, 3 top-K start (the shared expert's gate/up done), 4 top-K
+ * done, 5 gate/up done, 6 h rows of all blocks visible, 7 h staged, 8 down rows done,
+ * 9 token done, 10 router logits of all blocks visible, 11 expert ranks start, 12 expert
+ * ranks done, 14 first batch of h loaded, 15 h loaded.  NULL (default) disables it. */
 fmoe_status fmoe_layer_debug_timeline(fmoe_layer_t layer, uint64_t* dev_buf, int token);
 
 /* Number of thread blocks one forward launch uses (one per SM of the device). */
