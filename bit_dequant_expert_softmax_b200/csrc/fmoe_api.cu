@@ -171,8 +171,8 @@ fmoe_status plan(fmoe_layer* L) {
   const int G = L->sms;
   // P1: x in doubles and the router rows a block touches from the start of the
   // staging area, its shared gate/up rows at the end (both in flight together); the
-  // shared rows are consumed before top-K, whose logits and candidates then may use
-  // the whole area
+  // shared rows are consumed while top-K starts, so its logits and candidates must
+  // not reach them either
   const long long U = (long long)(c.n_experts + c.has_shared) * L->nq;
   const uint32_t rows_touched = (uint32_t)(((U + G - 1) / G + L->nq - 1) / L->nq + 1);
   const int shared_rows = (c.inter + G - 1) / G;
@@ -184,7 +184,7 @@ fmoe_status plan(fmoe_layer* L) {
   // top-K: logits, selection keys, per-warp candidates
   if ((uint64_t)r128((uint32_t)(c.n_experts + 1) * 8u) + (uint64_t)((c.n_experts + 15) & ~15) * 8u +
           (uint64_t)((c.n_experts + 31) / 32) * c.top_k * 12u >
-      staging)
+      sc_off)
     return FMOE_ERR_UNSUPPORTED;
   // P2: at least one gate/up row pair per round
   if (g.gu_bytes(1) > staging) return FMOE_ERR_UNSUPPORTED;

@@ -908,11 +908,10 @@ struct LayerKernel {
       if (!phase1_consume(buf, route)) break;
       if (route) publish(p.rflags, t);
       mark(2);
-      if (has_sc_) {  // the shared expert does not depend on the routing: its gate/up
-        gu_consume(&sc_, 1, buf);  // rows are consumed while the router partials travel
-        __syncthreads();
-        if (hdr->abort_flag) break;
-      }
+      // the shared expert does not depend on the routing: warps 1-15 consume its
+      // gate/up rows while warp 0 already polls for the router partials (top-K's
+      // scratch and the shared rows occupy disjoint parts of the staging area)
+      if (has_sc_) gu_consume(&sc_, 1, buf, 1);
       if (route) {
         topk(buf, t);
         if (hdr->abort_flag) break;
