@@ -106,16 +106,29 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+KERNEL_SOURCES = ("fmoe_layer.cuh", "fmoe_device.cuh", "fmoe_topk.cuh")
+
+
+def kernel_source_digest(texts) -> str:
+    """sha256 of the layer kernel's sources with comments and whitespace removed (a
+    change to a comment does not change the kernel the counters were taken from)."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for t in texts:
+        t = re.sub(r"/\*.*?\*/", " ", t, flags=re.S)
+        t = re.sub(r"//[^\n]*", " ", t)
+        h.update(" ".join(t.split()).encode())
+    return h.hexdigest()
+
+
 def profiled_traffic():
     """DRAM bytes per launch of the layer kernel from the committed ncu summary, if
     the kernel source is the one that was profiled (else None)."""
-    import hashlib
-    src = [os.path.join(ROOT, "bit_dequant_expert_softmax_b200", "csrc", f)
-           for f in ("fmoe_layer.cuh", "fmoe_device.cuh", "fmoe_topk.cuh")]
-    h = hashlib.sha256()
-    for f in src:
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+    texts = []
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "bit_dequant_expert_softmax_b200", "csrc", f)) as fh:
+            texts.append(fh.read())
     path = os.path.join(ROOT, "profiles", "fmoe_layer_kernel_layer4096.md")
     if not os.path.exists(path):
         return None
@@ -123,11 +136,11 @@ def profiled_traffic():
     with open(path) as f:
         for line in f:
             line = line.strip()
-            if line.startswith("kernel_source_sha256:"):
+            if line.startswith("kernel_source_digest:"):
                 want = line.split(":", 1)[1].strip()
             elif line.startswith("traffic_bytes_per_launch:"):
                 traffic = int(line.split(":", 1)[1].strip())
-    return traffic if want == h.hexdigest() else None
+    return traffic if want == kernel_source_digest(texts) else None
 
 
 def max_over_ranks(value: float, world: int, device="cuda") -> float:

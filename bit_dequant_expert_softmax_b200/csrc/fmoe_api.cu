@@ -560,10 +560,11 @@ fmoe_status fmoe_layer_set_batch_workspace(fmoe_layer_t L, void* dev_ptr, size_t
   if (bytes < bl.size) return FMOE_ERR_NO_WORKSPACE;
   const fmoe_status st = plan_batched(L, max_tokens);
   if (st != FMOE_OK) return st;
-  if (!set_smem(grouped_router_kernel, L->g_router_smem) || !set_smem(grouped_topk_kernel, L->g_topk_smem) ||
-      !set_smem(grouped_matvec_kernel<4, false>, L->g_gu_smem) ||
-      !set_smem(grouped_matvec_kernel<2, false>, L->g_gu_smem) ||
-      !set_smem(grouped_matvec_kernel<4, true>, L->g_dn_smem) || !set_smem(grouped_matvec_kernel<2, true>, L->g_dn_smem))
+  // the attribute is an upper bound shared by every layer using these kernels: set it
+  // to the device maximum (a layer-sized value would break larger layers' launches)
+  if (!set_smem(grouped_router_kernel, kMaxSmem) || !set_smem(grouped_topk_kernel, kMaxSmem) ||
+      !set_smem(grouped_matvec_kernel<4, false>, kMaxSmem) || !set_smem(grouped_matvec_kernel<2, false>, kMaxSmem) ||
+      !set_smem(grouped_matvec_kernel<4, true>, kMaxSmem) || !set_smem(grouped_matvec_kernel<2, true>, kMaxSmem))
     return FMOE_ERR_CUDA;
   if (cudaMemset(dev_ptr, 0, bl.size) != cudaSuccess) return FMOE_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;

@@ -11,11 +11,12 @@
 //            pairs in (expert, token) order and tiles of <= kTileTok pairs of one
 //            expert, each with a work weight
 //   gate/up  persistent blocks, each a contiguous, weight-balanced range of
-//            (tile, row pair) units: a tile's activations are staged once, every
-//            warp streams its own row pairs through a two-slot ring of bulk copies;
+//            (tile, 8 row pairs) units: a tile's activations are staged once, every
+//            warp streams its own units' rows through a two-slot ring of bulk copies
+//            and multiplies them on the tensor cores (mma.sync, exact bf16 operands);
 //            h = silu(W_g x) * (W_u x) for each pair of the tile
-//   down     the same over (tile, output-row block) units, activations = h of the
-//            tile's pairs; o = W_d h per pair
+//   down     the same over (tile, 16 output rows) units, activations = h of the
+//            tile's pairs (bf16 hi + lo); o = W_d h per pair
 //   combine  y = resid + sum_k w_k o_k + sigma o_s per token, in slot order, rounded
 //            once to bf16
 //

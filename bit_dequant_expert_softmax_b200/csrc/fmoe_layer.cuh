@@ -3,20 +3,21 @@
 // One persistent thread block per SM (cooperative launch).  Per token:
 //
 //   P1  router matvec (fp64 accumulation of exact fp32 x bf16 products) over a
-//       slice of router rows per block; the shared expert's gate/up rows.
-//   B1  grid-wide barrier (bounded wait).
-//   P2  every block computes softmax / top-K / renormalisation redundantly from
-//       the logits (one warp); then streams its slice of the K routed experts'
-//       gate/up row pairs, h = silu(g) * u; the down rows it will need are
-//       fetched in the same burst when shared memory allows.
-//   B2  grid-wide barrier.
+//       slice of router rows per block, partials published with a per-block flag;
+//       while they travel, warps 1-15 consume the block's slice of the shared
+//       expert's gate/up rows (they do not depend on the routing) and warp 0 polls.
+//   P2  every block computes top-K from the logits redundantly; thread 0 requests
+//       the block's slice of the K routed experts' gate/up row pairs one copy after
+//       another, then its down rows (P3's data); warps 1-15 compute
+//       h = silu(g) * u, warp 0 the renormalised softmax weights; h is published
+//       with a per-block flag.
 //   P3  every block stages h of all K+1 experts, computes its slice of output
 //       rows of the K+1 down matvecs and the combine
 //       y = resid + sum_k w_k o_k + sigma o_s, rounded once to bf16.
 //
 // All weight bytes move HBM -> shared memory through the bulk-copy (TMA) engine
-// as contiguous row ranges, completion tracked by mbarriers; a block issues its
-// whole share of a phase at once when it fits, so its loads are all in flight.
+// as contiguous row ranges, completion tracked by mbarriers; every wait (flags,
+// mbarriers) is bounded.
 #pragma once
 
 #include "fmoe_device.cuh"

@@ -243,13 +243,14 @@ fmoe_status fmoe_graph_destroy(fmoe_graph_t graph);
 fmoe_status fmoe_layer_get_error(fmoe_layer_t layer, uint32_t* device_error);
 
 /* Upper bound, in nanoseconds, of every device-side wait of this layer (grid-wide
- * barriers, bulk-copy completion).  Default 2e9 (2 s).  A wait that exceeds it sets an
+ * exchanges of partial results, bulk-copy completion).  Default 2e9 (2 s).  A wait that exceeds it sets an
  * error bit and the kernel returns. */
 fmoe_status fmoe_layer_set_wait_limit(fmoe_layer_t layer, uint64_t nanoseconds);
 
 /* Test hook for the failure path: when cta >= 0, thread block `cta` of the next forward
- * calls returns before its first grid-wide barrier, so the other blocks' bounded wait
- * runs out and FMOE_DEVERR_BARRIER_TIMEOUT is set.  -1 (default) disables it. */
+ * calls returns before it publishes anything, so the other blocks' bounded wait for
+ * its partial results runs out and FMOE_DEVERR_BARRIER_TIMEOUT is set.  -1 (default)
+ * disables it. */
 fmoe_status fmoe_layer_debug_hold_block(fmoe_layer_t layer, int cta);
 
 /* Diagnostic hook: when dev_buf != NULL (a device buffer of fmoe_layer_grid_size() * 32

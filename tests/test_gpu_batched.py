@@ -243,3 +243,26 @@ def test_stack16_batched_full_size(cuda_lib):
     for (l, t, j, y, (idx, w, sig)), (r_idx, r_w, r_sig, r_y) in zip(gpu, refs):
         r = SimpleNamespace(idx=r_idx, w=r_w, sigma=r_sig, y=r_y)
         _assert_token(f"stack16 layer {l} token {t}", y, idx, w, sig, j, r, True)
+
+
+def test_batched_layers_of_different_shapes_interleaved(cuda_lib):
+    """A large and a small layer, attached one after the other, run alternately (the
+    kernels' shared-memory limit is shared by all layers)."""
+    big, small = SHAPES["mid_2bit"], SHAPES["tiny"]
+    Lb = _layer(cuda_lib, big, seed=26, max_tokens=16)
+    Ls = _layer(cuda_lib, small, seed=27, max_tokens=16)
+    xb = _x(26, 0, 16, big.hidden)
+    xs = _x(27, 0, 16, small.hidden)
+    yb1 = Lb.forward_batched(xb)
+    ys1 = Ls.forward_batched(xs)
+    yb2 = Lb.forward_batched(xb)
+    torch.cuda.synchronize()
+    assert Lb.error() == 0 and Ls.error() == 0
+    assert torch.equal(yb1.view(torch.int16), yb2.view(torch.int16))
+    ob = oracle.synthetic_layer(26, 0, big, lazy=True)
+    osm = oracle.synthetic_layer(27, 0, small, lazy=True)
+    ib, wb, sb = (a.cpu().numpy() for a in Lb.route_batched(xb))
+    is_, ws, ss = (a.cpu().numpy() for a in Ls.route_batched(xs))
+    for t in (0, 15):
+        _assert_token(f"big token {t}", _bf(yb1)[t], ib, wb, sb, t, ob.forward(_bf(xb)[t]), True)
+        _assert_token(f"small token {t}", _bf(ys1)[t], is_, ws, ss, t, osm.forward(_bf(xs)[t]), True)
