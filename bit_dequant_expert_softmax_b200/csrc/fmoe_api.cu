@@ -146,6 +146,15 @@ bool set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
+// The largest dynamic shared memory a kernel can be given (the per-block maximum less
+// its static shared memory).
+template <typename K>
+bool set_smem_max(K kernel) {
+  cudaFuncAttributes a;
+  if (cudaFuncGetAttributes(&a, kernel) != cudaSuccess) return false;
+  return set_smem(kernel, kMaxSmem - static_cast<int>(a.sharedSizeBytes));
+}
+
 template <int BITS>
 int chunk_cols() {
   return Chunk<BITS>::kCols;
@@ -297,8 +306,9 @@ fmoe_status plan_batched(fmoe_layer* L, int T) {
     return sizeof(GHeader) + (size_t)g.frag_bytes + (size_t)g.sum_bytes + (size_t)kGWarps * kRing * g.piece_bytes;
   };
   const size_t gsm = mv_smem(false), dsm = mv_smem(true);
-  if (rsm > (size_t)kMaxSmem || tsm > (uint32_t)kMaxSmem || gsm > (size_t)kMaxSmem || dsm > (size_t)kMaxSmem)
-    return FMOE_ERR_UNSUPPORTED;
+  // (less a little for the kernels' static shared words)
+  const size_t room = (size_t)kMaxSmem - 1024;
+  if (rsm > room || tsm > room || gsm > room || dsm > room) return FMOE_ERR_UNSUPPORTED;
   // segments a block's unit range can touch: its share of the total weight over the
   // lightest tile, plus the partial tiles at both ends
   const long long mt = batch_max_tiles(c, T);
@@ -562,9 +572,9 @@ fmoe_status fmoe_layer_set_batch_workspace(fmoe_layer_t L, void* dev_ptr, size_t
   if (st != FMOE_OK) return st;
   // the attribute is an upper bound shared by every layer using these kernels: set it
   // to the device maximum (a layer-sized value would break larger layers' launches)
-  if (!set_smem(grouped_router_kernel, kMaxSmem) || !set_smem(grouped_topk_kernel, kMaxSmem) ||
-      !set_smem(grouped_matvec_kernel<4, false>, kMaxSmem) || !set_smem(grouped_matvec_kernel<2, false>, kMaxSmem) ||
-      !set_smem(grouped_matvec_kernel<4, true>, kMaxSmem) || !set_smem(grouped_matvec_kernel<2, true>, kMaxSmem))
+  if (!set_smem_max(grouped_router_kernel) || !set_smem_max(grouped_topk_kernel) ||
+      !set_smem_max(grouped_matvec_kernel<4, false>) || !set_smem_max(grouped_matvec_kernel<2, false>) ||
+      !set_smem_max(grouped_matvec_kernel<4, true>) || !set_smem_max(grouped_matvec_kernel<2, true>))
     return FMOE_ERR_CUDA;
   if (cudaMemset(dev_ptr, 0, bl.size) != cudaSuccess) return FMOE_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
