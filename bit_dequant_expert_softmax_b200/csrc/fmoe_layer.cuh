@@ -8,9 +8,9 @@
 //       expert's gate/up rows (they do not depend on the routing) and warp 0 polls.
 //   P2  every block computes top-K from the logits redundantly; thread 0 requests
 //       the block's slice of the K routed experts' gate/up row pairs one copy after
-//       another, then its down rows (P3's data); warps 1-15 compute
-//       h = silu(g) * u, warp 0 the renormalised softmax weights; h is published
-//       with a per-block flag.
+//       another, and its down rows (P3's data) once half of those have landed;
+//       warps 1-15 compute h = silu(g) * u, warp 0 the renormalised softmax
+//       weights; h is published with a per-block flag.
 //   P3  every block stages h of all K+1 experts, computes its slice of output
 //       rows of the K+1 down matvecs and the combine
 //       y = resid + sum_k w_k o_k + sigma o_s, rounded once to bf16.
@@ -812,9 +812,17 @@ struct LayerKernel {
         ch[k].first += nitem;
       }
       issue_gu(ch, pl.nc);
-      issue_down_items(j0, j1, 0, ndown, down_first, doff);
       nitem += static_cast<uint32_t>(pl.gitems + ndown);
       if (route) route_weights(tok_);
+      // the down rows are requested once the first half of the gate/up rows has
+      // landed (thread 0 consumes none of them): requested together, both streams are
+      // served interleaved and the gate/up rows complete late, while the down rows are
+      // needed only after the h exchange.  The copies are issued whatever the wait
+      // returns.
+      if (threadIdx.x == 0) {
+        if (pl.gitems > 0) (void)wait_item(down_first - static_cast<uint32_t>(pl.gitems - (pl.gitems - 1) / 2));
+        issue_down_items(j0, j1, 0, ndown, down_first, doff);
+      }
       gu_consume(ch, pl.nc, buf, 1);
       __syncthreads();
       if (hdr->abort_flag) return false;
