@@ -175,6 +175,23 @@ def test_router_logits_are_matvec():
         assert math.isclose(l[e], math.fsum(float(Wr[e, c]) * x[c] for c in range(H)), rel_tol=1e-14, abs_tol=1e-15)
 
 
+def test_router_bias_is_added():
+    """A zero router leaves exactly the bias as logits; a bias large enough to
+    dominate moves the selection to its expert (workload of the batched stack: a
+    per-expert bias skews expert popularity)."""
+    H, E = 64, 8
+    x = _x(H)
+    b = np.array([0.5, -1.25, 2.0, 0.0, -3.0, 1.5, 0.25, -0.75], dtype=np.float32)
+    assert np.array_equal(oracle.router_logits(x, np.zeros((E, H), np.float32), b), b.astype(np.float64))
+    Wr = synth.gen_router(1, 0, E, H)
+    base = oracle.router_logits(x, Wr)
+    skew = np.zeros(E, np.float32)
+    skew[5] = 100.0
+    lb = oracle.router_logits(x, Wr, skew)
+    assert lb[5] == base[5] + 100.0 and np.array_equal(np.delete(lb, 5), np.delete(base, 5))
+    assert oracle.topk_renorm(lb, 2)[0][0] == 5
+
+
 # --------------------------------------------------------- swiglu/combine ----
 def test_silu_matches_library():
     t = np.linspace(-30, 30, 1001)
@@ -219,6 +236,21 @@ def test_zero_scale_bias_routed_gives_x_plus_shared():
 
 def test_shared_gate_zero_gives_half():
     assert oracle.shared_sigma(np.zeros(64), np.ones(64)) == 0.5
+
+
+def test_shared_gate_matches_library_sigmoid():
+    """sigma = expit(g_s . x): a dot product of ln 3 gives 3/4; random vectors agree
+    with the library's logistic function."""
+    gs = np.zeros(64)
+    gs[3] = math.log(3.0)
+    x = np.zeros(64)
+    x[3] = 1.0
+    assert math.isclose(oracle.shared_sigma(gs, x), 0.75, rel_tol=1e-15)
+    rng = np.random.default_rng(9)
+    for _ in range(20):
+        gs, x = rng.standard_normal(64), rng.standard_normal(64)
+        s = math.fsum(float(a) * float(b) for a, b in zip(gs, x))
+        assert math.isclose(oracle.shared_sigma(gs, x), float(scipy.special.expit(s)), rel_tol=1e-14)
 
 
 def test_power_of_two_down_scaling_is_exact():
@@ -292,6 +324,15 @@ def test_whole_layer_matches_brute_force():
         assert np.allclose(r.y, yb, rtol=1e-12, atol=1e-12)
 
 
+def test_expert_forward_equals_forward_with_its_routing():
+    """The split entry point's reference (combine for given routing) reproduces the
+    whole layer exactly when handed the layer's own routing."""
+    lay, sh = _tiny_layer()
+    x = _x(sh.hidden, seed=8)
+    r = lay.forward(x)
+    assert np.array_equal(lay.expert_forward(x, x, r.idx, r.w, r.sigma), r.y)
+
+
 # ------------------------------------------------------ pre-norm block ----
 def test_block_residual_is_the_unnormalised_input():
     """Experts whose down projections are zero add nothing: the block returns h
@@ -338,6 +379,21 @@ def test_rmsnorm_constant_and_library():
     refb = oracle.f64_to_bf16_bits(ref.numpy())
     assert np.mean(n == refb) > 0.999
     assert np.max(np.abs(oracle.bf16_to_f64(n) - oracle.bf16_to_f64(refb))) <= 2 ** -7 * np.max(np.abs(oracle.bf16_to_f64(n)))
+
+
+def test_rmsnorm_eps_inside_the_root():
+    """Where mean(h^2) is of the order of eps, eps decides the result: a constant
+    vector a gives a / sqrt(a^2 + eps) (here 2^-10 / sqrt(2^-20 + 2^-20) = 2^-1/2), and
+    small random vectors agree with the library routine."""
+    a = 2.0 ** -10
+    n = oracle.bf16_to_f64(oracle.rmsnorm_bf16(np.full(512, a), 2.0 ** -20))
+    assert np.all(n == oracle.bf16_to_f64(oracle.f64_to_bf16_bits(np.array([math.sqrt(0.5)])))[0])
+    rng = np.random.default_rng(6)
+    h = oracle.bf16_to_f64(synth.bf16_bits(rng.standard_normal(1024) * 1e-3))
+    n = oracle.rmsnorm_bf16(h, 1e-6)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(h), (1024,), eps=1e-6)
+    refb = oracle.f64_to_bf16_bits(ref.numpy())
+    assert np.mean(n == refb) > 0.999
 
 
 def test_tolerance_helper():
