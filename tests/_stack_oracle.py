@@ -8,13 +8,14 @@ import oracle
 
 
 def block_case(args):
-    """(seed, layer, shape fields, h as bf16 bits) -> (idx, w, sigma, y unrounded)."""
+    """(seed, layer, shape fields, h as bf16 bits) -> (idx, w, sigma, y unrounded,
+    logits)."""
     seed, layer, fields, h_bits = args
     shape = synth.LayerShape(*fields)
     lay = oracle.synthetic_layer(seed, layer, shape, lazy=True)
     h = oracle.bf16_to_f64(np.asarray(h_bits, dtype=np.uint16))
     r = oracle.block_forward(lay, h)
-    return r.idx, r.w, r.sigma, r.y
+    return r.idx, r.w, r.sigma, r.y, r.logits
 
 
 def shape_fields(shape):

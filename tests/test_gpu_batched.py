@@ -21,6 +21,7 @@ import torch
 
 import fmoe_synth as synth
 import oracle
+from _ties import index_mismatch
 from _stack_oracle import block_case, shape_fields
 
 pytestmark = pytest.mark.gpu
@@ -50,7 +51,7 @@ def _x(seed, t0, T, H):
 
 
 def _assert_token(ctx, y, idx, w, sig, t, r, has_shared):
-    assert list(idx[t]) == list(r.idx), f"{ctx}: idx {list(idx[t])} vs oracle {list(r.idx)}"
+    assert list(idx[t]) == list(r.idx), index_mismatch(ctx, idx[t], r.idx, r.logits)
     assert np.allclose(w[t], r.w, rtol=1e-6, atol=1e-7), f"{ctx}: w"
     if has_shared:
         assert abs(float(sig[t]) - r.sigma) <= 1e-6 * abs(r.sigma), f"{ctx}: sigma"
@@ -240,8 +241,8 @@ def test_stack16_batched_full_size(cuda_lib):
         torch.cuda.empty_cache()
     with ProcessPoolExecutor(max_workers=len(jobs), mp_context=multiprocessing.get_context("spawn")) as ex:
         refs = list(ex.map(block_case, jobs))
-    for (l, t, j, y, (idx, w, sig)), (r_idx, r_w, r_sig, r_y) in zip(gpu, refs):
-        r = SimpleNamespace(idx=r_idx, w=r_w, sigma=r_sig, y=r_y)
+    for (l, t, j, y, (idx, w, sig)), (r_idx, r_w, r_sig, r_y, r_logits) in zip(gpu, refs):
+        r = SimpleNamespace(idx=r_idx, w=r_w, sigma=r_sig, y=r_y, logits=r_logits)
         _assert_token(f"stack16 layer {l} token {t}", y, idx, w, sig, j, r, True)
 
 

@@ -17,6 +17,7 @@ import torch
 
 import fmoe_synth as synth
 import oracle
+from _ties import index_mismatch
 
 pytestmark = pytest.mark.gpu
 
@@ -47,7 +48,7 @@ def _check_tokens(olay, xg, yg, idxg, wg, sigg, tokens, ctx=""):
     worst = 0.0
     for t in tokens:
         r = olay.forward(xs[t])
-        assert list(idx[t]) == list(r.idx), f"{ctx} token {t}: idx {list(idx[t])} vs oracle {list(r.idx)}"
+        assert list(idx[t]) == list(r.idx), index_mismatch(f"{ctx} token {t}", idx[t], r.idx, r.logits)
         assert np.allclose(w[t], r.w, rtol=1e-6, atol=1e-7), f"{ctx} token {t}: w"
         if olay.has_shared and sigg is not None:
             assert math.isclose(float(sigg.cpu()[t]), r.sigma, rel_tol=1e-6), f"{ctx} token {t}: sigma"
@@ -116,7 +117,8 @@ def test_split_api_equals_fused_and_oracle(cuda_lib):
         r = olay.forward(xs[t])
         ye = olay.expert_forward(xs[t], xs[t], idx[t].cpu().numpy(), w[t].cpu().numpy(), float(sig[t]))
         assert oracle.within_tolerance(_bf(ys)[t], ye)[0]
-        assert list(idx[t].cpu().numpy()) == list(r.idx)
+        assert list(idx[t].cpu().numpy()) == list(r.idx), index_mismatch(f"token {t}", idx[t].cpu().numpy(), r.idx,
+                                                                         r.logits)
 
 
 def test_resid_differs_from_x_and_in_place(cuda_lib):

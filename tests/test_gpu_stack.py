@@ -19,6 +19,7 @@ import torch
 
 import fmoe_synth as synth
 import oracle
+from _ties import index_mismatch
 from _stack_oracle import block_case, shape_fields
 
 pytestmark = pytest.mark.gpu
@@ -60,8 +61,9 @@ def _gpu_routing(fm, L, h):
 
 def _assert_block(ctx, y_gpu, route, t, ref):
     idx, w, sig = route
-    r_idx, r_w, r_sig, r_y = ref
-    assert list(idx[t].cpu().numpy()) == list(r_idx), f"{ctx}: idx {list(idx[t].cpu().numpy())} vs {list(r_idx)}"
+    r_idx, r_w, r_sig, r_y = ref[:4]
+    r_logits = ref[4] if len(ref) > 4 else None
+    assert list(idx[t].cpu().numpy()) == list(r_idx), index_mismatch(ctx, idx[t].cpu().numpy(), r_idx, r_logits)
     assert np.allclose(w[t].cpu().numpy(), r_w, rtol=1e-6, atol=1e-7), f"{ctx}: w"
     ok, ratio = oracle.within_tolerance(y_gpu, r_y)
     assert ok, f"{ctx}: worst error/bound {ratio:.3f}"
@@ -96,7 +98,7 @@ def test_block_equals_norm_then_layer_and_oracle(cuda_lib, name):
     hs, ys = _bf(h), _bf(y)
     for t in range(T):
         r = oracle.block_forward(olay, hs[t], EPS)
-        _assert_block(f"{name} token {t}", ys[t], route, t, (r.idx, r.w, r.sigma, r.y))
+        _assert_block(f"{name} token {t}", ys[t], route, t, (r.idx, r.w, r.sigma, r.y, r.logits))
 
 
 @pytest.mark.parametrize("name", ["tiny", "tiny_2bit"])
@@ -132,7 +134,7 @@ def test_small_stack_graph_teacher_forced(cuda_lib, name):
         hin, hout = _bf(hs[l]), _bf(hs[l + 1])
         for t in range(T):
             r = oracle.block_forward(olay, hin[t], EPS)
-            _assert_block(f"{name} layer {l} token {t}", hout[t], route, t, (r.idx, r.w, r.sigma, r.y))
+            _assert_block(f"{name} layer {l} token {t}", hout[t], route, t, (r.idx, r.w, r.sigma, r.y, r.logits))
 
 
 def _full_stack_gpu(cuda_lib, shape, NL, T, seed, samples):
