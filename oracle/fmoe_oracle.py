@@ -83,7 +83,10 @@ def f64_to_bf16_bits(v) -> np.ndarray:
 
 def unpack_codes(words: np.ndarray, bits: int) -> np.ndarray:
     """uint32 words [..., W] -> integer codes [..., W * 32/bits], code k of a word
-    taken from bits [bits*k, bits*k + bits) (lowest bits first)."""
+    taken from bits [bits*k, bits*k + bits) (lowest bits first).
+
+    4-bit (or 2-bit) expert weights packed into 32-bit words: hotdry.top,
+    "量化策略"; the order inside a word is a reading (the pages are silent)."""
     words = np.asarray(words, dtype=np.uint32)
     per = 32 // bits
     mask = (1 << bits) - 1
@@ -97,7 +100,11 @@ def dequantise(codes: np.ndarray, sb: np.ndarray) -> np.ndarray:
     """Explicit dequantisation W[r, c] = scale[r, c//64] * q[r, c] + bias[r, c//64].
 
     ``sb`` holds one uint32 per (row, group): bf16 scale in the low half,
-    bf16 bias in the high half."""
+    bf16 bias in the high half.  The affine form ``code * scale + bias`` is that of
+    hotdry.top, "量化策略", and of the juejin.cn shader section "Metal 着色器" (whose
+    ``fma(code, scale*x, bias*x)`` is the same product reordered); the group of 64
+    along the input dimension is the reading that fits the pages' 6.75 MB per
+    expert."""
     sb = np.asarray(sb, dtype=np.uint32)
     scale = bf16_to_f64((sb & 0xFFFF).astype(np.uint16))
     bias = bf16_to_f64((sb >> 16).astype(np.uint16))
@@ -131,7 +138,8 @@ def record_regions(H: int, I: int, bits: int) -> dict:
 
 
 def decode_record(rec: np.ndarray, H: int, I: int, bits: int) -> DenseExpert:
-    """Read one packed record and dequantise its three matrices to float64."""
+    """Read one packed record and dequantise its three matrices to float64 (gate
+    and up [I, H], down [H, I]: the expert FFN of hotdry.top, "Metal GPU管线")."""
     R = record_regions(H, I, bits)
     rec = np.asarray(rec, dtype=np.uint8)
     wh, wi = H * bits // 32, I * bits // 32
@@ -149,7 +157,9 @@ def decode_record(rec: np.ndarray, H: int, I: int, bits: int) -> DenseExpert:
 # the layer, step by step
 # ----------------------------------------------------------------------------
 def router_logits(x: np.ndarray, Wr: np.ndarray, bias: Optional[np.ndarray] = None) -> np.ndarray:
-    """l_e = sum_c Wr[e, c] x_c (+ b_e), float64 (router GEMV)."""
+    """l_e = sum_c Wr[e, c] x_c (+ b_e), float64 (router GEMV; routing runs on the
+    GPU in tinai-dev README, "Pipeline mỗi lớp").  The bias is the batched
+    workload's per-expert popularity skew."""
     l = Wr.astype(np.float64) @ np.asarray(x, dtype=np.float64)
     if bias is not None:
         l = l + np.asarray(bias, dtype=np.float64)
@@ -157,6 +167,8 @@ def router_logits(x: np.ndarray, Wr: np.ndarray, bias: Optional[np.ndarray] = No
 
 
 def softmax(l: np.ndarray) -> np.ndarray:
+    """Softmax over all experts (intelliparadigm.com, section 2.1 router snippet),
+    shifted by the maximum (the same value in exact arithmetic)."""
     m = np.max(l)
     e = np.exp(l - m)
     return e / np.sum(e)
@@ -164,7 +176,10 @@ def softmax(l: np.ndarray) -> np.ndarray:
 
 def topk_renorm(l: np.ndarray, K: int):
     """Softmax over all experts, top-K by probability (descending, ties to the
-    lower index), then the K probabilities renormalised to sum to one."""
+    lower index), then the K probabilities renormalised to sum to one
+    (intelliparadigm.com, section 2.1: softmax, then top-K on the probabilities;
+    tinai-dev README, "Pipeline mỗi lớp": softmax + top-K routing).  The
+    renormalisation and the tie rule are readings."""
     p = softmax(l)
     order = sorted(range(len(p)), key=lambda e: (-p[e], e))
     idx = np.array(order[:K], dtype=np.int64)
@@ -173,11 +188,14 @@ def topk_renorm(l: np.ndarray, K: int):
 
 
 def silu(t: np.ndarray) -> np.ndarray:
+    """silu(t) = t * sigmoid(t), the gate activation of the fused SwiGLU (hotdry.top,
+    "Metal GPU管线")."""
     return t / (1.0 + np.exp(-t))
 
 
 def expert_ffn(ex: DenseExpert, x: np.ndarray) -> np.ndarray:
-    """o = W_d (silu(W_g x) * (W_u x)) in float64."""
+    """o = W_d (silu(W_g x) * (W_u x)) in float64 (hotdry.top, "Metal GPU管线":
+    fused SwiGLU, then the down projection)."""
     x = np.asarray(x, dtype=np.float64)
     g = ex.Wg @ x
     u = ex.Wu @ x
@@ -186,11 +204,14 @@ def expert_ffn(ex: DenseExpert, x: np.ndarray) -> np.ndarray:
 
 
 def expert_hidden(ex: DenseExpert, x: np.ndarray) -> np.ndarray:
+    """h = silu(W_g x) * (W_u x), the SwiGLU hidden vector alone."""
     x = np.asarray(x, dtype=np.float64)
     return silu(ex.Wg @ x) * (ex.Wu @ x)
 
 
 def shared_sigma(gs: np.ndarray, x: np.ndarray) -> float:
+    """sigma = 1 / (1 + exp(-g_s . x)), the sigmoid gate of the shared expert
+    (hotdry.top, "Metal GPU管线"); a vector g_s is the reading."""
     s = float(np.asarray(gs, dtype=np.float64) @ np.asarray(x, dtype=np.float64))
     return 1.0 / (1.0 + math.exp(-s))
 
@@ -237,7 +258,9 @@ class OracleLayer:
         return idx, w, sig, l
 
     def forward(self, x: np.ndarray, resid: Optional[np.ndarray] = None) -> LayerResult:
-        """y = resid + sum_k w_k o_k(x) + sigma o_s(x); resid defaults to x."""
+        """y = resid + sum_k w_k o_k(x) + sigma o_s(x); resid defaults to x (the
+        fused combine with the residual and the sigmoid-gated shared expert of
+        hotdry.top, "Metal GPU管线")."""
         x = np.asarray(x, dtype=np.float64)
         r = x if resid is None else np.asarray(resid, dtype=np.float64)
         idx, w, sig, l = self.route(x)
@@ -262,7 +285,8 @@ class OracleLayer:
 def rmsnorm_bf16(h: np.ndarray, eps: float = 1e-6) -> np.ndarray:
     """n = bf16(h / sqrt(mean(h^2) + eps)), gamma = 1; returns bf16 bit patterns.
 
-    Two passes as on the pages: the sum of squares, then the scaling."""
+    Two passes, the sum of squares and then the scaling, as in hotdry.top,
+    "Metal GPU管线"; gamma = 1 and eps = 1e-6 are readings."""
     h = np.asarray(h, dtype=np.float64)
     ss = 0.0
     for v in h:
