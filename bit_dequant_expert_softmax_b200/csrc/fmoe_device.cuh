@@ -150,6 +150,11 @@ __device__ __noinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, u
   }
 }
 
+// The dequantised weight is code * scale + bias per 64-column group (hotdry.top,
+// "量化策略"); the juejin.cn shader section "Metal 着色器" rewrites the product as
+// fma(code, scale*x, bias*x).  Here the same sum is folded once per chunk:
+// scale * sum(code * x) + bias * sum(x).
+//
 // Codes as floats without conversion instructions: a code c masked in place at bit
 // offset s (s + bits <= 24) reads, as an IEEE float, exactly c * 2^s * 2^-149 (a
 // subnormal or the first normal binade).  The activation multiplying it is stored

@@ -21,6 +21,11 @@
 //            once to bf16
 //
 // There are no grid-wide waits: the kernel boundaries order the phases.
+//
+// The pages decode one token at a time (Flash-MoE); grouping a batch's (token,
+// expert) pairs by expert is this library's addition for batched decode, with the
+// per-pair arithmetic of the single-token path (hotdry.top, "量化策略" and "Metal
+// GPU管线").
 #pragma once
 
 #include "fmoe_device.cuh"

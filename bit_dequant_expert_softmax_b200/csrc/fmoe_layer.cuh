@@ -18,6 +18,15 @@
 // All weight bytes move HBM -> shared memory through the bulk-copy (TMA) engine
 // as contiguous row ranges, completion tracked by mbarriers; every wait (flags,
 // mbarriers) is bounded.
+//
+// What is computed follows the Flash-MoE pages: routing on the GPU (tinai-dev
+// README, "Pipeline mỗi lớp"), softmax then top-K on the probabilities
+// (intelliparadigm.com, section 2.1 router snippet; the selection is made on the
+// fp64 logits, the same order), 4-/2-bit codes dequantised as code * scale + bias
+// (hotdry.top, "量化策略"), fused SwiGLU and the fused combine with the residual and
+// the sigmoid-gated shared expert (hotdry.top, "Metal GPU管线").  How it is computed
+// (one persistent kernel, grid-wide flag exchanges, HBM-resident records) is this
+// library's own design for B200.
 #pragma once
 
 #include "fmoe_device.cuh"

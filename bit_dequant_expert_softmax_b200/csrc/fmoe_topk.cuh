@@ -1,7 +1,8 @@
 // Top-K selection by ranks, shared by the single-token and the batched kernels.
 //
 // The K largest router logits, ordered by logit descending with ties to the lower
-// expert index (the selection of the pages' softmax-then-top-K: the softmax is
+// expert index (the selection of the pages' softmax-then-top-K -- intelliparadigm.com,
+// section 2.1 router snippet; tinai-dev README, "Pipeline mỗi lớp" -- the softmax is
 // monotone, so ranking logits or probabilities picks the same experts), compared
 // through the order-preserving 64-bit key of each fp64 logit.  Two levels of ranks,
 // no dependent reductions: every expert's rank within its group of 32 consecutive
