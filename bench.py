@@ -41,7 +41,10 @@ def parse():
     ap.add_argument("--impl", default="fmoe", choices=["fmoe", "reference"])
     ap.add_argument("--config", default="layer4096")
     ap.add_argument("--tokens", type=int, default=None)
-    ap.add_argument("--cpu-sample", type=int, default=4, help="tokens timed for the CPU oracle baseline")
+    ap.add_argument("--cpu-sample", type=int, default=10,
+                    help="tokens timed once for the CPU oracle baseline of the GPU arm")
+    ap.add_argument("--ref-tokens", type=int, default=1,
+                    help="tokens per step of the reference arm (the CPU oracle)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -204,7 +207,7 @@ def run_reference(args, rank):
     if rank != 0:
         return
     shape = synth.CONFIGS[args.config]["shape"]
-    per_step = max(1, args.cpu_sample)
+    per_step = max(1, args.ref_tokens)
     for _ in range(args.warmup and 1):
         cpu_oracle_rate(shape, 1)
     t_all = 0.0
