@@ -78,3 +78,46 @@ def test_stack_and_batch_argument_checks(lib):
     assert L.fmoe_layer_forward_batched(None, None, None, 1, None, None) == 1
     assert L.fmoe_block_forward_batched(None, None, 1, 1e-6, None, None) == 1
     assert L.fmoe_route_batched(None, None, 1, None, None, None, None) == 1
+
+
+def _create(lib, cfg, experts=0x10000, router=0x20000, bias=0x30000, gate=0x40000):
+    """fmoe_layer_create with fake (never dereferenced) weight addresses."""
+    L = lib.lib()
+    h = ctypes.c_void_p()
+    w = lib.fmoe_weights(experts, router, bias, gate)
+    return L.fmoe_layer_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)), h
+
+
+@pytest.mark.parametrize("fields", [
+    (4000, 1024, 512, 4, 4, 1, 0),   # hidden not a multiple of 64
+    (4096, 1000, 512, 4, 4, 1, 0),   # inter not a multiple of 64
+    (4096, 1024, 512, 4, 3, 1, 0),   # bits other than 2 or 4
+    (4096, 1024, 512, 0, 4, 1, 0),   # K = 0
+    (4096, 1024, 4, 5, 4, 1, 0),     # K > E
+    (4096, 1024, 0, 1, 4, 1, 0),     # no experts
+    (4096, 1024, 512, 4, 4, 2, 0),   # has_shared not 0/1
+    (4096, 1024, 512, 4, 4, 1, 7),   # has_router_bias not 0/1
+    (-64, 1024, 512, 4, 4, 1, 0),    # negative size
+])
+def test_invalid_configs_are_rejected_on_the_host(lib, fields):
+    cfg = lib.fmoe_config(*fields)
+    assert lib.fmoe_workspace_bytes(cfg) == 0
+    assert _create(lib, cfg)[0] == 1
+
+
+def test_weight_pointer_checks(lib):
+    cfg = lib.fmoe_config(4096, 1024, 512, 4, 4, 1, 1)
+    assert _create(lib, cfg, experts=0x10000 + 128)[0] == 1      # records not 256-byte aligned
+    assert _create(lib, cfg, router=0x20000 + 8)[0] == 1         # router not 16-byte aligned
+    assert _create(lib, cfg, gate=0)[0] == 1                     # shared expert without its gate
+    assert _create(lib, cfg, gate=0x40000 + 4)[0] == 1
+    assert _create(lib, cfg, bias=0)[0] == 1                     # router bias declared, not given
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the behaviour without a device")
+def test_no_device_fails_loudly(lib):
+    """Valid arguments but no CUDA device: the library refuses (FMOE_ERR_CUDA) instead of
+    falling back to anything."""
+    cfg = lib.fmoe_config(4096, 1024, 512, 4, 4, 1, 1)
+    st, h = _create(lib, cfg)
+    assert st == 3 and not h.value
