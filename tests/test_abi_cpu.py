@@ -121,3 +121,13 @@ def test_no_device_fails_loudly(lib):
     cfg = lib.fmoe_config(4096, 1024, 512, 4, 4, 1, 1)
     st, h = _create(lib, cfg)
     assert st == 3 and not h.value
+
+
+def test_missing_library_raises(lib, monkeypatch, tmp_path):
+    """Without the built library the binding raises; nothing else is tried."""
+    monkeypatch.setattr(lib, "_lib", None)
+    monkeypatch.setattr(lib, "SO", str(tmp_path / "libfmoe.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        lib.lib()
+    with pytest.raises(RuntimeError):
+        lib.fmoe_record_bytes(4096, 1024, 4)
