@@ -1,0 +1,80 @@
+"""IEEE identities the dequantising dot products rely on (CPU, numpy float32).
+
+The single-token kernel reads a code masked in place at bit offset s of a 32-bit word
+as a float32 and multiplies it by an activation stored pre-scaled by 2^(100 - s).
+These tests check, for every code and every position of 4- and 2-bit words:
+  - the masked bit pattern read as float32 is exactly code * 2^(s - 149) (a subnormal,
+    or the first normal binade when bit 23 is set);
+  - the pre-scale factor 2^(100 - s) is a plain power of two built from its exponent;
+  - code * (x * 2^(100 - s)) equals code * x * 2^-49 exactly for bf16 activations, so
+    the per-chunk sum needs one rescale by 2^49;
+  - the positions whose code would cross bit 24 are read from the word shifted right by
+    8 without picking up bits of the neighbouring word.
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+PRE_EXP = 100
+
+
+def shift_pos(bits, p):
+    """Bit offset at which position p of a word is masked (after the 8-bit shift when
+    the code would end above bit 24)."""
+    return bits * p - 8 if bits * p + bits > 24 else bits * p
+
+
+def as_f32(pattern):
+    return np.array([pattern], dtype=np.uint32).view(np.float32)[0]
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_masked_code_reads_as_scaled_subnormal(bits):
+    for p in range(32 // bits):
+        s = shift_pos(bits, p)
+        assert 0 <= s and s + bits <= 24
+        for c in range(1 << bits):
+            v = float(as_f32(c << s))
+            assert v == c * 2.0 ** (s - 149), (bits, p, c)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_prescale_factor_is_the_power_of_two(bits):
+    for p in range(32 // bits):
+        s = shift_pos(bits, p)
+        assert float(as_f32((127 + PRE_EXP - s) << 23)) == 2.0 ** (PRE_EXP - s)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_products_with_prescaled_bf16_activations_are_exact(bits):
+    rng = np.random.default_rng(0)
+    x = oracle.bf16_to_f64(oracle.f64_to_bf16_bits(rng.standard_normal(256) * np.exp(rng.standard_normal(256) * 3)))
+    for p in range(32 // bits):
+        s = shift_pos(bits, p)
+        xs = (x * 2.0 ** (PRE_EXP - s)).astype(np.float32)
+        assert np.array_equal(xs.astype(np.float64), x * 2.0 ** (PRE_EXP - s))  # scaling is exact
+        for c in range(1 << bits):
+            prod = (as_f32(c << s) * xs).astype(np.float64)   # float32 multiply
+            assert np.array_equal(prod, c * x * 2.0 ** (PRE_EXP - 149)), (bits, p, c)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_shifted_pair_does_not_mix_words(bits):
+    """Two words viewed as one 64-bit value (w_a low, w_b high), shifted right by 8: the
+    masks of the high positions select only w_a's (resp. w_b's) own bits."""
+    rng = np.random.default_rng(1)
+    for _ in range(200):
+        wa, wb = (int(v) for v in rng.integers(0, 2 ** 32, size=2, dtype=np.uint64))
+        pair = (wb << 32) | wa
+        shifted = pair >> 8
+        for p in range(32 // bits):
+            if bits * p + bits <= 24:
+                continue
+            s = shift_pos(bits, p)
+            m32 = ((1 << bits) - 1) << s
+            mask = (m32 << 32) | m32
+            got = shifted & mask
+            code_a = (wa >> (bits * p)) & ((1 << bits) - 1)
+            code_b = (wb >> (bits * p)) & ((1 << bits) - 1)
+            assert got == ((code_b << s) << 32) | (code_a << s), (bits, p)
