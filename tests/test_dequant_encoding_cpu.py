@@ -78,3 +78,68 @@ def test_shifted_pair_does_not_mix_words(bits):
             code_a = (wa >> (bits * p)) & ((1 << bits) - 1)
             code_b = (wb >> (bits * p)) & ((1 << bits) - 1)
             assert got == ((code_b << s) << 32) | (code_a << s), (bits, p)
+
+
+# ------------------------------------------------------------- batched path --
+# The grouped (tensor-core) matvecs enter a code c as the bf16 value 1 + c/2^b' (b' = 4
+# for 4-bit codes, 2 for 2-bit), built by one rotate and one mask-and-or from the code
+# word, and fold each 64-column group's accumulator D = sum (1 + c/2^b') x with the
+# group's scale and bias.
+
+def rotr(w, n):
+    n &= 31
+    return ((w >> n) | (w << (32 - n))) & 0xFFFFFFFF if n else w
+
+
+def bf16_value(bits16):
+    return float(np.array([bits16 << 16], dtype=np.uint32).view(np.float32)[0])
+
+
+def test_rotate_builds_bf16_pairs_of_4bit_codes():
+    rng = np.random.default_rng(2)
+    for w in [0, 0xFFFFFFFF, 0x76543210, 0xFEDCBA98] + [int(v) for v in rng.integers(0, 2 ** 32, 50, dtype=np.uint64)]:
+        for q in range(4):
+            r = (rotr(w, 4 * q - 3) & 0x00780078) | 0x3F803F80
+            lo, hi = (w >> (4 * q)) & 15, (w >> (4 * (q + 4))) & 15
+            assert bf16_value(r & 0xFFFF) == 1 + lo / 16 and bf16_value(r >> 16) == 1 + hi / 16
+
+
+def test_rotate_builds_bf16_pairs_of_2bit_codes():
+    rng = np.random.default_rng(3)
+    for w in [0, 0xFFFFFFFF, 0xE4E4E4E4] + [int(v) for v in rng.integers(0, 2 ** 32, 50, dtype=np.uint64)]:
+        for q in range(4):
+            for h in range(2):
+                r = (rotr(w, 2 * q + 8 * h - 5) & 0x00600060) | 0x3F803F80
+                k = q + 4 * h
+                lo, hi = (w >> (2 * k)) & 3, (w >> (2 * (k + 8))) & 3
+                assert bf16_value(r & 0xFFFF) == 1 + lo / 4 and bf16_value(r >> 16) == 1 + hi / 4
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_group_fold_identity_is_exact(bits):
+    """sum_c (s c + b) x_c = (2^b' s) D + (b - 2^b' s) X, in exact rational arithmetic."""
+    from fractions import Fraction
+    rng = np.random.default_rng(4)
+    for _ in range(20):
+        c = rng.integers(0, 1 << bits, 64)
+        x = oracle.bf16_to_f64(oracle.f64_to_bf16_bits(rng.standard_normal(64)))
+        s = float(oracle.bf16_to_f64(oracle.f64_to_bf16_bits(np.array([abs(rng.standard_normal()) * 0.02])))[0])
+        b = float(oracle.bf16_to_f64(oracle.f64_to_bf16_bits(
+            np.array([-(2 ** bits / 2) * s + rng.standard_normal() * 1e-3])))[0])
+        F = [Fraction(float(v)) for v in x]
+        lhs = sum((Fraction(s) * int(ci) + Fraction(b)) * xi for ci, xi in zip(c, F))
+        D = sum((1 + Fraction(int(ci), 2 ** bits)) * xi for ci, xi in zip(c, F))
+        X = sum(F)
+        assert lhs == Fraction(2 ** bits) * Fraction(s) * D + (Fraction(b) - Fraction(2 ** bits) * Fraction(s)) * X
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_fold_coefficients_exact_in_fp32_for_the_workload(bits):
+    """b - 2^b' s is exact in float32 for the workload's (scale, bias) values."""
+    import fmoe_synth as synth
+    p = synth.gen_expert(0, 0, 3, 512, 128, bits)
+    for sb in (p.gate_sb, p.up_sb, p.down_sb):
+        s = oracle.bf16_to_f64((sb & 0xFFFF).astype(np.uint16))
+        b = oracle.bf16_to_f64((sb >> 16).astype(np.uint16))
+        f32 = (b.astype(np.float32) - (s * 2 ** bits).astype(np.float32)).astype(np.float64)
+        assert np.array_equal(f32, b - s * 2 ** bits)
