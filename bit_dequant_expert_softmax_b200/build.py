@@ -9,8 +9,20 @@ SO = os.path.join(HERE, "libfmoe.so")
 CSRC = os.path.join(HERE, "csrc")
 MAIN = os.path.join(CSRC, "fmoe_api.cu")
 
+# -ftz=false is explicit: the single-token dot products read 4-/2-bit codes masked in
+# place as subnormal floats (code * 2^(s - 149)); flushing subnormals to zero would turn
+# every code into 0.  Fast-math flags imply flushing and are refused below.
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
-              "-Xcompiler", "-fPIC", "-shared"]
+              "-ftz=false", "-Xcompiler", "-fPIC", "-shared"]
+FORBIDDEN_FLAGS = ("-ftz=true", "--use_fast_math", "-use_fast_math", "--ftz=true")
+
+
+def check_flags(flags) -> None:
+    """Raises if the flags would flush subnormals (the kernels rely on them)."""
+    bad = [f for f in flags if f in FORBIDDEN_FLAGS]
+    if bad:
+        raise ValueError(f"libfmoe.so must be built without {bad}: its dequantising dot products "
+                         "read codes as subnormal floats")
 
 
 def _sources():
@@ -22,6 +34,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         newest = max(os.path.getmtime(s) for s in _sources())
         if os.path.getmtime(SO) >= newest:
             return SO
+    check_flags(NVCC_FLAGS)
     cmd = ["nvcc", *NVCC_FLAGS, MAIN, "-o", SO]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")

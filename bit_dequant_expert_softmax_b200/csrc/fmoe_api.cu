@@ -131,6 +131,7 @@ struct fmoe_layer {
   int hold_cta;
   uint64_t* timeline;
   int timeline_token;
+  int used_noalloc;  // fmoe_layer_forward_noalloc has run this layer (its errors land in the fixed array)
   // batched path
   void* bws;
   size_t bws_bytes;
@@ -207,6 +208,17 @@ fmoe_status plan(fmoe_layer* L) {
   return FMOE_OK;
 }
 
+// Pointers of the single-token kernel's scratch words inside a workspace laid out as
+// `w` (the caller's workspace, or the fixed array of fmoe_layer_forward_noalloc).
+void set_workspace_ptrs(Params& p, const WsLayout& w, uint8_t* ws) {
+  p.err = reinterpret_cast<uint32_t*>(ws + w.err);
+  p.tokens = reinterpret_cast<uint32_t*>(ws + w.tokens);
+  p.rflags = reinterpret_cast<uint32_t*>(ws + w.rflags);
+  p.hflags = reinterpret_cast<uint32_t*>(ws + w.hflags);
+  p.lpart = reinterpret_cast<double*>(ws + w.lpart);
+  p.hbuf = reinterpret_cast<float*>(ws + w.hbuf);
+}
+
 Params base_params(const fmoe_layer* L, int mode, int T) {
   Params p{};
   const fmoe_config& c = L->cfg;
@@ -233,13 +245,7 @@ Params base_params(const fmoe_layer* L, int mode, int T) {
   p.router = L->w.router;
   p.rbias = L->w.router_bias;
   p.sgate = L->w.shared_gate;
-  uint8_t* ws = static_cast<uint8_t*>(L->ws);
-  p.err = reinterpret_cast<uint32_t*>(ws + L->wsl.err);
-  p.tokens = reinterpret_cast<uint32_t*>(ws + L->wsl.tokens);
-  p.rflags = reinterpret_cast<uint32_t*>(ws + L->wsl.rflags);
-  p.hflags = reinterpret_cast<uint32_t*>(ws + L->wsl.hflags);
-  p.lpart = reinterpret_cast<double*>(ws + L->wsl.lpart);
-  p.hbuf = reinterpret_cast<float*>(ws + L->wsl.hbuf);
+  if (L->ws) set_workspace_ptrs(p, L->wsl, static_cast<uint8_t*>(L->ws));
   p.staging_bytes = L->staging_bytes;
   p.wait_ns = L->wait_ns;
   p.hold_cta = L->hold_cta;
@@ -415,6 +421,49 @@ fmoe_status ready(const fmoe_layer* L) {
   if (!L) return FMOE_ERR_INVALID_ARG;
   if (!L->ws) return FMOE_ERR_NO_WORKSPACE;
   return FMOE_OK;
+}
+
+// The fixed scratch array of fmoe_layer_forward_noalloc (one per device that loads the
+// library) and its device address per device.
+__device__ __align__(256) uint8_t g_noalloc_scratch[FMOE_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the array on device `dev` (current); looked up once per device.
+// In host code the array's name is only a host-side handle, never a device address.
+fmoe_status noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (dev < 0 || dev >= kMaxDevices) return FMOE_ERR_UNSUPPORTED;
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FMOE_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FMOE_OK;
+}
+
+// Device error bits of the last fmoe_layer_forward_noalloc call on L's device (they live
+// in the fixed array's error word, shared by every layer that uses it); cleared with the
+// array's control words when set.  No allocation: the copies go to and from host
+// variables through the array's cached device address.
+fmoe_status noalloc_get_error(const fmoe_layer* L, uint32_t* device_error) {
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return FMOE_ERR_CUDA;
+  if (cur != L->device) return FMOE_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  const fmoe_status st = noalloc_scratch(L->device, &scratch);
+  if (st != FMOE_OK) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  uint32_t e = 0;
+  if (cudaMemcpy(&e, ws + L->wsl.err, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return FMOE_ERR_CUDA;
+  *device_error = e;
+  if (e == 0) return FMOE_OK;
+  if (cudaMemset(ws, 0, L->wsl.lpart) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
+  return FMOE_ERR_DEVICE;
 }
 
 }  // namespace
@@ -642,7 +691,7 @@ fmoe_status fmoe_rmsnorm(const uint16_t* h, uint16_t* out, int T, int H, double 
 fmoe_status fmoe_layer_get_error(fmoe_layer_t L, uint32_t* device_error) {
   if (!L || !device_error) return FMOE_ERR_INVALID_ARG;
   *device_error = 0;
-  if (!L->ws && !L->bws) return FMOE_OK;
+  if (!L->ws && !L->bws) return L->used_noalloc ? noalloc_get_error(L, device_error) : FMOE_OK;
   if (cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
   uint32_t e = 0, eb = 0;
   uint8_t* ws = static_cast<uint8_t*>(L->ws);
@@ -805,42 +854,6 @@ fmoe_status fmoe_graph_destroy(fmoe_graph_t G) {
 // ---------------------------------------------------------------------------
 // fmoe_layer_forward_noalloc: the same fused kernel with its scratch in a fixed
 // file-scope device array instead of a caller-provided workspace.
-}  // extern "C"
-
-namespace {
-
-__device__ __align__(256) uint8_t g_noalloc_scratch[FMOE_NOALLOC_SCRATCH_BYTES];
-
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of the array on device `dev` (current); looked up once per device.
-// In host code the array's name is only a host-side handle, never a device address.
-fmoe_status noalloc_scratch(int dev, void** out) {
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (dev < 0 || dev >= kMaxDevices) return FMOE_ERR_UNSUPPORTED;
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FMOE_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
-  return FMOE_OK;
-}
-
-void set_workspace_ptrs(Params& p, const WsLayout& w, uint8_t* ws) {
-  p.err = reinterpret_cast<uint32_t*>(ws + w.err);
-  p.tokens = reinterpret_cast<uint32_t*>(ws + w.tokens);
-  p.rflags = reinterpret_cast<uint32_t*>(ws + w.rflags);
-  p.hflags = reinterpret_cast<uint32_t*>(ws + w.hflags);
-  p.lpart = reinterpret_cast<double*>(ws + w.lpart);
-  p.hbuf = reinterpret_cast<float*>(ws + w.hbuf);
-}
-
-}  // namespace
-
-extern "C" {
 
 fmoe_status fmoe_layer_forward_noalloc(fmoe_layer_t L, const uint16_t* x, const uint16_t* resid, int T, uint16_t* y,
                                        void* stream) {
@@ -864,6 +877,7 @@ fmoe_status fmoe_layer_forward_noalloc(fmoe_layer_t L, const uint16_t* x, const 
   p.x = x;
   p.resid = resid;
   p.y = y;
+  L->used_noalloc = 1;
   // the memset above precedes the launch: no programmatic overlap with it
   return launch(L, p, stream, false);
 }

@@ -158,8 +158,14 @@ __device__ __noinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, u
 // Codes as floats without conversion instructions: a code c masked in place at bit
 // offset s (s + bits <= 24) reads, as an IEEE float, exactly c * 2^s * 2^-149 (a
 // subnormal or the first normal binade).  The activation multiplying it is stored
-// pre-scaled by 2^(kPreExp - s), so every product is code * x * 2^(kPreExp - 149)
-// exactly, and the per-chunk sum is rescaled by 2^(149 - kPreExp) once.
+// pre-scaled by 2^(P - s), so every product is code * x * 2^(P - 149) exactly, and the
+// per-chunk sum is rescaled by 2^(149 - P) once.  P is chosen per chunk from the
+// largest exponent e of the chunk's activations, P = 100 - e (e clamped to
+// [kMinExp, kMaxExp]): the pre-scaled values stay below 2^101 and the products of the
+// chunk's largest activations near 2^-45, far inside the normal range, whatever the
+// activations' magnitude (the clamp keeps the factor 2^(P - s) and the rescale
+// 2^(149 - P) representable; it leaves |x| < 2^-103 or |x| >= 2^105 outside the exact
+// range).
 //
 // Codes are taken in pairs from two adjacent words {w_a, w_b} of a 16-byte load,
 // viewed as one 64-bit register: a 64-bit AND with the same mask in both halves
@@ -169,7 +175,20 @@ __device__ __noinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, u
 // selected by the masks).  The activations are laid out so that one 64-bit shared
 // load gives the matching pair {x(word a, p), x(word b, p)}.
 constexpr int kPreExp = 100;
-constexpr float kUnscale = 562949953421312.0f;  // 2^(149 - kPreExp) = 2^49
+constexpr int kMinExp = -26;
+constexpr int kMaxExp = 78;
+
+// Pre-scale exponent P of a chunk whose largest |activation| has the float bit pattern
+// `maxbits` (sign cleared).
+__device__ __forceinline__ int chunk_pre(uint32_t maxbits) {
+  const int e = static_cast<int>(maxbits >> 23) - 127;
+  return kPreExp - min(max(e, kMinExp), kMaxExp);
+}
+
+// 2^(149 - P): the rescale of a chunk's sum of products.
+__device__ __forceinline__ float chunk_unscale(int pre) {
+  return __uint_as_float(static_cast<uint32_t>(127 + 149 - pre) << 23);
+}
 
 __device__ __forceinline__ void fma2(unsigned long long& acc, unsigned long long c, unsigned long long x) {
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(c), "l"(x));
@@ -257,8 +276,16 @@ struct Chunk {
   }
 };
 
-__device__ __forceinline__ float prescale_factor(int shift) {
-  return __uint_as_float(static_cast<uint32_t>(127 + kPreExp - shift) << 23);
+// 2^(P - shift): the pre-scale of an activation met by codes masked at bit `shift`.
+__device__ __forceinline__ float prescale_factor(int pre, int shift) {
+  return __uint_as_float(static_cast<uint32_t>(127 + pre - shift) << 23);
+}
+
+// Largest |v| bit pattern of four floats (sign bits cleared; NaN-free inputs).
+__device__ __forceinline__ uint32_t max_abs_bits(float4 v) {
+  const uint32_t a = max(__float_as_uint(v.x) & 0x7FFFFFFFu, __float_as_uint(v.y) & 0x7FFFFFFFu);
+  const uint32_t b = max(__float_as_uint(v.z) & 0x7FFFFFFFu, __float_as_uint(v.w) & 0x7FFFFFFFu);
+  return max(a, b);
 }
 
 // (scale, bias) pair word -> floats
@@ -277,9 +304,11 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   return v;
 }
 
-// Order-preserving map of a double to an unsigned key (larger double -> larger key).
+// Order-preserving map of a double to an unsigned key (larger double -> larger key);
+// -0.0 and +0.0 get the same key (they compare equal, so they tie).
 __device__ __forceinline__ unsigned long long dkey(double d) {
-  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(d));
+  unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(d));
+  if (b == 0x8000000000000000ull) b = 0ull;
   return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
 

@@ -139,11 +139,11 @@ struct Geometry {
     return static_cast<uint32_t>((n / cols + 31) / 32) * 32u * static_cast<uint32_t>(cols);
   }
   __host__ __device__ uint32_t h_bytes() const {
-    return r128(static_cast<uint32_t>(nslots) * padded(I) * 4u + static_cast<uint32_t>(nslots) * (I / cols) * 4u);
+    return r128(static_cast<uint32_t>(nslots) * padded(I) * 4u + static_cast<uint32_t>(nslots) * (I / cols) * 8u);
   }
-  // header + activations + chunk sums, before the staging area
+  // header + activations + per-chunk (sum, rescale) pairs, before the staging area
   __host__ __device__ uint32_t fixed_bytes(uint32_t header) const {
-    return r128(header + padded(H) * 4u + static_cast<uint32_t>(H / cols) * 4u);
+    return r128(header + padded(H) * 4u + static_cast<uint32_t>(H / cols) * 8u);
   }
   __host__ __device__ uint32_t router_item() const { return static_cast<uint32_t>(H) * 4u; }
 };
@@ -158,7 +158,7 @@ struct LayerKernel {
   Geometry g;
   SmemHeader* hdr;
   float* xs;       // pre-scaled, lane-interleaved activations [padded H]
-  float* xsum;     // per-chunk sums of the unscaled activations [H / kCols]
+  float2* xsum;    // per chunk: (sum of the unscaled activations, rescale 2^(149 - P)) [H / kCols]
   uint8_t* stage;  // staging area
   uint32_t cap;    // staging bytes
   uint32_t nitem;  // items issued so far (same value in every thread)
@@ -170,7 +170,7 @@ struct LayerKernel {
     g = Geometry{p.H, p.I, p.qh, p.qi, p.sh, p.si, p.rp, p.db, nslots, C::kCols};
     hdr = reinterpret_cast<SmemHeader*>(smem);
     xs = reinterpret_cast<float*>(smem + sizeof(SmemHeader));
-    xsum = xs + g.padded(p.H);
+    xsum = reinterpret_cast<float2*>(xs + g.padded(p.H));
     stage = smem + g.fixed_bytes(sizeof(SmemHeader));
     cap = static_cast<uint32_t>(p.staging_bytes);
     nitem = 0;
@@ -327,19 +327,23 @@ struct LayerKernel {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
         const float4 v = bf16x4(nat[k]);
         float sum = (v.x + v.y) + (v.z + v.w);
+        uint32_t mx = max_abs_bits(v);
 #pragma unroll
-        for (int o = 1; o < TPC; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        for (int o = 1; o < TPC; o <<= 1) {
+          sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
         if (q < n4) {
           if (xa) {
             xa[q] = make_double2(v.x, v.y);
             xb[q] = make_double2(v.z, v.w);
           }
-          const int c0 = 4 * q;
-          xs[phys(c0 + 0)] = v.x * prescale_factor(C::shift_of(c0 + 0));
-          xs[phys(c0 + 1)] = v.y * prescale_factor(C::shift_of(c0 + 1));
-          xs[phys(c0 + 2)] = v.z * prescale_factor(C::shift_of(c0 + 2));
-          xs[phys(c0 + 3)] = v.w * prescale_factor(C::shift_of(c0 + 3));
-          if (q % TPC == 0) xsum[q / TPC] = sum;
+          const int c0 = 4 * q, pre = chunk_pre(mx);
+          xs[phys(c0 + 0)] = v.x * prescale_factor(pre, C::shift_of(c0 + 0));
+          xs[phys(c0 + 1)] = v.y * prescale_factor(pre, C::shift_of(c0 + 1));
+          xs[phys(c0 + 2)] = v.z * prescale_factor(pre, C::shift_of(c0 + 2));
+          xs[phys(c0 + 3)] = v.w * prescale_factor(pre, C::shift_of(c0 + 3));
+          if (q % TPC == 0) xsum[q / TPC] = make_float2(sum, chunk_unscale(pre));
         }
       }
     }
@@ -349,7 +353,7 @@ struct LayerKernel {
   // has published): coalesced 16-byte loads (thread -> 4 consecutive columns), all of
   // a thread's loads in flight together; chunk sums by shuffles over the kCols/4
   // threads of a chunk; pre-scaled values scattered into the interleaved layout.
-  __device__ void stage_h(const float* hb, float* hs, uint32_t hstride, float* hsum) {
+  __device__ void stage_h(const float* hb, float* hs, uint32_t hstride, float2* hsum) {
     constexpr int TPC = C::kCols / 4;
     const int per_slot = p.I / 4, nch = p.I / C::kCols;
     const int n4 = nslots * per_slot;
@@ -365,16 +369,20 @@ struct LayerKernel {
       for (int k = 0; k < 4; ++k) {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
         float sum = (v[k].x + v[k].y) + (v[k].z + v[k].w);
+        uint32_t mx = max_abs_bits(v[k]);
 #pragma unroll
-        for (int o = 1; o < TPC; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        for (int o = 1; o < TPC; o <<= 1) {
+          sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
         if (q < n4) {
-          const int slot = q / per_slot, c0 = (q % per_slot) * 4;
+          const int slot = q / per_slot, c0 = (q % per_slot) * 4, pre = chunk_pre(mx);
           float* d = hs + static_cast<size_t>(slot) * hstride;
-          d[phys(c0 + 0)] = v[k].x * prescale_factor(C::shift_of(c0 + 0));
-          d[phys(c0 + 1)] = v[k].y * prescale_factor(C::shift_of(c0 + 1));
-          d[phys(c0 + 2)] = v[k].z * prescale_factor(C::shift_of(c0 + 2));
-          d[phys(c0 + 3)] = v[k].w * prescale_factor(C::shift_of(c0 + 3));
-          if (q % TPC == 0) hsum[slot * nch + c0 / C::kCols] = sum;
+          d[phys(c0 + 0)] = v[k].x * prescale_factor(pre, C::shift_of(c0 + 0));
+          d[phys(c0 + 1)] = v[k].y * prescale_factor(pre, C::shift_of(c0 + 1));
+          d[phys(c0 + 2)] = v[k].z * prescale_factor(pre, C::shift_of(c0 + 2));
+          d[phys(c0 + 3)] = v[k].w * prescale_factor(pre, C::shift_of(c0 + 3));
+          if (q % TPC == 0) hsum[slot * nch + c0 / C::kCols] = make_float2(sum, chunk_unscale(pre));
         }
       }
       if (base == 0) mark(14);
@@ -389,7 +397,7 @@ struct LayerKernel {
   // sharing the activation loads (W = scale*code + bias; v pre-scaled, interleaved).
   template <bool TWO>
   __device__ __forceinline__ void dotn(const uint8_t* q0, const uint32_t* s0, const uint8_t* q1,
-                                       const uint32_t* s1, const float* vs, const float* vsum, int nch, float& r0,
+                                       const uint32_t* s1, const float* vs, const float2* vsum, int nch, float& r0,
                                        float& r1) const {
     const int lane = threadIdx.x & 31;
 #pragma unroll 2
@@ -402,14 +410,14 @@ struct LayerKernel {
       unsigned long long a0 = 0ull, a1 = 0ull, b0 = 0ull, b1 = 0ull;
       C::template word_pair2<TWO>(a.x, b.x, xv0, a0, b0);
       C::template word_pair2<TWO>(a.y, b.y, xv1, a1, b1);
-      const float vm = vsum[m];
+      const float2 vm = vsum[m];  // (sum of the chunk's activations, rescale of its products)
       const uint32_t sa = s0[C::sb_index(m)];
-      r0 = fmaf(sb_scale(sa), (pair_sum(a0) + pair_sum(a1)) * kUnscale, r0);
-      r0 = fmaf(sb_bias(sa), vm, r0);
+      r0 = fmaf(sb_scale(sa), (pair_sum(a0) + pair_sum(a1)) * vm.y, r0);
+      r0 = fmaf(sb_bias(sa), vm.x, r0);
       if (TWO) {
         const uint32_t sbv = s1[C::sb_index(m)];
-        r1 = fmaf(sb_scale(sbv), (pair_sum(b0) + pair_sum(b1)) * kUnscale, r1);
-        r1 = fmaf(sb_bias(sbv), vm, r1);
+        r1 = fmaf(sb_scale(sbv), (pair_sum(b0) + pair_sum(b1)) * vm.y, r1);
+        r1 = fmaf(sb_bias(sbv), vm.x, r1);
       }
     }
   }
@@ -576,7 +584,7 @@ struct LayerKernel {
   }
 
   // Consume a down item (rows [ja, ja+n)): y = resid + sum_s w_s o_s.
-  __device__ bool down_item(uint32_t item, uint32_t off, int ja, int n, const float* hs, const float* hsum,
+  __device__ bool down_item(uint32_t item, uint32_t off, int ja, int n, const float* hs, const float2* hsum,
                             const uint16_t* resid_t, uint16_t* y_t) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ia = warp, ib = warp + kWarps;
@@ -594,7 +602,7 @@ struct LayerKernel {
       const uint32_t* sbase = reinterpret_cast<const uint32_t*>(blk + g.dn_q(n) + lead);
       float oa = 0.f, ob = 0.f;
       const float* hsl = hs + static_cast<size_t>(s) * g.padded(p.I);
-      const float* hsm = hsum + static_cast<size_t>(s) * nch;
+      const float2* hsm = hsum + static_cast<size_t>(s) * nch;
       if (two)
         dotn<true>(blk + static_cast<uint32_t>(ia) * p.qi, sbase + ia * (p.si / 4),
                    blk + static_cast<uint32_t>(ib) * p.qi, sbase + ib * (p.si / 4), hsl, hsm, nch, oa, ob);
@@ -845,7 +853,7 @@ struct LayerKernel {
     const uint32_t hbase = prefetch ? hoff : 0u;
     float* hs = reinterpret_cast<float*>(stage + hbase);
     const uint32_t hstride = g.padded(p.I);
-    float* hsum = hs + static_cast<size_t>(nslots) * hstride;
+    float2* hsum = reinterpret_cast<float2*>(hs + static_cast<size_t>(nslots) * hstride);
     if (!wait_all(p.hflags, tok_)) {
       if (threadIdx.x == 0) hdr->abort_flag = 1;
       __syncthreads();

@@ -142,7 +142,12 @@ fmoe_status fmoe_expert_forward(fmoe_layer_t layer, const uint16_t* x, const uin
 
 /* The whole layer: routing, experts and combine, one token after another:
  * y[t] = resid[t] + sum_k w_k o_k(x[t]) + sigma o_s(x[t]).  resid may equal x; y may
- * alias resid but not x. */
+ * alias resid but not x.
+ * Range: the dequantising dot products scale each chunk of 32 (4-bit) or 64 (2-bit)
+ * activations by a power of two chosen from the chunk's largest magnitude, so their
+ * products stay exact for activations x (and hidden values h = silu(W_g x)(W_u x))
+ * from about 2^-103 to 2^105 in magnitude whatever their spread; h and the outputs must
+ * fit fp32 (and y bf16), which bounds useful inputs well inside that range. */
 fmoe_status fmoe_layer_forward(fmoe_layer_t layer, const uint16_t* x, const uint16_t* resid, int T,
                                uint16_t* y, void* stream);
 
@@ -239,7 +244,10 @@ fmoe_status fmoe_graph_destroy(fmoe_graph_t graph);
 
 /* Synchronises the device, returns the layer's device error bits in *device_error
  * (0 if none) and clears them (and the layer's barrier state).  Returns FMOE_OK when no
- * error was set, FMOE_ERR_DEVICE when one was. */
+ * error was set, FMOE_ERR_DEVICE when one was.  A layer without any workspace that has
+ * run fmoe_layer_forward_noalloc reports the bits of the last fmoe_layer_forward_noalloc
+ * call on its device (whatever layer made it: the calls share one array) and clears
+ * them; call it with that device current. */
 fmoe_status fmoe_layer_get_error(fmoe_layer_t layer, uint32_t* device_error);
 
 /* Upper bound, in nanoseconds, of every device-side wait of this layer (grid-wide
@@ -282,12 +290,15 @@ int fmoe_layer_grid_size(fmoe_layer_t layer);
  * A layer whose fmoe_workspace_bytes() exceed that size is rejected with
  * FMOE_ERR_SCRATCH_LIMIT before anything is enqueued.  The first call on a device
  * looks up the array's device address (cudaGetSymbolAddress, with that device
- * current), so make that first call before any stream capture.  Each call first
- * clears the array's control words (an asynchronous memset on `stream`, no
- * allocation) and nothing else allocates or frees memory.  All calls, on all layers
- * and streams, share the one array: calls that overlap on the GPU race and must be
- * ordered by the caller.  Device-side error bits of a call land in the array's
- * control words, which the next call clears; they are not reported. */
+ * current), so make that first call before any stream capture.  That address is cached
+ * per device for the life of the process: after cudaDeviceReset() on a device the
+ * cached address belongs to the destroyed context, and the library must not be used on
+ * that device again.  Each call first clears the array's control words (an
+ * asynchronous memset on `stream`, no allocation) and nothing else allocates or frees
+ * memory.  All calls, on all layers and streams, share the one array: calls that
+ * overlap on the GPU race and must be ordered by the caller.  Device-side error bits of
+ * a call land in the array's error word; fmoe_layer_get_error on a layer without
+ * workspace reads and clears them, and the next call clears them too. */
 fmoe_status fmoe_layer_forward_noalloc(fmoe_layer_t layer, const uint16_t* x, const uint16_t* resid, int T,
                                        uint16_t* y, void* stream);
 

@@ -20,7 +20,7 @@ Sources (the Flash-MoE pages):
 * intelliparadigm.com page, section 2.1 (router snippet): softmax over all
   experts, then top-K on the probabilities.
 
-Readings where the pages are silent (each listed in the design notes):
+Readings where the pages are silent, taken here:
 
 * group size 64 along the input (reduction) dimension, one (scale, bias) pair
   per group and row; codes low-bits-first inside little-endian uint32 words;

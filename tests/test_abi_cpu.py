@@ -131,3 +131,14 @@ def test_missing_library_raises(lib, monkeypatch, tmp_path):
         lib.lib()
     with pytest.raises(RuntimeError):
         lib.fmoe_record_bytes(4096, 1024, 4)
+
+
+def test_build_keeps_subnormals():
+    """The library is built with -ftz=false and refuses flags that flush subnormals
+    (the single-token dot products read codes as subnormal floats)."""
+    from bit_dequant_expert_softmax_b200 import build as b
+    assert "-ftz=false" in b.NVCC_FLAGS
+    b.check_flags(b.NVCC_FLAGS)
+    for bad in ("--use_fast_math", "-ftz=true"):
+        with pytest.raises(ValueError):
+            b.check_flags(b.NVCC_FLAGS + [bad])

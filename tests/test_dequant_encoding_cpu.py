@@ -1,13 +1,17 @@
 """IEEE identities the dequantising dot products rely on (CPU, numpy float32).
 
 The single-token kernel reads a code masked in place at bit offset s of a 32-bit word
-as a float32 and multiplies it by an activation stored pre-scaled by 2^(100 - s).
-These tests check, for every code and every position of 4- and 2-bit words:
+as a float32 and multiplies it by an activation stored pre-scaled by 2^(P - s), where
+the exponent P = 100 - e is chosen per chunk of activations from the largest exponent
+e of the chunk (e clamped to [-26, 78]).  These tests check, for every code and every
+position of 4- and 2-bit words:
   - the masked bit pattern read as float32 is exactly code * 2^(s - 149) (a subnormal,
     or the first normal binade when bit 23 is set);
-  - the pre-scale factor 2^(100 - s) is a plain power of two built from its exponent;
-  - code * (x * 2^(100 - s)) equals code * x * 2^-49 exactly for bf16 activations, so
-    the per-chunk sum needs one rescale by 2^49;
+  - the pre-scale factor 2^(P - s) and the rescale 2^(149 - P) are plain powers of two
+    built from their exponents, for every exponent the clamp admits;
+  - code * (x * 2^(P - s)) equals code * x * 2^(P - 149) exactly, for activations from
+    2^-100 to 2^100 in magnitude (bf16 x, and fp32 h), so the per-chunk sum needs one
+    rescale by 2^(149 - P);
   - the positions whose code would cross bit 24 are read from the word shifted right by
     8 without picking up bits of the neighbouring word.
 """
@@ -17,6 +21,14 @@ import pytest
 import oracle
 
 PRE_EXP = 100
+MIN_EXP, MAX_EXP = -26, 78
+
+
+def chunk_pre(max_abs):
+    """The kernel's pre-scale exponent for a chunk whose largest |activation| is max_abs."""
+    bits = int(np.array([max_abs], dtype=np.float32).view(np.uint32)[0]) & 0x7FFFFFFF
+    e = (bits >> 23) - 127
+    return PRE_EXP - min(max(e, MIN_EXP), MAX_EXP)
 
 
 def shift_pos(bits, p):
@@ -40,23 +52,59 @@ def test_masked_code_reads_as_scaled_subnormal(bits):
 
 
 @pytest.mark.parametrize("bits", [4, 2])
-def test_prescale_factor_is_the_power_of_two(bits):
-    for p in range(32 // bits):
-        s = shift_pos(bits, p)
-        assert float(as_f32((127 + PRE_EXP - s) << 23)) == 2.0 ** (PRE_EXP - s)
+def test_prescale_and_rescale_are_powers_of_two(bits):
+    for e in range(MIN_EXP, MAX_EXP + 1):
+        pre = PRE_EXP - e
+        assert float(as_f32((127 + 149 - pre) << 23)) == 2.0 ** (149 - pre)
+        for p in range(32 // bits):
+            s = shift_pos(bits, p)
+            assert 1 <= 127 + pre - s <= 254
+            assert float(as_f32((127 + pre - s) << 23)) == 2.0 ** (pre - s)
 
 
 @pytest.mark.parametrize("bits", [4, 2])
-def test_products_with_prescaled_bf16_activations_are_exact(bits):
+@pytest.mark.parametrize("magnitude", [1e-20, 2.0 ** -30, 1.0, 2.0 ** 20, 2.0 ** 46, 2.0 ** 64])
+def test_products_with_prescaled_activations_are_exact(bits, magnitude):
+    """A chunk of bf16 activations spread over about +-13 binades around `magnitude`
+    (and an fp32 chunk of the same spread, as h is), its largest exponent inside the
+    clamp: pre-scaled values are finite and exact; every product with a masked code is
+    exact for bf16 activations and the correctly rounded fp32 product (no underflow)
+    for fp32 ones."""
     rng = np.random.default_rng(0)
-    x = oracle.bf16_to_f64(oracle.f64_to_bf16_bits(rng.standard_normal(256) * np.exp(rng.standard_normal(256) * 3)))
-    for p in range(32 // bits):
-        s = shift_pos(bits, p)
-        xs = (x * 2.0 ** (PRE_EXP - s)).astype(np.float32)
-        assert np.array_equal(xs.astype(np.float64), x * 2.0 ** (PRE_EXP - s))  # scaling is exact
-        for c in range(1 << bits):
-            prod = (as_f32(c << s) * xs).astype(np.float64)   # float32 multiply
-            assert np.array_equal(prod, c * x * 2.0 ** (PRE_EXP - 149)), (bits, p, c)
+    z = rng.standard_normal(64) * np.exp(rng.standard_normal(64) * 3)
+    for exact, x in ((True, oracle.bf16_to_f64(oracle.f64_to_bf16_bits(z * magnitude))),
+                     (False, (z * magnitude).astype(np.float32).astype(np.float64))):
+        pre = chunk_pre(np.max(np.abs(x)))
+        for p in range(32 // bits):
+            s = shift_pos(bits, p)
+            xs = (x * 2.0 ** (pre - s)).astype(np.float32)
+            assert np.all(np.isfinite(xs))
+            assert np.array_equal(xs.astype(np.float64), x * 2.0 ** (pre - s))  # scaling is exact
+            for c in range(1 << bits):
+                prod = (as_f32(c << s) * xs).astype(np.float64)   # float32 multiply
+                want = c * x * 2.0 ** (pre - 149)
+                if not exact:
+                    want = want.astype(np.float32).astype(np.float64)
+                assert np.array_equal(prod, want), (bits, p, c)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_prescaled_values_stay_finite_outside_the_clamp(bits):
+    """Chunks whose largest exponent lies outside the clamp: up to |x| < 2^105 the
+    pre-scaled values are finite, and products of the chunk's largest entries are
+    still exact; tiny chunks (down to 2^-100) never overflow either."""
+    for mx in (2.0 ** 79, 2.0 ** 90, 2.0 ** 104.9, 2.0 ** -27, 2.0 ** -60, 2.0 ** -100):
+        x = np.array([mx, mx / 3.0, -mx / 7.0, mx / 1024.0])
+        x = oracle.bf16_to_f64(oracle.f64_to_bf16_bits(x))
+        pre = chunk_pre(np.max(np.abs(x)))
+        for p in range(32 // bits):
+            s = shift_pos(bits, p)
+            xs = (x * 2.0 ** (pre - s)).astype(np.float32)
+            assert np.all(np.isfinite(xs)), (mx, p)
+            c = (1 << bits) - 1
+            prod = (as_f32(c << s) * xs[:1]).astype(np.float64)
+            if mx >= 2.0 ** -50:
+                assert np.array_equal(prod, c * x[:1] * 2.0 ** (pre - 149)), (mx, p)
 
 
 @pytest.mark.parametrize("bits", [4, 2])

@@ -10,6 +10,9 @@ ulp check covers outputs with |oracle| >= rms/16, where the bf16 ulp exceeds the
 fp32 sum's absolute rounding error.
 """
 import math
+import multiprocessing
+import os
+from concurrent.futures import ProcessPoolExecutor
 
 import numpy as np
 import pytest
@@ -17,6 +20,7 @@ import torch
 
 import fmoe_synth as synth
 import oracle
+from _stack_oracle import layer_tokens, shape_fields
 from _ties import index_mismatch
 
 pytestmark = pytest.mark.gpu
@@ -40,25 +44,34 @@ def _bf(t):
     return oracle.bf16_to_f64(t.view(torch.int16).cpu().numpy().view(np.uint16))
 
 
+def _check_token(t, ref, xs, ys, idx, w, sig, has_shared, ctx=""):
+    """One token's GPU routing and output against the oracle's (idx, w, sigma, y,
+    logits); returns the worst error/bound ratio."""
+    r_idx, r_w, r_sigma, r_y, r_logits = ref
+    assert list(idx[t]) == list(r_idx), index_mismatch(f"{ctx} token {t}", idx[t], r_idx, r_logits)
+    assert np.allclose(w[t], r_w, rtol=1e-6, atol=1e-7), f"{ctx} token {t}: w"
+    if has_shared and sig is not None:
+        assert math.isclose(float(sig[t]), r_sigma, rel_tol=1e-6), f"{ctx} token {t}: sigma"
+    ok, ratio = oracle.within_tolerance(ys[t], r_y)
+    assert ok, f"{ctx} token {t}: worst error/bound {ratio:.3f}"
+    same, ulps = oracle.bf16_agreement(ys[t], r_y, min_rel_rms=1.0 / 16)
+    n_diff = round((1.0 - same) * ys.shape[1])
+    assert n_diff <= max(2, 0.01 * ys.shape[1]) and ulps <= 1.0, \
+        f"{ctx} token {t}: {n_diff} outputs differ from the rounded oracle, max {ulps} ulps"
+    return ratio
+
+
 def _check_tokens(olay, xg, yg, idxg, wg, sigg, tokens, ctx=""):
     xs = _bf(xg)
     ys = _bf(yg)
     idx = idxg.cpu().numpy()
     w = wg.cpu().numpy()
+    sig = None if sigg is None else sigg.cpu().numpy()
     worst = 0.0
     for t in tokens:
         r = olay.forward(xs[t])
-        assert list(idx[t]) == list(r.idx), index_mismatch(f"{ctx} token {t}", idx[t], r.idx, r.logits)
-        assert np.allclose(w[t], r.w, rtol=1e-6, atol=1e-7), f"{ctx} token {t}: w"
-        if olay.has_shared and sigg is not None:
-            assert math.isclose(float(sigg.cpu()[t]), r.sigma, rel_tol=1e-6), f"{ctx} token {t}: sigma"
-        ok, ratio = oracle.within_tolerance(ys[t], r.y)
-        worst = max(worst, ratio)
-        assert ok, f"{ctx} token {t}: worst error/bound {ratio:.3f}"
-        same, ulps = oracle.bf16_agreement(ys[t], r.y, min_rel_rms=1.0 / 16)
-        n_diff = round((1.0 - same) * ys.shape[1])
-        assert n_diff <= max(2, 0.01 * ys.shape[1]) and ulps <= 1.0, \
-            f"{ctx} token {t}: {n_diff} outputs differ from the rounded oracle, max {ulps} ulps"
+        ref = (r.idx, r.w, r.sigma, r.y, r.logits)
+        worst = max(worst, _check_token(t, ref, xs, ys, idx, w, sig, olay.has_shared, ctx))
     return worst
 
 
@@ -158,10 +171,11 @@ def test_deterministic_and_graph_replay(cuda_lib):
     assert L.error() == 0
 
 
-def test_full_size_layer_sampled_tokens(cuda_lib):
+def test_full_size_layer_64_tokens(cuda_lib):
     """hidden 4096, intermediate 1024, 512 experts + shared, top-4, 4-bit (the
-    full-size decode layer), single-token calls as the benchmark times them;
-    sampled tokens against the oracle."""
+    full-size decode layer), single-token calls as the benchmark times them; all 64
+    tokens (the first and the last among them) against the oracle, which runs in a
+    spawned process pool."""
     shape = synth.CONFIGS["layer4096"]["shape"]
     _, L = _mk(cuda_lib, shape, seed=0)
     T = 64
@@ -172,10 +186,58 @@ def test_full_size_layer_sampled_tokens(cuda_lib):
     idx, w, sig = L.route(x)
     torch.cuda.synchronize()
     assert L.error() == 0
-    olay = oracle.synthetic_layer(0, 0, shape, lazy=True)
-    tokens = [0, 1, 31, 62, 63]
-    worst = _check_tokens(olay, x, y, idx, w, sig, tokens, "layer4096")
-    print(f"layer4096 worst error/bound {worst:.3f}")
+    L.close()
+    xb = x.view(torch.int16).cpu().numpy().view(np.uint16)
+    workers = max(1, min(16, os.cpu_count() or 1))
+    jobs = [(0, 0, shape_fields(shape), [xb[t] for t in range(T) if t % workers == j]) for j in range(workers)]
+    with ProcessPoolExecutor(max_workers=workers, mp_context=multiprocessing.get_context("spawn")) as ex:
+        parts = list(ex.map(layer_tokens, jobs))
+    refs = {}
+    for j, part in enumerate(parts):
+        for t, ref in zip([t for t in range(T) if t % workers == j], part):
+            refs[t] = ref
+    xs, ys = _bf(x), _bf(y)
+    idx, w, sig = idx.cpu().numpy(), w.cpu().numpy(), sig.cpu().numpy()
+    worst = 0.0
+    for t in range(T):
+        worst = max(worst, _check_token(t, refs[t], xs, ys, idx, w, sig, True, "layer4096"))
+    print(f"layer4096 worst error/bound over {T} tokens {worst:.3f}")
+
+
+@pytest.mark.parametrize("scale,zero_resid", [(2.0 ** 20, False), (1e-20, False), (2.0 ** -40, True),
+                                              (1e-10, True)])
+@pytest.mark.parametrize("name", ["tiny", "tiny_2bit"])
+def test_activation_magnitudes(cuda_lib, name, scale, zero_resid):
+    """Activations far from unit size: x scaled by 2^20 (the hidden h reaches about
+    2^46), by 1e-20, and by 2^-40 and 1e-10 with a zero residual (so that y is the MoE
+    output alone, of the order of scale^2).  The dequantising dot products pick their
+    power-of-two pre-scale per chunk of activations, so the single-token and the
+    batched path both stay within the tolerance of the oracle."""
+    shape = SHAPES[name]
+    T = 8
+    _, L = _mk(cuda_lib, shape, seed=14)
+    x = (_x(14, 0, T, shape.hidden).float() * scale).to(torch.bfloat16)
+    resid = torch.zeros_like(x) if zero_resid else x
+    y = torch.empty_like(x)
+    for t in range(T):
+        cuda_lib.fmoe_layer_forward(L.handle, x[t:t + 1], resid[t:t + 1], 1, y[t:t + 1])
+    idx, w, sig = L.route(x)
+    L.attach_batch(T)
+    yb = L.forward_batched(x, resid=resid)
+    torch.cuda.synchronize()
+    assert L.error() == 0
+    olay = oracle.synthetic_layer(14, 0, shape, lazy=True)
+    xs, rs, ys, ybs = _bf(x), _bf(resid), _bf(y), _bf(yb)
+    idx, w = idx.cpu().numpy(), w.cpu().numpy()
+    for t in range(T):
+        r = olay.forward(xs[t], rs[t])
+        assert list(idx[t]) == list(r.idx), index_mismatch(f"{name} x*{scale:g} token {t}", idx[t], r.idx, r.logits)
+        assert np.allclose(w[t], r.w, rtol=1e-6, atol=1e-7)
+        if zero_resid:  # y is the MoE output alone: nonzero, of the order of scale^2
+            assert 0.0 < np.max(np.abs(r.y)) < 1e4 * scale * scale
+        for label, got in (("single-token", ys[t]), ("batched", ybs[t])):
+            ok, worst = oracle.within_tolerance(got, r.y)
+            assert ok, f"{label} {name} x*{scale:g} token {t}: worst error/bound {worst:.3f}"
 
 
 def test_rmsnorm_matches_oracle(cuda_lib):

@@ -113,6 +113,16 @@ def _regions_down_swapped(H, I, bits):
     return R
 
 
+def _regions_offsets_from_4bit_rows(H, I, bits):
+    """Region offsets laid out as if the rows had 4-bit width (the row sizes stay
+    right); identical to the true layout for 4-bit records."""
+    R = dict(ORIG["record_regions"](H, I, bits))
+    R4 = ORIG["record_regions"](H, I, 4)
+    for k in ("gu_q", "gu_sb", "d_q", "d_sb"):
+        R[k] = R4[k]
+    return R
+
+
 def _bf16_truncate(v):
     f = np.asarray(v, dtype=np.float64).astype(np.float32)
     return (f.view(np.uint32) >> 16).astype(np.uint16)
@@ -131,6 +141,7 @@ MUTATIONS = {
     "gate and up rows swapped": {"decode_record": lambda rec, H, I, bits: (
         lambda ex: fo.DenseExpert(ex.Wu, ex.Wg, ex.Wd))(ORIG["decode_record"](rec, H, I, bits))},
     "down regions swapped": {"record_regions": _regions_down_swapped},
+    "2-bit region offsets computed with 4-bit row bytes": {"record_regions": _regions_offsets_from_4bit_rows},
     # SwiGLU / down
     "silu applied to up": {"expert_ffn": lambda ex, x: ex.Wd @ (
         (ex.Wg @ np.asarray(x, np.float64)) * fo.silu(ex.Wu @ np.asarray(x, np.float64)))},

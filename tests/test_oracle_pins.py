@@ -273,19 +273,21 @@ def test_power_of_two_down_scaling_is_exact():
 # ------------------------------------------------------------ whole layer ----
 def _brute_force_layer(lay, x):
     """Independent naive path: every expert dense (codes read by integer
-    division), full softmax, mask to the top K, renormalise, sum over all E."""
-    H, I, E, K = lay.H, lay.I, lay.E, lay.K
-    rb = oracle.record_regions(H, I, 4)["size"]
+    division from the generator's plain words, not from the packed record), full
+    softmax, mask to the top K, renormalise, sum over all E."""
+    H, I, E, K, bits = lay.H, lay.I, lay.E, lay.K, lay.bits
+    per = 32 // bits          # codes per word
+    base = 2 ** bits          # code c of a word is digit c in base 2^bits
 
     def dense(e):
-        p = synth.gen_expert(3, 0, e, H, I, 4)
+        p = synth.gen_expert(3, 0, e, H, I, bits)
 
         def deq(words, sbs, rows, cols):
             W = np.zeros((rows, cols))
             for r in range(rows):
                 for c in range(cols):
-                    wd = int(words[r, c // 8])
-                    q = (wd // (16 ** (c % 8))) % 16
+                    wd = int(words[r, c // per])
+                    q = (wd // (base ** (c % per))) % base
                     pair = int(sbs[r, c // 64])
                     s = synth.bf16_to_f64(np.array([pair % 65536], dtype=np.uint16))[0]
                     b = synth.bf16_to_f64(np.array([pair // 65536], dtype=np.uint16))[0]
@@ -314,8 +316,11 @@ def _brute_force_layer(lay, x):
 
 
 @pytest.mark.slow
-def test_whole_layer_matches_brute_force():
-    lay, sh = _tiny_layer(H=64, I=64, E=6, K=2)
+@pytest.mark.parametrize("bits", [4, 2])
+def test_whole_layer_matches_brute_force(bits):
+    """The whole layer against the naive path, for 4-bit and 2-bit records (the 2-bit
+    case pins the 2-bit region offsets and code order of the packed format)."""
+    lay, sh = _tiny_layer(H=64, I=64, E=6, K=2, bits=bits)
     for t in range(2):
         x = oracle.bf16_to_f64(synth.gen_x_token(20, t, sh.hidden))
         r = lay.forward(x)

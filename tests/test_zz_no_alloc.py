@@ -58,17 +58,21 @@ def test_noalloc_forward_matches_workspace_forward(cuda_lib, name):
 
 
 def test_noalloc_rejects_layers_beyond_the_scratch_size(cuda_lib):
+    """A layer whose workspace exceeds the fixed array is refused before anything is
+    enqueued.  The weight buffers have the sizes the config implies (zeros), so that
+    even a launch that should not have happened would read only memory it owns."""
     fm = cuda_lib
-    # hidden 4096, intermediate 1024, 512 experts, top-10: workspace above 128 KiB.
-    # Rejected on the host before anything is enqueued, so small stand-in buffers do.
-    cfg = fm.fmoe_config(4096, 1024, 512, 10, 4, 1, 0)
+    # hidden 64, intermediate 8192, 2 experts + shared, top-1: its h buffers alone take
+    # 2 x 2 x 8192 x 4 bytes, more than the 128 KiB array
+    H, I, E = 64, 8192, 2
+    cfg = fm.fmoe_config(H, I, E, 1, 4, 1, 0)
     assert fm.fmoe_workspace_bytes(cfg) > fm.NOALLOC_SCRATCH_BYTES
-    experts = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
-    router = torch.zeros(1024, dtype=torch.float32, device="cuda")
-    gs = torch.zeros(4096, dtype=torch.float32, device="cuda")
+    experts = torch.zeros(fm.fmoe_record_bytes(H, I, 4) * (E + 1), dtype=torch.uint8, device="cuda")
+    router = torch.zeros(E, H, dtype=torch.float32, device="cuda")
+    gs = torch.zeros(H, dtype=torch.float32, device="cuda")
     h = fm.fmoe_layer_create(cfg, experts, router, None, gs)
     try:
-        x = torch.zeros(1, 4096, dtype=torch.bfloat16, device="cuda")
+        x = torch.ones(1, H, dtype=torch.bfloat16, device="cuda")
         y = torch.zeros_like(x)
         with pytest.raises(fm.FmoeError) as e:
             fm.fmoe_layer_forward_noalloc(h, x, x, 1, y)
@@ -77,3 +81,36 @@ def test_noalloc_rejects_layers_beyond_the_scratch_size(cuda_lib):
         assert int(y.view(torch.int16).abs().sum()) == 0
     finally:
         fm.fmoe_layer_destroy(h)
+
+
+def test_noalloc_reports_device_errors(cuda_lib):
+    """A device-side error of a no-allocation call (a bounded wait that runs out: one
+    block is held back by the test hook, the others give up after 50 ms) is reported by
+    fmoe_layer_get_error on the layer, which has no workspace, and cleared; the next
+    call is correct again."""
+    from fmoe_synth.torch_layer import make_device_layer, make_device_x
+    fm = cuda_lib
+    shape = synth.CONFIGS["tiny"]["shape"]
+    w = make_device_layer(shape, 0, 0)
+    cfg = fm.fmoe_config(shape.hidden, shape.inter, shape.n_experts, shape.top_k, shape.bits,
+                         shape.has_shared, shape.router_bias)
+    ref_layer = fm.Layer.create(cfg, w.experts, w.router, w.router_bias, w.shared_gate)
+    bare = fm.fmoe_layer_create(cfg, w.experts, w.router, w.router_bias, w.shared_gate)
+    try:
+        x = make_device_x(4, 0, 1, shape.hidden)
+        y_ref = ref_layer.forward(x)
+        fm.fmoe_layer_set_wait_limit(bare, 50_000_000)
+        fm.fmoe_layer_debug_hold_block(bare, 1)
+        y = torch.zeros_like(x)
+        fm.fmoe_layer_forward_noalloc(bare, x, x, 1, y)
+        torch.cuda.synchronize()
+        assert fm.fmoe_layer_get_error(bare) & fm.DEVERR_BARRIER_TIMEOUT
+        assert fm.fmoe_layer_get_error(bare) == 0  # cleared
+        fm.fmoe_layer_debug_hold_block(bare, -1)
+        fm.fmoe_layer_forward_noalloc(bare, x, x, 1, y)
+        torch.cuda.synchronize()
+        assert fm.fmoe_layer_get_error(bare) == 0
+        assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+    finally:
+        fm.fmoe_layer_destroy(bare)
+        ref_layer.close()
