@@ -179,9 +179,16 @@ def topk_renorm(l: np.ndarray, K: int):
     lower index), then the K probabilities renormalised to sum to one
     (intelliparadigm.com, section 2.1: softmax, then top-K on the probabilities;
     tinai-dev README, "Pipeline mỗi lớp": softmax + top-K routing).  The
-    renormalisation and the tie rule are readings."""
+    renormalisation and the tie rule are readings.
+
+    The softmax is strictly increasing in the logit, so the K largest
+    probabilities belong to the K largest logits, and two probabilities are equal
+    exactly when their logits are.  The order is taken on the logits: in fp64 the
+    probabilities of logits more than ~745 below the largest underflow to 0.0 and
+    would tie, which the exact probabilities never do."""
+    l = np.asarray(l, dtype=np.float64)
     p = softmax(l)
-    order = sorted(range(len(p)), key=lambda e: (-p[e], e))
+    order = sorted(range(len(l)), key=lambda e: (-l[e], e))
     idx = np.array(order[:K], dtype=np.int64)
     w = p[idx] / np.sum(p[idx])
     return idx, w

@@ -154,6 +154,7 @@ MUTATIONS = {
         weights=lambda p, idx, l: l[idx] / np.sum(l[idx]))},
     "ties to the higher index": {"topk_renorm": _topk_with(key=lambda p: (lambda e: (-p[e], -e)))},
     "smallest K selected": {"topk_renorm": _topk_with(key=lambda p: (lambda e: (p[e], e)))},
+    "ranked on fp64 probabilities (underflowed ones tie)": {"topk_renorm": _topk_with()},
     "router bias subtracted": {"router_logits": lambda x, Wr, bias=None: ORIG["router_logits"](
         x, Wr, None if bias is None else -np.asarray(bias))},
     "shared gate sign flipped": {"shared_sigma": lambda gs, x: 1.0 - ORIG["shared_sigma"](gs, x)},

@@ -153,6 +153,21 @@ def test_router_dominant_and_ties():
     assert list(idx) == [1, 2] and w[0] == w[1] == 0.5
 
 
+def test_router_order_follows_exact_probabilities_beyond_underflow():
+    """Logits hundreds apart: fp64 probabilities of all but the largest underflow to
+    0.0, yet the exact probabilities stay strictly ordered.  The selection must be
+    the order of the log-probabilities (scipy's log_softmax, which does not
+    underflow), ties to the lower index; the weights are the fp64 ones (1, 0, ...)."""
+    l = np.array([-3000.0, 0.0, -900.0, -2000.0, -900.0, -5000.0, -1200.0])
+    lp = scipy.special.log_softmax(l)
+    want = sorted(range(len(l)), key=lambda e: (-lp[e], e))
+    for K in (1, 3, 4, 7):
+        idx, w = oracle.topk_renorm(l, K)
+        assert list(idx) == want[:K]
+        assert w[0] == 1.0 and np.all(w[1:] == 0.0)
+    assert want[:4] == [1, 2, 4, 6]
+
+
 def test_router_topk_is_best_subset_by_brute_force():
     rng = np.random.default_rng(11)
     E = 8
