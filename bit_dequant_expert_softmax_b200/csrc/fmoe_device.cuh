@@ -243,36 +243,30 @@ struct Chunk {
     }
   }
 
-  // Word pairs of one or two rows against shared activation pairs.
-  template <bool TWO>
-  __device__ __forceinline__ static void word_pair2(unsigned long long Wa, unsigned long long Wb,
-                                                    const ulonglong2* xv, unsigned long long& acc_a,
-                                                    unsigned long long& acc_b) {
-    const unsigned long long Va = Wa >> 8;
-    const unsigned long long Vb = TWO ? (Wb >> 8) : 0ull;
+  // Word pairs of NR rows against the same activation pairs: float4 k of the chunk
+  // (xv[k * 32]) holds the activations of positions 2k and 2k+1 of both words; every
+  // row's accumulator takes the positions in the same order.
+  template <int K, int NR>
+  __device__ __forceinline__ static void steps(const unsigned long long (&W)[NR], const unsigned long long (&V)[NR],
+                                               const ulonglong2* xv, unsigned long long (&acc)[NR]) {
+    if constexpr (K < kF4PerPair) {
+      const ulonglong2 x = xv[K * 32];
 #pragma unroll
-    for (int k = 0; k < kF4PerPair; ++k) {
-      const ulonglong2 x = xv[k * 32];
-      // positions 2k (x.x) and 2k+1 (x.y)
-      switch (k) {
-#define FMOE_POS_CASE(K)                                  \
-  case K:                                                 \
-    pos<2 * K>(Wa, Va, x.x, acc_a);                       \
-    pos<2 * K + 1>(Wa, Va, x.y, acc_a);                   \
-    if (TWO) pos<2 * K>(Wb, Vb, x.x, acc_b);              \
-    if (TWO) pos<2 * K + 1>(Wb, Vb, x.y, acc_b);          \
-    break;
-        FMOE_POS_CASE(0)
-        FMOE_POS_CASE(1)
-        FMOE_POS_CASE(2)
-        FMOE_POS_CASE(3)
-        FMOE_POS_CASE(4)
-        FMOE_POS_CASE(5)
-        FMOE_POS_CASE(6)
-        FMOE_POS_CASE(7)
-#undef FMOE_POS_CASE
+      for (int r = 0; r < NR; ++r) {
+        pos<2 * K>(W[r], V[r], x.x, acc[r]);
+        pos<2 * K + 1>(W[r], V[r], x.y, acc[r]);
       }
+      steps<K + 1, NR>(W, V, xv, acc);
     }
+  }
+
+  template <int NR>
+  __device__ __forceinline__ static void word_pairs(const unsigned long long (&W)[NR], const ulonglong2* xv,
+                                                    unsigned long long (&acc)[NR]) {
+    unsigned long long V[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) V[r] = W[r] >> 8;
+    steps<0, NR>(W, V, xv, acc);
   }
 };
 

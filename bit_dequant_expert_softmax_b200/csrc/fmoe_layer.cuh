@@ -73,7 +73,7 @@ struct Params {
   uint32_t* tokens;  // tokens this workspace has seen (tag base)
   uint32_t* rflags;  // [kMaxGrid * kFlagStride] per-block "router partials written" tags
   uint32_t* hflags;  // [kMaxGrid * kFlagStride] per-block "h rows written" tags
-  double* lpart;     // [2][(E+1)*nq] router partials
+  double* logits;    // [2][E+1] router logits (the shared gate's dot product last)
   float* hbuf;       // [2][(K+1)*I]  h values
   int norm;         // 1: the input is a pre-norm block's h (the NORM kernel variant)
   double norm_eps;
@@ -393,31 +393,32 @@ struct LayerKernel {
   __device__ __forceinline__ static int phys(int c) { return C::phys(c); }
 
   // ---------------------------------------------------------------- dot products
-  // Lane partial of sum_c W[r][c] v[c] over the lane's chunks, for one or two rows
-  // sharing the activation loads (W = scale*code + bias; v pre-scaled, interleaved).
-  template <bool TWO>
-  __device__ __forceinline__ void dotn(const uint8_t* q0, const uint32_t* s0, const uint8_t* q1,
-                                       const uint32_t* s1, const float* vs, const float2* vsum, int nch, float& r0,
-                                       float& r1) const {
+  // Lane partials of sum_c W[r][c] v[c] over the lane's chunks for NR rows sharing the
+  // activation loads (W = scale*code + bias; v pre-scaled, interleaved).  Every row is
+  // summed in the same order whatever NR is.
+  template <int NR>
+  __device__ __forceinline__ void dotr(const uint8_t* const (&q)[NR], const uint32_t* const (&sb)[NR],
+                                       const float* vs, const float2* vsum, int nch, float (&res)[NR]) const {
     const int lane = threadIdx.x & 31;
-#pragma unroll 2
+#pragma unroll(NR <= 2 ? 2 : 1)
     for (int m = lane; m < nch; m += 32) {
-      const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(q0 + 16 * m);
-      ulonglong2 b = make_ulonglong2(0ull, 0ull);
-      if (TWO) b = *reinterpret_cast<const ulonglong2*>(q1 + 16 * m);
-      const ulonglong2* xv0 = C::f4(vs, m, 0);
-      const ulonglong2* xv1 = C::f4(vs, m, C::kF4PerPair);
-      unsigned long long a0 = 0ull, a1 = 0ull, b0 = 0ull, b1 = 0ull;
-      C::template word_pair2<TWO>(a.x, b.x, xv0, a0, b0);
-      C::template word_pair2<TWO>(a.y, b.y, xv1, a1, b1);
+      unsigned long long wx[NR], wy[NR], a0[NR], a1[NR];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        const ulonglong2 w = *reinterpret_cast<const ulonglong2*>(q[r] + 16 * m);
+        wx[r] = w.x;
+        wy[r] = w.y;
+        a0[r] = 0ull;
+        a1[r] = 0ull;
+      }
+      C::template word_pairs<NR>(wx, C::f4(vs, m, 0), a0);
+      C::template word_pairs<NR>(wy, C::f4(vs, m, C::kF4PerPair), a1);
       const float2 vm = vsum[m];  // (sum of the chunk's activations, rescale of its products)
-      const uint32_t sa = s0[C::sb_index(m)];
-      r0 = fmaf(sb_scale(sa), (pair_sum(a0) + pair_sum(a1)) * vm.y, r0);
-      r0 = fmaf(sb_bias(sa), vm.x, r0);
-      if (TWO) {
-        const uint32_t sbv = s1[C::sb_index(m)];
-        r1 = fmaf(sb_scale(sbv), (pair_sum(b0) + pair_sum(b1)) * vm.y, r1);
-        r1 = fmaf(sb_bias(sbv), vm.x, r1);
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        const uint32_t sbv = sb[r][C::sb_index(m)];
+        res[r] = fmaf(sb_scale(sbv), (pair_sum(a0[r]) + pair_sum(a1[r])) * vm.y, res[r]);
+        res[r] = fmaf(sb_bias(sbv), vm.x, res[r]);
       }
     }
   }
@@ -460,47 +461,61 @@ struct LayerKernel {
     }
   }
 
-  // h of row pair r of the chunk -> hbuf[buf][slot][r]  (one warp)
-  __device__ bool gu_unit(const GuChunk& c, int r, int buf) {
+  // h of row pairs r .. r+np-1 (np = 1 or 2) of the chunk -> hbuf[buf][slot][r ..]  (one
+  // warp); two row pairs are four rows sharing the activation loads.
+  __device__ bool gu_unit(const GuChunk& c, int r, int np, int buf) {
     const int n = c.rb - c.ra, i = r - c.ra;
     if (!wait_item(c.first + i / p.rp)) return false;
+    if ((i + np - 1) / p.rp != i / p.rp && !wait_item(c.first + (i + np - 1) / p.rp)) return false;
     if (i >= p.rp && !wait_item(c.first)) return false;  // (scale,bias) rows ride on item 0
     const uint8_t* qg = stage + c.off + static_cast<uint32_t>(i) * 2u * p.qh;
-    const uint8_t* qu = qg + p.qh;
     const uint32_t lead =
         static_cast<uint32_t>((p.o_gu_sb + static_cast<unsigned long long>(c.ra) * 2u * p.sh) & 15ull);
     const uint32_t* sg = reinterpret_cast<const uint32_t*>(stage + c.off + g.gu_q(n) + lead) + i * 2 * (p.sh / 4);
-    const uint32_t* su = sg + p.sh / 4;
-    float gv = 0.f, uv = 0.f;
-    dotn<true>(qg, sg, qu, su, xs, xsum, p.H / C::kCols, gv, uv);
-    gv = warp_sum(gv);
-    uv = warp_sum(uv);
-    if ((threadIdx.x & 31) == 0) {
-      const float hval = (gv / (1.0f + expf(-gv))) * uv;
-      p.hbuf[static_cast<size_t>(buf) * (p.K + 1) * p.I + static_cast<size_t>(c.slot) * p.I + r] = hval;
+    const int sw = p.sh / 4;
+    float* hout = p.hbuf + static_cast<size_t>(buf) * (p.K + 1) * p.I + static_cast<size_t>(c.slot) * p.I + r;
+    if (np == 2) {
+      const uint8_t* const q[4] = {qg, qg + p.qh, qg + 2 * p.qh, qg + 3 * p.qh};
+      const uint32_t* const sb[4] = {sg, sg + sw, sg + 2 * sw, sg + 3 * sw};
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      dotr<4>(q, sb, xs, xsum, p.H / C::kCols, v);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) v[k] = warp_sum(v[k]);
+      if ((threadIdx.x & 31) == 0) {
+        hout[0] = (v[0] / (1.0f + expf(-v[0]))) * v[1];
+        hout[1] = (v[2] / (1.0f + expf(-v[2]))) * v[3];
+      }
+    } else {
+      const uint8_t* const q[2] = {qg, qg + p.qh};
+      const uint32_t* const sb[2] = {sg, sg + sw};
+      float v[2] = {0.f, 0.f};
+      dotr<2>(q, sb, xs, xsum, p.H / C::kCols, v);
+      v[0] = warp_sum(v[0]);
+      v[1] = warp_sum(v[1]);
+      if ((threadIdx.x & 31) == 0) hout[0] = (v[0] / (1.0f + expf(-v[0]))) * v[1];
     }
     return true;
   }
 
-  // Consume every row pair of `nc` chunks, spread over warps w0 .. kWarps-1 (unit u ->
-  // warp w0 + u % (kWarps - w0)); w0 = 1 keeps warp 0, which issues the copies and
-  // computes the routing weights meanwhile, out of the routed rows.
+  // Consume every row pair of `nc` chunks in units of two row pairs, spread over warps
+  // w0 .. kWarps-1 (unit u -> warp w0 + u % (kWarps - w0)); w0 = 1 keeps warp 0, which
+  // issues the copies and computes the routing weights meanwhile, out of the routed rows.
   __device__ void gu_consume(const GuChunk* ch, int nc, int buf, int w0 = 0) {
     const int warp = threadIdx.x >> 5;
     if (warp < w0) return;
     const int nw = kWarps - w0;
     int base = 0;
     for (int k = 0; k < nc; ++k) {
-      const int n = ch[k].rb - ch[k].ra;
+      const int n = ch[k].rb - ch[k].ra, nu = (n + 1) / 2;
       int first = (warp - w0 - base) % nw;
       if (first < 0) first += nw;
-      for (int i = first; i < n; i += nw) {
-        if (!gu_unit(ch[k], ch[k].ra + i, buf)) {
+      for (int u = first; u < nu; u += nw) {
+        if (!gu_unit(ch[k], ch[k].ra + 2 * u, min(2, n - 2 * u), buf)) {
           hdr->abort_flag = 1;
           return;
         }
       }
-      base += n;
+      base += nu;
     }
   }
 
@@ -583,71 +598,80 @@ struct LayerKernel {
     }
   }
 
-  // Consume a down item (rows [ja, ja+n)): y = resid + sum_s w_s o_s.
+  // Consume a down item (rows [ja, ja+n) of every slot): units (slot, group of up to
+  // four rows) are spread over the warps, four rows sharing each activation load; the
+  // rows' results o_s[j] are gathered in shared memory over the activations x (no
+  // longer read in this phase), then y = resid + sum_s w_s o_s[j], summed in slot order
+  // and rounded once.  Called by every thread; returns false for all on an abort.
   __device__ bool down_item(uint32_t item, uint32_t off, int ja, int n, const float* hs, const float2* hsum,
                             const uint16_t* resid_t, uint16_t* y_t) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ia = warp, ib = warp + kWarps;
-    if (ia >= n) return true;
-    if (!wait_item(item)) {
-      hdr->abort_flag = 1;
-      return false;
-    }
-    const bool two = ib < n;
+    const int ng = (n + 3) >> 2, nu = nslots * ng;
     const uint32_t lead = static_cast<uint32_t>((p.o_d_sb + static_cast<unsigned long long>(ja) * p.si) & 15ull);
-    const int nch = p.I / C::kCols;
-    float pa = 0.f, pb = 0.f;
-    for (int s = 0; s < nslots; ++s) {
+    const int nch = p.I / C::kCols, sw = p.si / 4;
+    float* ob = xs;  // [nslots][n]
+    bool ok = warp >= nu || wait_item(item);
+    if (!ok) hdr->abort_flag = 1;
+    for (int u = warp; ok && u < nu; u += kWarps) {
+      const int s = u / ng, j0 = (u % ng) * 4, nr = min(4, n - j0);
       const uint8_t* blk = stage + off + s * g.dn_slot(n);
-      const uint32_t* sbase = reinterpret_cast<const uint32_t*>(blk + g.dn_q(n) + lead);
-      float oa = 0.f, ob = 0.f;
+      const uint8_t* q0 = blk + static_cast<uint32_t>(j0) * p.qi;
+      const uint32_t* s0 = reinterpret_cast<const uint32_t*>(blk + g.dn_q(n) + lead) + j0 * sw;
       const float* hsl = hs + static_cast<size_t>(s) * g.padded(p.I);
       const float2* hsm = hsum + static_cast<size_t>(s) * nch;
-      if (two)
-        dotn<true>(blk + static_cast<uint32_t>(ia) * p.qi, sbase + ia * (p.si / 4),
-                   blk + static_cast<uint32_t>(ib) * p.qi, sbase + ib * (p.si / 4), hsl, hsm, nch, oa, ob);
-      else
-        dotn<false>(blk + static_cast<uint32_t>(ia) * p.qi, sbase + ia * (p.si / 4), nullptr, nullptr, hsl, hsm,
-                    nch, oa, ob);
-      const float ws = hdr->wsl[s];
-      pa = fmaf(ws, oa, pa);
-      pb = fmaf(ws, ob, pb);
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (nr > 2) {  // a group of three repeats its last row (the fourth result is dropped)
+        const int r3 = nr - 1;
+        const uint8_t* const q[4] = {q0, q0 + p.qi, q0 + 2 * p.qi, q0 + r3 * p.qi};
+        const uint32_t* const sb[4] = {s0, s0 + sw, s0 + 2 * sw, s0 + r3 * sw};
+        dotr<4>(q, sb, hsl, hsm, nch, v);
+      } else {
+        const int r1 = nr - 1;
+        const uint8_t* const q[2] = {q0, q0 + r1 * p.qi};
+        const uint32_t* const sb[2] = {s0, s0 + r1 * sw};
+        float v2[2] = {0.f, 0.f};
+        dotr<2>(q, sb, hsl, hsm, nch, v2);
+        v[0] = v2[0];
+        v[1] = v2[1];
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) v[k] = warp_sum(v[k]);
+      if (lane < nr) ob[s * n + j0 + lane] = lane == 0 ? v[0] : lane == 1 ? v[1] : lane == 2 ? v[2] : v[3];
     }
-    pa = warp_sum(pa);
-    pb = warp_sum(pb);
-    if (lane == 0) {
-      y_t[ja + ia] = f32_to_bf16(bf16_to_f32(resid_t[ja + ia]) + pa);
-      if (two) y_t[ja + ib] = f32_to_bf16(bf16_to_f32(resid_t[ja + ib]) + pb);
+    __syncthreads();
+    if (hdr->abort_flag) return false;
+    for (int j = threadIdx.x; j < n; j += kThreads) {
+      float pa = 0.f;
+      for (int s = 0; s < nslots; ++s) pa = fmaf(hdr->wsl[s], ob[s * n + j], pa);
+      y_t[ja + j] = f32_to_bf16(bf16_to_f32(resid_t[ja + j]) + pa);
     }
+    __syncthreads();
     return true;
   }
 
   // ---------------------------------------------------------------- P1
-  // Router units [u0, u1) over (E + has_shared) rows x nq splits (the shared gate
-  // vector is the last row) staged after the router's doubles; the block's slice of
-  // the shared expert's gate/up rows staged at the end of the staging area, to be
-  // consumed after top-K while the routed rows are in flight.  All copies are issued
-  // before the activations are staged (they do not depend on them).
-  int u0_, u1_, row0_, row1_;
-  uint32_t p1first_, rbase_;
+  // Router rows [row0, row1) of the (E + has_shared) rows (the shared gate vector is the
+  // last row), whole rows per block, staged after the router's doubles; the block's
+  // slice of the shared expert's gate/up rows staged at the end of the staging area, to
+  // be consumed while the router logits travel.  These are weights only: the copies are
+  // issued before the kernel waits for the previous grid, and before the activations.
+  int row0_, row1_;
+  uint32_t p1first_, rbase_, rpart_;
   GuChunk sc_;
   bool has_sc_;
 
   __device__ void phase1_issue(bool route, bool shared_gu) {
     const int rows = p.E + (p.has_shared ? 1 : 0);
     const int G = gridDim.x, b = blockIdx.x;
-    u0_ = u1_ = row0_ = row1_ = 0;
+    row0_ = row1_ = 0;
     if (route) {
-      const long long U = static_cast<long long>(rows) * p.nq;
-      u0_ = static_cast<int>(U * b / G);
-      u1_ = static_cast<int>(U * (b + 1) / G);
-      row0_ = u0_ / p.nq;
-      row1_ = (u1_ + p.nq - 1) / p.nq;
+      row0_ = static_cast<int>(static_cast<long long>(rows) * b / G);
+      row1_ = static_cast<int>(static_cast<long long>(rows) * (b + 1) / G);
     }
-    const int hc = p.H / p.nq;
     const uint32_t rib = g.router_item();
     rbase_ = route ? r128(static_cast<uint32_t>(p.H) * 8u) : 0u;
     const int nrouter = row1_ - row0_;
+    rpart_ = r128(rbase_ + static_cast<uint32_t>(nrouter) * rib);
     p1first_ = nitem;
     sc_ = GuChunk{p.K, 0, 0, 0, p1first_ + static_cast<uint32_t>(nrouter)};
     if (shared_gu) {
@@ -660,14 +684,10 @@ struct LayerKernel {
     if (threadIdx.x < 32) {
       fence_proxy_async_smem();
       for (int r = row0_ + static_cast<int>(threadIdx.x); r < row1_; r += 32) {
-        const int ua = max(u0_, r * p.nq), ub = min(u1_, r * p.nq + p.nq);
         uint64_t* bar = bar_of(p1first_ + (r - row0_));
-        const uint32_t bytes = static_cast<uint32_t>(ub - ua) * hc * 4u;
         const float* src = (r < p.E) ? p.router + static_cast<size_t>(r) * p.H : p.sgate;
-        src += static_cast<size_t>(ua - r * p.nq) * hc;
-        mbar_arrive_expect_tx(bar, bytes);
-        bulk_g2s(stage + rbase_ + (r - row0_) * rib + static_cast<uint32_t>(ua - r * p.nq) * hc * 4u, src, bytes,
-                 bar);
+        mbar_arrive_expect_tx(bar, rib);
+        bulk_g2s(stage + rbase_ + (r - row0_) * rib, src, rib, bar);
       }
       for (int i = static_cast<int>(threadIdx.x) - (nrouter % 32); i < nsh; i += 32)
         if (i >= 0) issue_gu_item(sc_, i);
@@ -675,7 +695,10 @@ struct LayerKernel {
     nitem += static_cast<uint32_t>(nrouter + nsh);
   }
 
-  // Router dot products of this block's units: fp64 sums of exact fp32 x bf16 products.
+  // Router logits of this block's rows: every (row, column split) unit is a warp's fp64
+  // sum of exact fp32 x bf16 products, lanes striding the split; the splits' sums are
+  // added in split order (the batched router's order too, so both give the same bits)
+  // and published for every block to read.
   __device__ bool phase1_consume(int buf, bool route) {
     if (route) {
       const int rows = p.E + (p.has_shared ? 1 : 0);
@@ -684,9 +707,10 @@ struct LayerKernel {
       const uint32_t rib = g.router_item();
       const double2* xa = reinterpret_cast<const double2*>(stage);
       const double2* xb = xa + p.H / 4;
-      double* lpart = p.lpart + static_cast<size_t>(buf) * rows * p.nq;
-      for (int u = u0_ + warp; u < u1_; u += kWarps) {
-        const int r = u / p.nq, qq = u % p.nq;
+      double* rpart = reinterpret_cast<double*>(stage + rpart_);
+      const int nu = (row1_ - row0_) * p.nq;
+      for (int u = warp; u < nu; u += kWarps) {
+        const int r = row0_ + u / p.nq, qq = u % p.nq;
         if (!wait_item(p1first_ + (r - row0_))) {
           hdr->abort_flag = 1;
           break;
@@ -705,7 +729,20 @@ struct LayerKernel {
           acc1 = fma(static_cast<double>(wv.w), bb.y, acc1);
         }
         const double acc = warp_sum_d(acc0 + acc1);
-        if (lane == 0) lpart[u] = acc;
+        if (lane == 0) rpart[u] = acc;
+      }
+      __syncthreads();
+      double* logits = p.logits + static_cast<size_t>(buf) * rows;
+      for (int i = threadIdx.x; i < row1_ - row0_; i += kThreads) {
+        const double* rp = rpart + i * p.nq;
+        double l;
+        if (p.nq == 4) {
+          l = ((rp[0] + rp[1]) + rp[2]) + rp[3];
+        } else {
+          l = 0.0;
+          for (int q = 0; q < p.nq; ++q) l += rp[q];
+        }
+        logits[row0_ + i] = l;
       }
     }
     __syncthreads();
@@ -731,9 +768,9 @@ struct LayerKernel {
     unsigned long long* skey = reinterpret_cast<unsigned long long*>(stage + r128(static_cast<uint32_t>(rows) * 8u));
     unsigned long long* ckey = skey + ((p.E + 15) & ~15);
     int* cidx = reinterpret_cast<int*>(ckey + ((p.E + 31) >> 5) * p.K);
-    const double* lpart = p.lpart + static_cast<size_t>(buf) * rows * p.nq;
+    const double* logits = p.logits + static_cast<size_t>(buf) * rows;
     for (int e = threadIdx.x; e < rows; e += kThreads) {
-      double l = router_logit(lpart + static_cast<size_t>(e) * p.nq, p.nq);
+      double l = __ldcg(logits + e);
       if (e < p.E && p.has_rbias) l += static_cast<double>(__ldg(p.rbias + e));
       slog[e] = l;
       if (e < p.E) skey[e] = dkey(l);
@@ -903,16 +940,28 @@ struct LayerKernel {
     } else if (threadIdx.x == 32 && p.mode != MODE_ROUTE) {
       plan_experts();
     }
-    // everything above touches only shared memory and the parameters; from here on
-    // the kernel reads what the previous grid may have written
+    __syncthreads();
+    if (p.timeline_token == 0) {  // diagnostic: the launch's start, before the grid dependency wait
+      tok_ = 0;
+      mark(13);
+      tok_ = -1;
+    }
+    const bool route = p.mode != MODE_EXPERTS;
+    const bool do_experts = p.mode != MODE_ROUTE;
+    // the first token's router rows and shared gate/up rows are weights, which no
+    // grid writes: their copies start before the wait for the previous grid
+    if (route) phase1_issue(route, do_experts && p.has_shared);
+    // everything above reads only weights, shared memory and the parameters; from here
+    // on the kernel reads what the previous grid may have written
     grid_dependency_wait();
     if (threadIdx.x == 0) hdr->tok_base = ld_relaxed_u32(p.tokens);
     const uint32_t err0 = ld_relaxed_u32(p.err);
     __syncthreads();
     tbase_ = hdr->tok_base;
-    if (err0 != 0) return;  // sticky error from an earlier call
-    const bool route = p.mode != MODE_EXPERTS;
-    const bool do_experts = p.mode != MODE_ROUTE;
+    if (err0 != 0) {  // sticky error from an earlier call
+      drain();
+      return;
+    }
     for (int t = 0; t < p.T; ++t) {
       const int buf = t & 1;
       tok_ = t;
@@ -921,8 +970,9 @@ struct LayerKernel {
         given_routing(t);
         if (hdr->skip_token) continue;
       }
-      // weight copies first, activations while they fly
-      phase1_issue(route, do_experts && p.has_shared);
+      // weight copies first (the first token's are in flight already), activations
+      // while they fly
+      if (!route || t > 0) phase1_issue(route, do_experts && p.has_shared);
       double2* xa = route ? reinterpret_cast<double2*>(stage) : nullptr;
       stage_x(p.x + static_cast<size_t>(t) * p.H, xa, xa ? xa + p.H / 4 : nullptr);
       __syncthreads();
