@@ -9,7 +9,11 @@ fmoe_layer_forward call (one fused kernel launch), the 1000 launches replayed
 from one CUDA graph.  Weights (3.64 GB) are resident in HBM; the L2 is flushed
 between steps.
 
-  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+The default single-GPU run adds sub-records for the layer stacks (24 layers of
+4-bit, 60 layers of 2-bit, 16 layers of batched top-10 decode), each with its own
+roofline, clocks and CPU-oracle sample.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--config NAME]
 
 With N > 1 (launched by torch.distributed.run) every rank runs an independent
 replica on its own GPU (the layer has no exchange step): value = tokens of all
@@ -41,8 +45,10 @@ def parse():
     ap.add_argument("--impl", default="fmoe", choices=["fmoe", "reference"])
     ap.add_argument("--config", default="layer4096")
     ap.add_argument("--tokens", type=int, default=None)
-    ap.add_argument("--cpu-sample", type=int, default=10,
+    ap.add_argument("--cpu-sample", type=int, default=6,
                     help="tokens timed once for the CPU oracle baseline of the GPU arm")
+    ap.add_argument("--sub-steps", type=int, default=3, help="timed steps of each stack sub-record")
+    ap.add_argument("--no-sub", action="store_true", help="skip the stack sub-records of the default run")
     ap.add_argument("--ref-tokens", type=int, default=1,
                     help="tokens per step of the reference arm (the CPU oracle)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -125,14 +131,14 @@ def kernel_source_digest(texts) -> str:
     return h.hexdigest()
 
 
-def profiled_traffic():
-    """DRAM bytes per launch of the layer kernel from the committed ncu summary, if
-    the kernel source is the one that was profiled (else None)."""
+def profiled_traffic(key: str = "traffic_bytes_per_launch", summary: str = "fmoe_layer_kernel_layer4096.md"):
+    """DRAM bytes per launch of the layer kernel (`key`) from a committed ncu summary,
+    if the kernel source is the one that was profiled (else None)."""
     texts = []
     for f in KERNEL_SOURCES:
         with open(os.path.join(ROOT, "bit_dequant_expert_softmax_b200", "csrc", f)) as fh:
             texts.append(fh.read())
-    path = os.path.join(ROOT, "profiles", "fmoe_layer_kernel_layer4096.md")
+    path = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(path):
         return None
     want, traffic = None, None
@@ -141,7 +147,7 @@ def profiled_traffic():
             line = line.strip()
             if line.startswith("kernel_source_digest:"):
                 want = line.split(":", 1)[1].strip()
-            elif line.startswith("traffic_bytes_per_launch:"):
+            elif line.startswith(key + ":"):
                 traffic = int(line.split(":", 1)[1].strip())
     return traffic if want == kernel_source_digest(texts) else None
 
@@ -173,32 +179,59 @@ def layer_bytes(shape):
     return experts, router + io
 
 
-def cpu_oracle_rate(shape, n_tokens: int, seed: int = 0):
-    """The fp64 oracle (as it stands) on n_tokens tokens of the workload: returns
-    (tokens/s, threads used, description).  Expert records are regenerated before
-    each token's timed forward, which is then run from the packed bytes."""
-    import numpy as np
-
+def cpu_oracle_rates(shape, n_tokens: int, block: bool = False, seed: int = 0, t0: int = 0, single: bool = True):
+    """The fp64 oracle (as it stands) on n_tokens tokens of the workload, timed twice:
+    with the BLAS thread pool limited to one thread, and with its default size (all
+    host cores).  block=True times pre-norm blocks (RMSNorm + layer), the unit of the
+    stacks.  Expert records are regenerated before each token's timed forward, which
+    then runs from the packed bytes (the decode of the records is timed).  Returns
+    {"single": tokens/s, "all": tokens/s, "threads_all": BLAS threads, "cores": nproc}."""
     import fmoe_synth as synth
     import oracle
     olay = oracle.synthetic_layer(seed, 0, shape, lazy=True)
-    total = 0.0
+    tokens = []
+    cache = {}
     for t in range(n_tokens):
-        x = oracle.bf16_to_f64(synth.gen_x_token(seed, t, shape.hidden))
-        idx, _, _, _ = olay.route(x)
-        recs = {int(e): synth.gen_record(seed, 0, int(e), shape.hidden, shape.inter, shape.bits)
-                for e in list(idx) + [shape.n_experts]}
-        olay._cache = {}
-        olay._records = lambda e, _r=recs: _r[e]
-        t0 = time.perf_counter()
-        olay.forward(x)
-        total += time.perf_counter() - t0
+        x = oracle.bf16_to_f64(synth.gen_x_token(seed, t0 + t, shape.hidden))
+        xin = oracle.bf16_to_f64(oracle.rmsnorm_bf16(x)) if block else x
+        idx, _, _, _ = olay.route(xin)
+        for e in list(idx) + ([shape.n_experts] if shape.has_shared else []):
+            if int(e) not in cache:
+                cache[int(e)] = synth.gen_record(seed, 0, int(e), shape.hidden, shape.inter, shape.bits)
+        tokens.append(x)
+
+    def timed():
+        total = 0.0
+        for x in tokens:
+            olay._cache = {}
+            olay._records = lambda e, _r=cache: _r[e]
+            t_start = time.perf_counter()
+            if block:
+                oracle.block_forward(olay, x)
+            else:
+                olay.forward(x)
+            total += time.perf_counter() - t_start
+        return n_tokens / total
+
+    threads_all, one = 1, None
     try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:  # noqa: BLE001
-        threads = 1
-    return n_tokens / total, threads, f"{n_tokens} tokens of the {shape.hidden}x{shape.inter} layer"
+        from threadpoolctl import threadpool_info, threadpool_limits
+        threads_all = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        if single:
+            with threadpool_limits(limits=1):
+                one = timed()
+    except ImportError:  # without threadpoolctl only the default pool is timed
+        pass
+    return {"single": one, "all": timed(), "threads_all": threads_all, "cores": os.cpu_count()}
+
+
+def cpu_baseline_line(rates, unit_scale: float, unit: str, sample: str):
+    """The bench line's cpu_baseline object: the all-core rate is the value (times
+    unit_scale, e.g. 1/L for an L-layer stack), the single-thread one beside it."""
+    return {"value": rates["all"] * unit_scale, "unit": unit, "cores": rates["cores"], "kind": "oracle",
+            "threads": rates["threads_all"],
+            "single_thread_value": None if rates["single"] is None else rates["single"] * unit_scale,
+            "sample": sample}
 
 
 def run_reference(args, rank):
@@ -208,16 +241,16 @@ def run_reference(args, rank):
         return
     shape = synth.CONFIGS[args.config]["shape"]
     per_step = max(1, args.ref_tokens)
-    for _ in range(args.warmup and 1):
-        cpu_oracle_rate(shape, 1)
     t_all = 0.0
     tok = 0
-    threads, desc = 1, ""
-    for _ in range(args.steps):
-        rate, threads, desc = cpu_oracle_rate(shape, per_step)
-        t_all += per_step / rate
+    threads = 1
+    for i in range(args.steps):
+        rates = cpu_oracle_rates(shape, per_step, t0=i * per_step, single=False)
+        threads = rates["threads_all"]
+        t_all += per_step / rates["all"]
         tok += per_step
     value = tok / t_all
+    desc = f"{per_step} tokens of the {shape.hidden}x{shape.inter} layer"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 * t_all / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -226,16 +259,17 @@ def run_reference(args, rank):
                                    f"inter {shape.inter}, {shape.n_experts}+{shape.has_shared} experts, "
                                    f"top-{shape.top_k}, {shape.bits}-bit",
                        "tokens_per_step": per_step},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                             "sample": f"{per_step} tokens per step ({desc})"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": os.cpu_count(), "threads": threads,
+                             "kind": "oracle", "sample": f"{per_step} tokens per step ({desc})"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def bench_stack(args, world, rank):
+def bench_stack(args, world, rank, config, steps, warmup, cpu_tokens):
     """A layer stack (pre-norm blocks) decoding its token set through the captured
     graph: token after token (batch 1) or in steps of `batch` tokens on the batched
-    path.  One step = every token of the set through every layer."""
+    path.  One step = every token of the set through every layer.  Returns the bench
+    line (rank 0; None elsewhere)."""
     import torch
     import torch.distributed as dist
 
@@ -243,7 +277,7 @@ def bench_stack(args, world, rank):
     from bit_dequant_expert_softmax_b200 import fmoe
     from fmoe_synth.torch_layer import make_device_layer, make_device_x
 
-    cfg_d = synth.CONFIGS[args.config]
+    cfg_d = synth.CONFIGS[config]
     shape, NL, B = cfg_d["shape"], cfg_d["layers"], cfg_d["batch"]
     tokens = args.tokens or cfg_d["tokens"]
     H = shape.hidden
@@ -269,18 +303,18 @@ def bench_stack(args, world, rank):
         torch.cuda.synchronize()
 
     with torch.cuda.stream(stream):
-        for _ in range(max(3, args.warmup)):
+        for _ in range(max(3, warmup)):
             h.copy_(h0)
             graph.launch(stream)
     torch.cuda.synchronize()
     sampler = ClockSampler(torch.cuda.current_device())
     sampler.start()
     time.sleep(0.3)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     barrier()
     with torch.cuda.stream(stream):
-        for i in range(args.steps):
+        for i in range(steps):
             h.copy_(h0)           # every step decodes the same token set
             flush.fill_(i & 0xFF)  # L2 flush (outside the timed events)
             starts[i].record(stream)
@@ -300,7 +334,7 @@ def bench_stack(args, world, rank):
     barrier()
     with torch.cuda.stream(stream):
         e_s.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             h.copy_(hh, non_blocking=True)
             graph.launch(stream)
             ho.copy_(h, non_blocking=True)
@@ -328,49 +362,51 @@ def bench_stack(args, world, rank):
         step_bytes = tokens * NL * ((shape.top_k + shape.has_shared) * rb + router_b)
         expert_bytes = tokens * NL * (shape.top_k + shape.has_shared) * rb
     peak, peak_kind = measured_peaks()
-    step_s = total_ms / 1e3 / args.steps
+    step_s = total_ms / 1e3 / steps
     achieved = step_bytes / step_s / 1e9
-    value = job_rate(tokens * args.steps, world, total_ms)
-    if rank == 0:
-        launches_per_layer = 1 if B == 1 else 6
-        line = {"metric": f"{NL}-layer stack decode tokens/s", "value": value, "unit": "tokens/s",
-                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-                "data": "synthetic",
-                "config": {"workload": f"{args.config}: {NL} pre-norm layers, hidden {H}, inter {shape.inter}, "
-                                       f"{shape.n_experts}+{shape.has_shared} experts, top-{shape.top_k}, "
-                                       f"{shape.bits}-bit, {tokens} tokens "
-                                       + ("one at a time" if B == 1 else f"in steps of {B} grouped by expert"),
-                           "tokens_per_step": tokens, "l2": "flushed between steps (512 MiB write)",
-                           "parallelism": f"replicas x{world}"},
-                "e2e": {"value": job_rate(tokens * args.steps, world, e2e_ms), "unit": "tokens/s",
-                        "h2d_bytes_per_step": hh.numel() * 2, "d2h_bytes_per_step": ho.numel() * 2},
-                "gpu_launches": args.steps * NL * (tokens if B == 1 else -(-tokens // B) * launches_per_layer),
-                "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                             "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
-                             "kernel": "whole step (all kernels)", "bytes_per_step": step_bytes,
-                             "expert_gbs": round(expert_bytes / step_s / 1e9, 1),
-                             "mean_distinct_experts_per_layer_step": mean_u},
-                "cpu_baseline": None, "clocks": clocks,
-                "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)}}
-        print(json.dumps(line), flush=True)
+    value = job_rate(tokens * steps, world, total_ms)
     graph.close()
     stack.close()
     for L in layers:
         L.close()
+    del layers, graph, stack
+    torch.cuda.empty_cache()
+    if rank != 0:
+        return None
+    cpu = None
+    if world == 1 and cpu_tokens > 0:
+        rates = cpu_oracle_rates(shape, cpu_tokens, block=True)
+        cpu = cpu_baseline_line(rates, 1.0 / NL, "tokens/s",
+                                f"{cpu_tokens} pre-norm blocks of layer 0 (fp64 numpy oracle), one token each; "
+                                f"rate through all {NL} layers = block rate / {NL}")
+    launches_per_layer = 1 if B == 1 else 6
+    return {"metric": f"{NL}-layer stack decode tokens/s", "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": steps, "warmup": max(3, warmup), "ms_per_step": total_ms / steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": f"{config}: {NL} pre-norm layers, hidden {H}, inter {shape.inter}, "
+                                   f"{shape.n_experts}+{shape.has_shared} experts, top-{shape.top_k}, "
+                                   f"{shape.bits}-bit, {tokens} tokens "
+                                   + ("one at a time" if B == 1 else f"in steps of {B} grouped by expert"),
+                       "tokens_per_step": tokens, "l2": "flushed between steps (512 MiB write)",
+                       "parallelism": f"replicas x{world}"},
+            "e2e": {"value": job_rate(tokens * steps, world, e2e_ms), "unit": "tokens/s",
+                    "h2d_bytes_per_step": hh.numel() * 2, "d2h_bytes_per_step": ho.numel() * 2},
+            "gpu_launches": steps * NL * (tokens if B == 1 else -(-tokens // B) * launches_per_layer),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "whole step (all kernels)", "bytes_per_step": step_bytes,
+                         "expert_gbs": round(expert_bytes / step_s / 1e9, 1),
+                         "expert_frac_of_8tbs": round(expert_bytes / step_s / 1e9 / HBM_NOMINAL_GBS, 4),
+                         "us_per_layer_token": round(step_s * 1e6 / (NL * tokens), 3),
+                         "mean_distinct_experts_per_layer_step": mean_u},
+            "cpu_baseline": cpu, "clocks": clocks,
+            "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)}}
 
 
-def main():
-    args = parse()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
-        run_reference(args, rank)
-        return
-
-    import datetime
-
+def bench_layer(args, world, rank, config):
+    """The single-layer workload: every token one fmoe_layer_forward call, the calls
+    of a step replayed from one CUDA graph.  Returns the bench line (rank 0)."""
     import torch
     import torch.distributed as dist
 
@@ -378,17 +414,8 @@ def main():
     from bit_dequant_expert_softmax_b200 import fmoe
     from fmoe_synth.torch_layer import make_device_layer, make_device_x
 
-    torch.cuda.set_device(local_rank)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
-    if synth.CONFIGS[args.config]["layers"] > 1 or synth.CONFIGS[args.config]["batch"] > 1:
-        bench_stack(args, world, rank)
-        if world > 1:
-            dist.destroy_process_group()
-        return
-    shape = synth.CONFIGS[args.config]["shape"]
-    tokens = args.tokens or synth.CONFIGS[args.config]["tokens"]
+    shape = synth.CONFIGS[config]["shape"]
+    tokens = args.tokens or synth.CONFIGS[config]["tokens"]
     H = shape.hidden
 
     w = make_device_layer(shape, 0, 0)
@@ -459,6 +486,10 @@ def main():
         e_e.record(stream)
     barrier()
     e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), world)
+    del graph
+    L.close()
+    del w, x, y, flush
+    torch.cuda.empty_cache()
 
     value = job_rate(tokens * args.steps, world, total_ms)
     e2e_value = job_rate(tokens * args.steps, world, e2e_ms)
@@ -469,34 +500,74 @@ def main():
     expert_gbs = expert_b / launch_s / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
-            "peak_kind": peak_kind, "kernel": "fmoe_layer_kernel<4>",
+            "traffic_warm": profiled_traffic("traffic_warm_bytes_per_launch"),
+            "traffic_note": "traffic: DRAM read+write bytes of one cold-L2 launch (ncu flushes L2); "
+                            "traffic_warm: per launch over consecutive launches without flushing, as in "
+                            "the timed loop (the router and the shared expert can stay in L2 there)",
+            "peak_kind": peak_kind, "kernel": f"fmoe_layer_kernel<{shape.bits}>",
             "bytes_per_launch": expert_b + other_b, "expert_bytes_per_launch": expert_b,
             "expert_gbs": round(expert_gbs, 1), "expert_frac_of_8tbs": round(expert_gbs / HBM_NOMINAL_GBS, 4),
             "expert_frac_of_measured": round(expert_gbs / peak, 4), "avg_launch_us": round(launch_s * 1e6, 3)}
+    if rank != 0:
+        return None
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, threads, desc = cpu_oracle_rate(shape, args.cpu_sample)
-        cpu = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"{args.cpu_sample} tokens ({desc}), fp64 numpy oracle"}
+    if world == 1 and not args.no_cpu_baseline:
+        rates = cpu_oracle_rates(shape, args.cpu_sample)
+        cpu = cpu_baseline_line(rates, 1.0, "tokens/s",
+                                f"{args.cpu_sample} tokens of the {H}x{shape.inter} layer (fp64 numpy oracle, "
+                                f"expert records decoded in the timed forward)")
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": f"{config}: single-token decode, hidden {H}, inter {shape.inter}, "
+                                   f"{shape.n_experts}+{shape.has_shared} experts, top-{shape.top_k}, "
+                                   f"{shape.bits}-bit group-64",
+                       "weights": f"{shape.bits}-bit codes, bf16 scale/bias per 64-group, HBM-resident",
+                       "tokens_per_step": tokens, "l2": "flushed between steps (512 MiB write)",
+                       "parallelism": f"replicas x{world}"},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": xh.numel() * 2,
+                    "d2h_bytes_per_step": yh.numel() * 2},
+            "gpu_launches": tokens * args.steps,
+            "roofline": roof, "cpu_baseline": cpu, "clocks": clocks,
+            "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)}}
+
+
+SUB_CONFIGS = ("stack24_4bit", "stack60_2bit", "stack16_batched")
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import fmoe_synth as synth
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    cfg = synth.CONFIGS[args.config]
+    if cfg["layers"] > 1 or cfg["batch"] > 1:
+        line = bench_stack(args, world, rank, args.config, args.steps, args.warmup,
+                           0 if args.no_cpu_baseline else 2)
+    else:
+        line = bench_layer(args, world, rank, args.config)
+        # the stacks ride along as sub-records of the default single-GPU run
+        if world == 1 and args.config == "layer4096" and not args.no_sub and args.tokens is None:
+            line["sub_records"] = [bench_stack(args, world, rank, c, args.sub_steps, 3,
+                                               0 if args.no_cpu_baseline else 2) for c in SUB_CONFIGS]
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-                "data": "synthetic",
-                "config": {"workload": f"{args.config}: single-token decode, hidden {H}, inter {shape.inter}, "
-                                       f"{shape.n_experts}+{shape.has_shared} experts, top-{shape.top_k}, "
-                                       f"{shape.bits}-bit group-64",
-                           "weights": f"{shape.bits}-bit codes, bf16 scale/bias per 64-group, HBM-resident",
-                           "tokens_per_step": tokens, "l2": "flushed between steps (512 MiB write)",
-                           "parallelism": f"replicas x{world}"},
-                "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": xh.numel() * 2,
-                        "d2h_bytes_per_step": yh.numel() * 2},
-                "gpu_launches": tokens * args.steps,
-                "roofline": roof, "cpu_baseline": cpu, "clocks": clocks,
-                "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)}}
         print(json.dumps(line), flush=True)
-    del graph
-    L.close()
     if world > 1:
         dist.destroy_process_group()
 

@@ -610,6 +610,9 @@ struct LayerKernel {
     const uint32_t lead = static_cast<uint32_t>((p.o_d_sb + static_cast<unsigned long long>(ja) * p.si) & 15ull);
     const int nch = p.I / C::kCols, sw = p.si / 4;
     float* ob = xs;  // [nslots][n]
+    // the residual of the item's rows, loaded before the dot products (one coalesced
+    // load; in a stack block y is the residual buffer itself, rows of this block only)
+    const float rj = threadIdx.x < n ? bf16_to_f32(resid_t[ja + threadIdx.x]) : 0.f;
     bool ok = warp >= nu || wait_item(item);
     if (!ok) hdr->abort_flag = 1;
     for (int u = warp; ok && u < nu; u += kWarps) {
@@ -640,10 +643,11 @@ struct LayerKernel {
     }
     __syncthreads();
     if (hdr->abort_flag) return false;
-    for (int j = threadIdx.x; j < n; j += kThreads) {
+    if (threadIdx.x < n) {
+      const int j = threadIdx.x;
       float pa = 0.f;
       for (int s = 0; s < nslots; ++s) pa = fmaf(hdr->wsl[s], ob[s * n + j], pa);
-      y_t[ja + j] = f32_to_bf16(bf16_to_f32(resid_t[ja + j]) + pa);
+      y_t[ja + j] = f32_to_bf16(rj + pa);
     }
     __syncthreads();
     return true;

@@ -218,9 +218,14 @@ def expert_hidden(ex: DenseExpert, x: np.ndarray) -> np.ndarray:
 
 def shared_sigma(gs: np.ndarray, x: np.ndarray) -> float:
     """sigma = 1 / (1 + exp(-g_s . x)), the sigmoid gate of the shared expert
-    (hotdry.top, "Metal GPU管线"); a vector g_s is the reading."""
+    (hotdry.top, "Metal GPU管线"); a vector g_s is the reading.  For a negative
+    argument the same value is written exp(s) / (1 + exp(s)), which does not
+    overflow."""
     s = float(np.asarray(gs, dtype=np.float64) @ np.asarray(x, dtype=np.float64))
-    return 1.0 / (1.0 + math.exp(-s))
+    if s >= 0.0:
+        return 1.0 / (1.0 + math.exp(-s))
+    e = math.exp(s)
+    return e / (1.0 + e)
 
 
 @dataclass

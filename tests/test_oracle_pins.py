@@ -266,6 +266,11 @@ def test_shared_gate_matches_library_sigmoid():
         gs, x = rng.standard_normal(64), rng.standard_normal(64)
         s = math.fsum(float(a) * float(b) for a, b in zip(gs, x))
         assert math.isclose(oracle.shared_sigma(gs, x), float(scipy.special.expit(s)), rel_tol=1e-14)
+    # arguments far beyond exp's range: sigma tends to 0 and 1 without overflowing
+    for s in (-800.0, -50.0, -3.5, 3.5, 50.0, 800.0, 1e6, -1e6):
+        gs, x = np.array([s]), np.array([1.0])
+        got = oracle.shared_sigma(gs, x)
+        assert math.isclose(got, float(scipy.special.expit(s)), rel_tol=1e-14, abs_tol=1e-300), s
 
 
 def test_power_of_two_down_scaling_is_exact():
