@@ -101,6 +101,21 @@ __device__ __forceinline__ ulonglong2 ld_volatile_v2_u64(const unsigned long lon
   return v;
 }
 
+// 16-byte store of two 64-bit words, each written single-copy atomically.
+__device__ __forceinline__ void st_relaxed_v2_u64(unsigned long long* p, unsigned long long a, unsigned long long b) {
+  asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(a), "l"(b) : "memory");
+}
+
+// Values exchanged between blocks travel with the token's 32-bit tag in the same
+// single-copy-atomic 64-bit word (tag in the high half): a reader that sees its
+// token's tag sees that token's value, with no flag, fence or second read.
+__device__ __forceinline__ unsigned long long tagged(uint32_t value, uint32_t tag) {
+  return (static_cast<unsigned long long>(tag) << 32) | value;
+}
+__device__ __forceinline__ bool has_tag(unsigned long long w, uint32_t tag) {
+  return static_cast<uint32_t>(w >> 32) == tag;
+}
+
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -268,7 +283,30 @@ struct Chunk {
     for (int r = 0; r < NR; ++r) V[r] = W[r] >> 8;
     steps<0, NR>(W, V, xv, acc);
   }
+
 };
+
+// Sums of four per-lane values over groups of G consecutive lanes (G = 4, 8, 16 or 32,
+// xor shuffles inside the group): value i ends in the lanes whose position p in the
+// group satisfies p / (G / 4) == i (the lane at p = i * G / 4 among them).  Six
+// shuffles for G = 32 instead of twenty.
+template <int G>
+__device__ __forceinline__ float group_sum4(float v0, float v1, float v2, float v3) {
+  const int p = static_cast<int>(threadIdx.x & 31) & (G - 1);
+  const bool hi1 = p & (G / 2);
+  // halves: the lower half of the group keeps values {0, 1}, the upper {2, 3}
+  const float s0 = hi1 ? v0 : v2, s1 = hi1 ? v1 : v3;
+  float k0 = hi1 ? v2 : v0, k1 = hi1 ? v3 : v1;
+  k0 += __shfl_xor_sync(0xffffffffu, s0, G / 2);
+  k1 += __shfl_xor_sync(0xffffffffu, s1, G / 2);
+  // quarters: keep one of the two
+  const bool hi2 = p & (G / 4);
+  float k = hi2 ? k1 : k0;
+  k += __shfl_xor_sync(0xffffffffu, hi2 ? k0 : k1, G / 4);
+#pragma unroll
+  for (int o = G / 8; o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
+  return k;
+}
 
 // 2^(P - shift): the pre-scale of an activation met by codes masked at bit `shift`.
 __device__ __forceinline__ float prescale_factor(int pre, int shift) {

@@ -2,17 +2,18 @@
 //
 // One persistent thread block per SM (cooperative launch).  Per token:
 //
-//   P1  router matvec (fp64 accumulation of exact fp32 x bf16 products) over a
-//       slice of router rows per block, partials published with a per-block flag;
-//       while they travel, warps 1-15 consume the block's slice of the shared
-//       expert's gate/up rows (they do not depend on the routing) and warp 0 polls.
-//   P2  every block computes top-K from the logits redundantly; thread 0 requests
-//       the block's slice of the K routed experts' gate/up row pairs one copy after
-//       another, and its down rows (P3's data) once half of those have landed;
-//       warps 1-15 compute h = silu(g) * u, warp 0 the renormalised softmax
-//       weights; h is published with a per-block flag.
-//   P3  every block stages h of all K+1 experts, computes its slice of output
-//       rows of the K+1 down matvecs and the combine
+//   P1  router matvec (fp64 accumulation of exact fp32 x bf16 products) over whole
+//       router rows per block (their copies start before the kernel waits for the
+//       previous grid), logits published as tagged words; while they travel, warps
+//       1-15 consume the block's slice of the shared expert's gate/up rows (they do
+//       not depend on the routing).
+//   P2  every block polls all logits and computes top-K redundantly; thread 0
+//       requests the block's slice of the K routed experts' gate/up row pairs one
+//       copy after another, and its down rows (P3's data) once half of those have
+//       landed; warps 1-15 compute h = silu(g) * u (four rows per activation load),
+//       warp 0 the renormalised softmax weights; h is published as tagged words.
+//   P3  every block polls h of all K+1 experts, computes its slice of output rows of
+//       the K+1 down matvecs (activations held in registers) and the combine
 //       y = resid + sum_k w_k o_k + sigma o_s, rounded once to bf16.
 //
 // All weight bytes move HBM -> shared memory through the bulk-copy (TMA) engine
@@ -43,8 +44,7 @@ constexpr int kMaxDownBlock = 2 * kWarps;  // output rows per down item (two per
 constexpr int kMaxChunks = 8;              // gate/up chunks per round
 constexpr int kMaxExperts = 2048;          // routed experts a layer may have
 constexpr int kMaxSplits = 4;              // router column splits
-constexpr int kMaxGrid = 256;              // blocks a launch may have (flag words reserved)
-constexpr int kFlagStride = 8;             // uint32 per flag (one 32-byte sector each)
+constexpr int kMaxGrid = 256;              // blocks a launch may have
 
 enum Mode : int { MODE_ROUTE = 1, MODE_EXPERTS = 2, MODE_FULL = 3 };
 
@@ -71,10 +71,8 @@ struct Params {
   const float* sig_in;
   uint32_t* err;
   uint32_t* tokens;  // tokens this workspace has seen (tag base)
-  uint32_t* rflags;  // [kMaxGrid * kFlagStride] per-block "router partials written" tags
-  uint32_t* hflags;  // [kMaxGrid * kFlagStride] per-block "h rows written" tags
-  double* logits;    // [2][E+1] router logits (the shared gate's dot product last)
-  float* hbuf;       // [2][(K+1)*I]  h values
+  unsigned long long* lx;  // [E+1][2] router logits as tagged words (high, low half of the double)
+  unsigned long long* hx;  // [(K+1)*I] h values as tagged words
   int norm;         // 1: the input is a pre-norm block's h (the NORM kernel variant)
   double norm_eps;
   int staging_bytes;
@@ -108,6 +106,7 @@ struct alignas(128) SmemHeader {
   float wsl[kMaxK + 1];  // weight of each slot (w_k; slot K = sigma)
   int abort_flag;
   int skip_token;
+  int shared_done;  // warps that have consumed their share of the shared expert's gate/up rows
   uint32_t tok_base;
   ExpertPlan plan;
 };
@@ -207,61 +206,33 @@ struct LayerKernel {
   }
 
   // ---------------------------------------------------------------- exchanges
-  // Values every block needs from all others (router partials, h rows) are written
-  // with plain stores; then the block publishes the token's tag in its own flag word
-  // with a release store.  A reader's warp 0 polls the grid's flags (each lane a few,
-  // all of a lane's loads in flight together, relaxed loads, bounded), fences, and
-  // the block then reads the values once from L2.  Buffers alternate by token parity;
-  // no block can run two tokens ahead of another because each token needs every
-  // block's values.
+  // Values every block needs from all others (router logits, h rows) travel as 64-bit
+  // words carrying the token's tag in their high half (fmoe::tagged).  Each word is
+  // written and read single-copy atomically (relaxed stores, volatile loads served by
+  // L2), so a reader polls the very words it needs until they carry its token's tag:
+  // no flags, no fences, no second read.  One buffer serves every token: a block
+  // overwrites its words with the next token's only after every block has read this
+  // token's (the next token's values need every block's values of this one).  Every
+  // wait is bounded by the layer's time limit.
   uint32_t tbase_;
   __device__ __forceinline__ uint32_t tag32(int t) const {
     return (tbase_ + static_cast<uint32_t>(t)) % 0xFFFFFFFFu + 1u;
   }
 
-  __device__ __forceinline__ void publish(uint32_t* flags, int t) {
-    __syncthreads();
-    if (threadIdx.x == 0) st_release_u32(flags + blockIdx.x * kFlagStride, tag32(t));
-  }
-
-  __device__ bool wait_all(const uint32_t* flags, int t) {
-    int fail = 0;
-    if (threadIdx.x < 32) {
-      const int G = gridDim.x, lane = threadIdx.x;
-      const uint32_t want = tag32(t);
-      constexpr int NF = kMaxGrid / 32;
-      uint32_t got[NF];
-#pragma unroll
-      for (int i = 0; i < NF; ++i) {
-        const int b = lane + 32 * i;
-        got[i] = b < G ? ld_relaxed_u32(flags + b * kFlagStride) : want;
+  // One step of a bounded poll: sleeps briefly; false (error bit set) once the limit
+  // has passed or another thread has given up already.
+  __device__ __forceinline__ bool poll_tick(uint64_t& t0, int& it) const {
+    if ((++it & 15) == 0) {
+      const uint64_t now = global_timer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > p.wait_ns || (ld_relaxed_u32(p.err) & FMOE_DEVERR_BARRIER_TIMEOUT)) {
+        atomicOr(p.err, FMOE_DEVERR_BARRIER_TIMEOUT);
+        return false;
       }
-      uint64_t t0 = 0;
-      for (int it = 0;; ++it) {
-        bool all = true;
-#pragma unroll
-        for (int i = 0; i < NF; ++i) all &= got[i] == want;
-        if (__all_sync(0xffffffffu, all)) break;
-        if ((it & 15) == 15) {
-          if (t0 == 0) t0 = global_timer_ns();
-          const bool bad =
-              (ld_relaxed_u32(p.err) & FMOE_DEVERR_BARRIER_TIMEOUT) || global_timer_ns() - t0 > p.wait_ns;
-          if (__any_sync(0xffffffffu, bad)) {
-            if (lane == 0) atomicOr(p.err, FMOE_DEVERR_BARRIER_TIMEOUT);
-            fail = 1;
-            break;
-          }
-        }
-        __nanosleep(32);
-#pragma unroll
-        for (int i = 0; i < NF; ++i) {
-          const int b = lane + 32 * i;
-          if (got[i] != want) got[i] = ld_relaxed_u32(flags + b * kFlagStride);
-        }
-      }
-      __threadfence();
     }
-    return __syncthreads_or(fail) == 0;
+    __nanosleep(32);
+    return true;
   }
 
   // ---------------------------------------------------------------- activations
@@ -349,27 +320,60 @@ struct LayerKernel {
     }
   }
 
-  // h of every slot (fp32, written by other blocks, read from L2 once every block
-  // has published): coalesced 16-byte loads (thread -> 4 consecutive columns), all of
-  // a thread's loads in flight together; chunk sums by shuffles over the kCols/4
-  // threads of a chunk; pre-scaled values scattered into the interleaved layout.
-  __device__ void stage_h(const float* hb, float* hs, uint32_t hstride, float2* hsum) {
+  // h of every slot (fp32 values in tagged words written by other blocks) polled from
+  // L2 until every word carries this token's tag: thread -> 4 consecutive columns (two
+  // 16-byte loads), all of a thread's loads in flight together; chunk sums and largest
+  // magnitudes by shuffles over the kCols/4 threads of a chunk; pre-scaled values
+  // scattered into the interleaved layout.  Returns false (in every thread that timed
+  // out) when a wait ran past the limit.
+  __device__ bool stage_h(float* hs, uint32_t hstride, float2* hsum) {
     constexpr int TPC = C::kCols / 4;
     const int per_slot = p.I / 4, nch = p.I / C::kCols;
     const int n4 = nslots * per_slot;
-    const float4* src = reinterpret_cast<const float4*>(hb);
-    for (int base = 0; base < n4; base += 4 * kThreads) {
-      float4 v[4];
+    const uint32_t want = tag32(tok_);
+    const unsigned long long* src = p.hx;
+    bool ok = true;
+    for (int base = 0; base < n4; base += 4 * kThreads) {  // block-uniform trip count
+      ulonglong2 a[4], b[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
-        v[k] = q < n4 ? __ldcg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (q < n4) {
+          a[k] = ld_volatile_v2_u64(src + 4 * q);
+          b[k] = ld_volatile_v2_u64(src + 4 * q + 2);
+        } else {
+          a[k] = b[k] = make_ulonglong2(tagged(0u, want), tagged(0u, want));
+        }
+      }
+      // every retry re-reads all words still missing, their loads in flight together
+      uint64_t t0 = 0;
+      int it = 0;
+      while (ok) {
+        bool all = true;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          all &= has_tag(a[k].x, want) && has_tag(a[k].y, want) && has_tag(b[k].x, want) && has_tag(b[k].y, want);
+        if (all) break;
+        if (!poll_tick(t0, it)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
+          if (!(has_tag(a[k].x, want) && has_tag(a[k].y, want))) a[k] = ld_volatile_v2_u64(src + 4 * q);
+          if (!(has_tag(b[k].x, want) && has_tag(b[k].y, want))) b[k] = ld_volatile_v2_u64(src + 4 * q + 2);
+        }
       }
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
-        float sum = (v[k].x + v[k].y) + (v[k].z + v[k].w);
-        uint32_t mx = max_abs_bits(v[k]);
+        const float4 v = make_float4(__uint_as_float(static_cast<uint32_t>(a[k].x)),
+                                     __uint_as_float(static_cast<uint32_t>(a[k].y)),
+                                     __uint_as_float(static_cast<uint32_t>(b[k].x)),
+                                     __uint_as_float(static_cast<uint32_t>(b[k].y)));
+        float sum = (v.x + v.y) + (v.z + v.w);
+        uint32_t mx = max_abs_bits(v);
 #pragma unroll
         for (int o = 1; o < TPC; o <<= 1) {
           sum += __shfl_xor_sync(0xffffffffu, sum, o);
@@ -378,47 +382,70 @@ struct LayerKernel {
         if (q < n4) {
           const int slot = q / per_slot, c0 = (q % per_slot) * 4, pre = chunk_pre(mx);
           float* d = hs + static_cast<size_t>(slot) * hstride;
-          d[phys(c0 + 0)] = v[k].x * prescale_factor(pre, C::shift_of(c0 + 0));
-          d[phys(c0 + 1)] = v[k].y * prescale_factor(pre, C::shift_of(c0 + 1));
-          d[phys(c0 + 2)] = v[k].z * prescale_factor(pre, C::shift_of(c0 + 2));
-          d[phys(c0 + 3)] = v[k].w * prescale_factor(pre, C::shift_of(c0 + 3));
+          d[phys(c0 + 0)] = v.x * prescale_factor(pre, C::shift_of(c0 + 0));
+          d[phys(c0 + 1)] = v.y * prescale_factor(pre, C::shift_of(c0 + 1));
+          d[phys(c0 + 2)] = v.z * prescale_factor(pre, C::shift_of(c0 + 2));
+          d[phys(c0 + 3)] = v.w * prescale_factor(pre, C::shift_of(c0 + 3));
           if (q % TPC == 0) hsum[slot * nch + c0 / C::kCols] = make_float2(sum, chunk_unscale(pre));
         }
       }
       if (base == 0) mark(14);
     }
     mark(15);
+    return ok;
   }
 
   __device__ __forceinline__ static int phys(int c) { return C::phys(c); }
 
   // ---------------------------------------------------------------- dot products
-  // Lane partials of sum_c W[r][c] v[c] over the lane's chunks for NR rows sharing the
-  // activation loads (W = scale*code + bias; v pre-scaled, interleaved).  Every row is
-  // summed in the same order whatever NR is.
+  // Lane partials of sum_c W[r][c] v[c] for NR rows sharing the activation loads (W =
+  // scale*code + bias; v pre-scaled, interleaved).  The lanes stride over chunk parts:
+  // a 4-bit chunk (32 columns) is one part; a 2-bit chunk (64 columns) is two, one word
+  // pair each, so that rows of few chunks still keep every lane busy (the chunk's bias
+  // term goes with its first part).  Every row is summed in the same order whatever NR
+  // is.
   template <int NR>
   __device__ __forceinline__ void dotr(const uint8_t* const (&q)[NR], const uint32_t* const (&sb)[NR],
                                        const float* vs, const float2* vsum, int nch, float (&res)[NR]) const {
+    constexpr int PPC = BITS == 2 ? 2 : 1;  // parts per chunk
     const int lane = threadIdx.x & 31;
 #pragma unroll(NR <= 2 ? 2 : 1)
-    for (int m = lane; m < nch; m += 32) {
-      unsigned long long wx[NR], wy[NR], a0[NR], a1[NR];
-#pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        const ulonglong2 w = *reinterpret_cast<const ulonglong2*>(q[r] + 16 * m);
-        wx[r] = w.x;
-        wy[r] = w.y;
-        a0[r] = 0ull;
-        a1[r] = 0ull;
-      }
-      C::template word_pairs<NR>(wx, C::f4(vs, m, 0), a0);
-      C::template word_pairs<NR>(wy, C::f4(vs, m, C::kF4PerPair), a1);
+    for (int u = lane; u < nch * PPC; u += 32) {
+      const int m = u / PPC, half = u % PPC;
+      unsigned long long a0[NR];
       const float2 vm = vsum[m];  // (sum of the chunk's activations, rescale of its products)
+      if constexpr (PPC == 1) {
+        unsigned long long wx[NR], wy[NR], a1[NR];
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        const uint32_t sbv = sb[r][C::sb_index(m)];
-        res[r] = fmaf(sb_scale(sbv), (pair_sum(a0[r]) + pair_sum(a1[r])) * vm.y, res[r]);
-        res[r] = fmaf(sb_bias(sbv), vm.x, res[r]);
+        for (int r = 0; r < NR; ++r) {
+          const ulonglong2 w = *reinterpret_cast<const ulonglong2*>(q[r] + 16 * m);
+          wx[r] = w.x;
+          wy[r] = w.y;
+          a0[r] = 0ull;
+          a1[r] = 0ull;
+        }
+        C::template word_pairs<NR>(wx, C::f4(vs, m, 0), a0);
+        C::template word_pairs<NR>(wy, C::f4(vs, m, C::kF4PerPair), a1);
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          const uint32_t sbv = sb[r][C::sb_index(m)];
+          res[r] = fmaf(sb_scale(sbv), (pair_sum(a0[r]) + pair_sum(a1[r])) * vm.y, res[r]);
+          res[r] = fmaf(sb_bias(sbv), vm.x, res[r]);
+        }
+      } else {
+        unsigned long long wx[NR];
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          wx[r] = *reinterpret_cast<const unsigned long long*>(q[r] + 16 * m + 8 * half);
+          a0[r] = 0ull;
+        }
+        C::template word_pairs<NR>(wx, C::f4(vs, m, half * C::kF4PerPair), a0);
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          const uint32_t sbv = sb[r][C::sb_index(m)];
+          res[r] = fmaf(sb_scale(sbv), pair_sum(a0[r]) * vm.y, res[r]);
+          if (half == 0) res[r] = fmaf(sb_bias(sbv), vm.x, res[r]);
+        }
       }
     }
   }
@@ -461,9 +488,9 @@ struct LayerKernel {
     }
   }
 
-  // h of row pairs r .. r+np-1 (np = 1 or 2) of the chunk -> hbuf[buf][slot][r ..]  (one
+  // h of row pairs r .. r+np-1 (np = 1 or 2) of the chunk -> the tagged h words of the slot (one
   // warp); two row pairs are four rows sharing the activation loads.
-  __device__ bool gu_unit(const GuChunk& c, int r, int np, int buf) {
+  __device__ bool gu_unit(const GuChunk& c, int r, int np) {
     const int n = c.rb - c.ra, i = r - c.ra;
     if (!wait_item(c.first + i / p.rp)) return false;
     if ((i + np - 1) / p.rp != i / p.rp && !wait_item(c.first + (i + np - 1) / p.rp)) return false;
@@ -473,7 +500,8 @@ struct LayerKernel {
         static_cast<uint32_t>((p.o_gu_sb + static_cast<unsigned long long>(c.ra) * 2u * p.sh) & 15ull);
     const uint32_t* sg = reinterpret_cast<const uint32_t*>(stage + c.off + g.gu_q(n) + lead) + i * 2 * (p.sh / 4);
     const int sw = p.sh / 4;
-    float* hout = p.hbuf + static_cast<size_t>(buf) * (p.K + 1) * p.I + static_cast<size_t>(c.slot) * p.I + r;
+    unsigned long long* hout = p.hx + static_cast<size_t>(c.slot) * p.I + r;
+    const uint32_t tag = tag32(tok_);
     if (np == 2) {
       const uint8_t* const q[4] = {qg, qg + p.qh, qg + 2 * p.qh, qg + 3 * p.qh};
       const uint32_t* const sb[4] = {sg, sg + sw, sg + 2 * sw, sg + 3 * sw};
@@ -482,8 +510,8 @@ struct LayerKernel {
 #pragma unroll
       for (int k = 0; k < 4; ++k) v[k] = warp_sum(v[k]);
       if ((threadIdx.x & 31) == 0) {
-        hout[0] = (v[0] / (1.0f + expf(-v[0]))) * v[1];
-        hout[1] = (v[2] / (1.0f + expf(-v[2]))) * v[3];
+        st_relaxed_u64(hout, tagged(__float_as_uint((v[0] / (1.0f + expf(-v[0]))) * v[1]), tag));
+        st_relaxed_u64(hout + 1, tagged(__float_as_uint((v[2] / (1.0f + expf(-v[2]))) * v[3]), tag));
       }
     } else {
       const uint8_t* const q[2] = {qg, qg + p.qh};
@@ -492,25 +520,27 @@ struct LayerKernel {
       dotr<2>(q, sb, xs, xsum, p.H / C::kCols, v);
       v[0] = warp_sum(v[0]);
       v[1] = warp_sum(v[1]);
-      if ((threadIdx.x & 31) == 0) hout[0] = (v[0] / (1.0f + expf(-v[0]))) * v[1];
+      if ((threadIdx.x & 31) == 0)
+        st_relaxed_u64(hout, tagged(__float_as_uint((v[0] / (1.0f + expf(-v[0]))) * v[1]), tag));
     }
     return true;
   }
 
-  // Consume every row pair of `nc` chunks in units of two row pairs, spread over warps
-  // w0 .. kWarps-1 (unit u -> warp w0 + u % (kWarps - w0)); w0 = 1 keeps warp 0, which
-  // issues the copies and computes the routing weights meanwhile, out of the routed rows.
-  __device__ void gu_consume(const GuChunk* ch, int nc, int buf, int w0 = 0) {
+  // Consume every row pair of `nc` chunks in units of `upairs` (1 or 2) row pairs, spread
+  // over warps w0 .. kWarps-1 (unit u -> warp w0 + u % (kWarps - w0)); w0 = 1 keeps warp
+  // 0, which issues the copies and computes the routing weights meanwhile, out of the
+  // routed rows.
+  __device__ void gu_consume(const GuChunk* ch, int nc, int w0 = 0, int upairs = 2) {
     const int warp = threadIdx.x >> 5;
     if (warp < w0) return;
     const int nw = kWarps - w0;
     int base = 0;
     for (int k = 0; k < nc; ++k) {
-      const int n = ch[k].rb - ch[k].ra, nu = (n + 1) / 2;
+      const int n = ch[k].rb - ch[k].ra, nu = (n + upairs - 1) / upairs;
       int first = (warp - w0 - base) % nw;
       if (first < 0) first += nw;
       for (int u = first; u < nu; u += nw) {
-        if (!gu_unit(ch[k], ch[k].ra + 2 * u, min(2, n - 2 * u), buf)) {
+        if (!gu_unit(ch[k], ch[k].ra + upairs * u, min(upairs, n - upairs * u))) {
           hdr->abort_flag = 1;
           return;
         }
@@ -521,7 +551,7 @@ struct LayerKernel {
 
   // Gate/up of routed units [v0, v1) (unit = slot*I + r) in rounds that fit the
   // whole staging area (used when the block's share does not fit at once).
-  __device__ bool gu_rounds(int v0, int v1, int buf) {
+  __device__ bool gu_rounds(int v0, int v1) {
     GuChunk ch[kMaxChunks];
     int nc = 0, items = 0;
     uint32_t used = 0;
@@ -548,7 +578,7 @@ struct LayerKernel {
         }
         issue_gu(ch, nc);
         nitem += static_cast<uint32_t>(items);
-        gu_consume(ch, nc, buf);
+        gu_consume(ch, nc);
         __syncthreads();
         if (hdr->abort_flag) return false;
         nc = 0;
@@ -598,55 +628,84 @@ struct LayerKernel {
     }
   }
 
-  // Consume a down item (rows [ja, ja+n) of every slot): units (slot, group of up to
-  // four rows) are spread over the warps, four rows sharing each activation load; the
-  // rows' results o_s[j] are gathered in shared memory over the activations x (no
-  // longer read in this phase), then y = resid + sum_s w_s o_s[j], summed in slot order
-  // and rounded once.  Called by every thread; returns false for all on an abort.
-  __device__ bool down_item(uint32_t item, uint32_t off, int ja, int n, const float* hs, const float2* hsum,
-                            const uint16_t* resid_t, uint16_t* y_t) {
+  // Down rows of an item as cells (group of up to four rows, slot): each warp takes a
+  // contiguous range of cells in group-major order, four rows sharing each activation
+  // load; its lanes accumulate w_s * o_s over the slots of a group and reduce the four
+  // rows once per group (group_sum4).  The weighted sum of a warp's run of slots
+  // [s0, s1) of group g goes to ob[s0 * n + j], zeros to the other slots of the run, so
+  // that every (slot, row) entry is written exactly once.
+  __device__ void down_cells(uint32_t off, int n, const float* hs, const float2* hsum, uint32_t lead, float* ob) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ng = (n + 3) >> 2, nu = nslots * ng;
-    const uint32_t lead = static_cast<uint32_t>((p.o_d_sb + static_cast<unsigned long long>(ja) * p.si) & 15ull);
     const int nch = p.I / C::kCols, sw = p.si / 4;
-    float* ob = xs;  // [nslots][n]
-    // the residual of the item's rows, loaded before the dot products (one coalesced
-    // load; in a stack block y is the residual buffer itself, rows of this block only)
-    const float rj = threadIdx.x < n ? bf16_to_f32(resid_t[ja + threadIdx.x]) : 0.f;
-    bool ok = warp >= nu || wait_item(item);
-    if (!ok) hdr->abort_flag = 1;
-    for (int u = warp; ok && u < nu; u += kWarps) {
-      const int s = u / ng, j0 = (u % ng) * 4, nr = min(4, n - j0);
-      const uint8_t* blk = stage + off + s * g.dn_slot(n);
+    const int ng = (n + 3) >> 2, cells = ng * nslots;
+    const int c0 = cells * warp / kWarps, c1 = cells * (warp + 1) / kWarps;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int cg = -1, s0 = 0;
+    auto flush = [&](int s1) {
+      const float r = group_sum4<32>(acc[0], acc[1], acc[2], acc[3]);
+      const int q = lane >> 3, j = 4 * cg + q;
+      if ((lane & 7) == 0 && j < n) {
+        ob[s0 * n + j] = r;
+        for (int sl = s0 + 1; sl < s1; ++sl) ob[sl * n + j] = 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] = 0.f;
+    };
+    for (int c = c0; c < c1; ++c) {
+      const int gi = c / nslots, sl = c % nslots;
+      if (gi != cg) {
+        if (cg >= 0) flush(nslots);
+        cg = gi;
+        s0 = sl;
+      }
+      const int j0 = 4 * gi, nr = min(4, n - j0);
+      const uint8_t* blk = stage + off + sl * g.dn_slot(n);
       const uint8_t* q0 = blk + static_cast<uint32_t>(j0) * p.qi;
-      const uint32_t* s0 = reinterpret_cast<const uint32_t*>(blk + g.dn_q(n) + lead) + j0 * sw;
-      const float* hsl = hs + static_cast<size_t>(s) * g.padded(p.I);
-      const float2* hsm = hsum + static_cast<size_t>(s) * nch;
+      const uint32_t* sp = reinterpret_cast<const uint32_t*>(blk + g.dn_q(n) + lead) + j0 * sw;
+      const float* hsl = hs + static_cast<size_t>(sl) * g.padded(p.I);
+      const float2* hsm = hsum + static_cast<size_t>(sl) * nch;
+      const float ws = hdr->wsl[sl];
       float v[4] = {0.f, 0.f, 0.f, 0.f};
       if (nr > 2) {  // a group of three repeats its last row (the fourth result is dropped)
         const int r3 = nr - 1;
         const uint8_t* const q[4] = {q0, q0 + p.qi, q0 + 2 * p.qi, q0 + r3 * p.qi};
-        const uint32_t* const sb[4] = {s0, s0 + sw, s0 + 2 * sw, s0 + r3 * sw};
+        const uint32_t* const sb[4] = {sp, sp + sw, sp + 2 * sw, sp + r3 * sw};
         dotr<4>(q, sb, hsl, hsm, nch, v);
       } else {
         const int r1 = nr - 1;
         const uint8_t* const q[2] = {q0, q0 + r1 * p.qi};
-        const uint32_t* const sb[2] = {s0, s0 + r1 * sw};
+        const uint32_t* const sb[2] = {sp, sp + r1 * sw};
         float v2[2] = {0.f, 0.f};
         dotr<2>(q, sb, hsl, hsm, nch, v2);
         v[0] = v2[0];
         v[1] = v2[1];
       }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) v[k] = warp_sum(v[k]);
-      if (lane < nr) ob[s * n + j0 + lane] = lane == 0 ? v[0] : lane == 1 ? v[1] : lane == 2 ? v[2] : v[3];
+      for (int k = 0; k < 4; ++k) acc[k] = fmaf(ws, v[k], acc[k]);
     }
+    if (cg >= 0) flush(min(nslots, c1 - cg * nslots));
+  }
+
+  // Consume a down item (rows [ja, ja+n) of every slot): the weighted contributions
+  // are gathered in shared memory over the activations x (no longer read in this
+  // phase), then y = resid + their sum in slot order, rounded once.  Called by every
+  // thread; returns false for all on an abort.
+  __device__ bool down_item(uint32_t item, uint32_t off, int ja, int n, const float* hs, const float2* hsum,
+                            const uint16_t* resid_t, uint16_t* y_t) {
+    const uint32_t lead = static_cast<uint32_t>((p.o_d_sb + static_cast<unsigned long long>(ja) * p.si) & 15ull);
+    float* ob = xs;  // [nslots][n]
+    // the residual of the item's rows, loaded before the dot products (one coalesced
+    // load; in a stack block y is the residual buffer itself, rows of this block only)
+    const float rj = threadIdx.x < n ? bf16_to_f32(resid_t[ja + threadIdx.x]) : 0.f;
+    const bool ok = wait_item(item);
+    if (!ok) hdr->abort_flag = 1;
+    if (ok) down_cells(off, n, hs, hsum, lead, ob);
     __syncthreads();
     if (hdr->abort_flag) return false;
     if (threadIdx.x < n) {
       const int j = threadIdx.x;
       float pa = 0.f;
-      for (int s = 0; s < nslots; ++s) pa = fmaf(hdr->wsl[s], ob[s * n + j], pa);
+      for (int sl = 0; sl < nslots; ++sl) pa += ob[sl * n + j];
       y_t[ja + j] = f32_to_bf16(rj + pa);
     }
     __syncthreads();
@@ -703,9 +762,8 @@ struct LayerKernel {
   // sum of exact fp32 x bf16 products, lanes striding the split; the splits' sums are
   // added in split order (the batched router's order too, so both give the same bits)
   // and published for every block to read.
-  __device__ bool phase1_consume(int buf, bool route) {
+  __device__ bool phase1_consume(bool route) {
     if (route) {
-      const int rows = p.E + (p.has_shared ? 1 : 0);
       const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
       const int hc = p.H / p.nq;
       const uint32_t rib = g.router_item();
@@ -736,7 +794,7 @@ struct LayerKernel {
         if (lane == 0) rpart[u] = acc;
       }
       __syncthreads();
-      double* logits = p.logits + static_cast<size_t>(buf) * rows;
+      const uint32_t tag = tag32(tok_);
       for (int i = threadIdx.x; i < row1_ - row0_; i += kThreads) {
         const double* rp = rpart + i * p.nq;
         double l;
@@ -746,7 +804,9 @@ struct LayerKernel {
           l = 0.0;
           for (int q = 0; q < p.nq; ++q) l += rp[q];
         }
-        logits[row0_ + i] = l;
+        const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(l));
+        st_relaxed_v2_u64(p.lx + 2 * (row0_ + i), tagged(static_cast<uint32_t>(bits >> 32), tag),
+                          tagged(static_cast<uint32_t>(bits), tag));
       }
     }
     __syncthreads();
@@ -759,35 +819,100 @@ struct LayerKernel {
   // descending with ties to the lower index (compared through the order-preserving
   // 64-bit key of each fp64 logit), then the renormalised softmax weights of the K
   // and the shared sigmoid gate.
-  __device__ void topk(int buf, int t) {
+  __device__ void topk(int t) {
     mark(3);
-    if (!wait_all(p.rflags, t)) {
+    const int rows = p.E + (p.has_shared ? 1 : 0);
+    const int lane = threadIdx.x & 31;
+    const int ngroups = (p.E + 31) >> 5;
+    // candidates of the first level: per group of 32 experts its K best, in rank order
+    unsigned long long* ckey = reinterpret_cast<unsigned long long*>(stage);
+    double* cval = reinterpret_cast<double*>(stage + r128(static_cast<uint32_t>(ngroups * p.K) * 8u));
+    int* cidx = reinterpret_cast<int*>(stage + 2 * r128(static_cast<uint32_t>(ngroups * p.K) * 8u));
+    // every thread polls the logits it ranks (all of its loads in flight together) and
+    // ranks each within its warp's group of 32 consecutive experts by shuffles
+    const uint32_t want = tag32(t);
+    bool ok = true;
+    for (int e0 = 0; e0 < rows; e0 += 2 * kThreads) {  // block-uniform trip count
+      ulonglong2 v[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = e0 + static_cast<int>(threadIdx.x) + k * kThreads;
+        v[k] = e < rows ? ld_volatile_v2_u64(p.lx + 2 * e) : make_ulonglong2(tagged(0u, want), tagged(0u, want));
+      }
+      {  // every retry re-reads all logits still missing, their loads in flight together
+        uint64_t t0 = 0;
+        int it = 0;
+        while (ok && !(has_tag(v[0].x, want) && has_tag(v[0].y, want) && has_tag(v[1].x, want) &&
+                       has_tag(v[1].y, want))) {
+          if (!poll_tick(t0, it)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int e = e0 + static_cast<int>(threadIdx.x) + k * kThreads;
+            if (!(has_tag(v[k].x, want) && has_tag(v[k].y, want))) v[k] = ld_volatile_v2_u64(p.lx + 2 * e);
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = e0 + static_cast<int>(threadIdx.x) + k * kThreads;
+        double l = __longlong_as_double(static_cast<long long>((v[k].x << 32) | (v[k].y & 0xFFFFFFFFull)));
+        if (e < p.E && p.has_rbias) l += static_cast<double>(__ldg(p.rbias + e));
+        if (e == p.E && p.has_shared) hdr->selog[p.K] = l;
+        // experts beyond E take key 0, below every logit's key (and never selected)
+        const unsigned long long key = e < p.E ? dkey(l) : 0ull;
+        if (e - static_cast<int>(lane) < p.E) {  // warp-uniform: the group's first expert exists
+          int rank = 0;
+#pragma unroll 8
+          for (int j = 0; j < 32; ++j) {
+            const unsigned long long kj = __shfl_sync(0xffffffffu, key, j);
+            rank += static_cast<int>(kj > key) | (static_cast<int>(kj == key) & static_cast<int>(j < lane));
+          }
+          if (rank < p.K) {
+            const int slot = (e >> 5) * p.K + rank;
+            ckey[slot] = key;
+            cval[slot] = l;
+            cidx[slot] = e < p.E ? e : 0x7fffffff;
+          }
+        }
+      }
+    }
+    if (__syncthreads_or(!ok)) {
       if (threadIdx.x == 0) hdr->abort_flag = 1;
       __syncthreads();
       return;
     }
     mark(10);
-    const int rows = p.E + (p.has_shared ? 1 : 0);
-    double* slog = reinterpret_cast<double*>(stage);
-    unsigned long long* skey = reinterpret_cast<unsigned long long*>(stage + r128(static_cast<uint32_t>(rows) * 8u));
-    unsigned long long* ckey = skey + ((p.E + 15) & ~15);
-    int* cidx = reinterpret_cast<int*>(ckey + ((p.E + 31) >> 5) * p.K);
-    const double* logits = p.logits + static_cast<size_t>(buf) * rows;
-    for (int e = threadIdx.x; e < rows; e += kThreads) {
-      double l = __ldcg(logits + e);
-      if (e < p.E && p.has_rbias) l += static_cast<double>(__ldg(p.rbias + e));
-      slog[e] = l;
-      if (e < p.E) skey[e] = dkey(l);
+    mark(11);
+    // second level: every candidate's rank among all groups' candidates, counted by
+    // kStripe consecutive lanes (each over every kStripe-th candidate), summed by shuffles
+    constexpr int kStripe = 8;
+    const int ncand = ngroups * p.K;
+    for (int base = 0; base < ncand * kStripe; base += kThreads) {  // block-uniform trip count
+      const int i = base + static_cast<int>(threadIdx.x);
+      const int c = i / kStripe, part = i % kStripe;
+      unsigned long long kc = 0;
+      int ic = 0, rank = 0;
+      if (c < ncand) {
+        kc = ckey[c];
+        ic = cidx[c];
+        for (int j = part; j < ncand; j += kStripe) {
+          const unsigned long long kj = ckey[j];
+          const int ij = cidx[j];
+          rank += static_cast<int>(kj > kc) | (static_cast<int>(kj == kc) & static_cast<int>(ij < ic));
+        }
+      }
+#pragma unroll
+      for (int o = 1; o < kStripe; o <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+      if (c < ncand && part == 0 && kc != 0 && rank < p.K) {
+        hdr->sel[rank] = ic;
+        hdr->selog[rank] = cval[c];
+      }
     }
     __syncthreads();
-    mark(11);
-    rank_topk<kThreads>(skey, ckey, cidx, p.E, p.K, hdr->sel);
     mark(12);
-    // keep the selection's logits: the staging area is about to receive the rows
-    if (threadIdx.x <= p.K)
-      hdr->selog[threadIdx.x] =
-          threadIdx.x < p.K ? slog[hdr->sel[threadIdx.x]] : (p.has_shared ? slog[p.E] : 0.0);
-    __syncthreads();
   }
 
   // Warp 0: the renormalised softmax weights of the selection and the shared sigmoid
@@ -853,11 +978,19 @@ struct LayerKernel {
     pl.doff = gtotal;
     const uint32_t dtotal = g.dn_total(pl.j1 - pl.j0);
     pl.hoff = g.h_bytes() <= pl.doff ? 0u : r128(pl.doff + dtotal);
-    pl.prefetch = (vend >= pl.v1) && (pl.doff + dtotal <= cap) && (pl.hoff + g.h_bytes() <= cap) &&
-                  (gitems + pl.ndown <= kMaxRoundItems);
+    // the shared expert's rows (staged at the end of the staging area in P1) are
+    // consumed while the routed rows fly in: the routed chunks must stop before them
+    uint32_t sc_off = cap;
+    if (p.has_shared) {
+      const int sa = static_cast<int>(static_cast<long long>(p.I) * b / G);
+      const int sb = static_cast<int>(static_cast<long long>(p.I) * (b + 1) / G);
+      if (sb > sa) sc_off = (cap - g.gu_bytes(sb - sa)) & ~127u;
+    }
+    pl.prefetch = (vend >= pl.v1) && (pl.doff <= sc_off) && (pl.doff + dtotal <= cap) &&
+                  (pl.hoff + g.h_bytes() <= cap) && (gitems + pl.ndown <= kMaxRoundItems);
   }
 
-  __device__ bool experts(int buf, bool route, const uint16_t* resid_t, uint16_t* y_t) {
+  __device__ bool experts(bool route, const uint16_t* resid_t, uint16_t* y_t) {
     const ExpertPlan& pl = hdr->plan;
     const int j0 = pl.j0, j1 = pl.j1, ndown = pl.ndown;
     const bool prefetch = pl.prefetch != 0;
@@ -875,34 +1008,46 @@ struct LayerKernel {
       // the down rows are requested once the first half of the gate/up rows has
       // landed (thread 0 consumes none of them): requested together, both streams are
       // served interleaved and the gate/up rows complete late, while the down rows are
-      // needed only after the h exchange.  The copies are issued whatever the wait
-      // returns.
+      // needed only after the h exchange.  They overwrite the shared expert's rows, so
+      // they also wait (bounded) for warps 1-15 to have consumed those.  The copies are
+      // issued whatever the waits return.
       if (threadIdx.x == 0) {
         if (pl.gitems > 0) (void)wait_item(down_first - static_cast<uint32_t>(pl.gitems - (pl.gitems - 1) / 2));
+        if (has_sc_) {
+          const uint64_t t0 = global_timer_ns();
+          while (atomicAdd(&hdr->shared_done, 0) < kWarps - 1 && global_timer_ns() - t0 < p.wait_ns) __nanosleep(64);
+        }
         issue_down_items(j0, j1, 0, ndown, down_first, doff);
       }
-      gu_consume(ch, pl.nc, buf, 1);
+      // warps 1-15: the shared expert's gate/up rows first (in shared memory since P1),
+      // while the first routed rows are in flight
+      if (has_sc_ && threadIdx.x >= 32) {
+        gu_consume(&sc_, 1, 1, 1);
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) atomicAdd(&hdr->shared_done, 1);
+      }
+      gu_consume(ch, pl.nc, 1);
       __syncthreads();
       if (hdr->abort_flag) return false;
     } else {
       if (route) route_weights(tok_);
-      if (!gu_rounds(pl.v0, pl.v1, buf)) return false;
+      if (has_sc_) gu_consume(&sc_, 1, 0, 1);
+      __syncthreads();
+      if (hdr->abort_flag || !gu_rounds(pl.v0, pl.v1)) return false;
     }
-    publish(p.hflags, tok_);
     mark(5);
-    // ---- P3: stage h of every slot, then the down rows
+    // ---- P3: stage h of every slot (polled from every block's tagged words), then the
+    // down rows
     const uint32_t hbase = prefetch ? hoff : 0u;
     float* hs = reinterpret_cast<float*>(stage + hbase);
     const uint32_t hstride = g.padded(p.I);
     float2* hsum = reinterpret_cast<float2*>(hs + static_cast<size_t>(nslots) * hstride);
-    if (!wait_all(p.hflags, tok_)) {
+    if (__syncthreads_or(!stage_h(hs, hstride, hsum))) {
       if (threadIdx.x == 0) hdr->abort_flag = 1;
       __syncthreads();
       return false;
     }
     mark(6);
-    stage_h(p.hbuf + static_cast<size_t>(buf) * (p.K + 1) * p.I, hs, hstride, hsum);
-    __syncthreads();
     mark(7);
     if (prefetch) {
       for (int k = 0; k < ndown; ++k) {
@@ -967,9 +1112,9 @@ struct LayerKernel {
       return;
     }
     for (int t = 0; t < p.T; ++t) {
-      const int buf = t & 1;
       tok_ = t;
       mark(0);
+      if (threadIdx.x == 0) hdr->shared_done = 0;  // first read after the barriers of P1
       if (!route) {
         given_routing(t);
         if (hdr->skip_token) continue;
@@ -985,21 +1130,16 @@ struct LayerKernel {
         drain();
         return;
       }
-      if (!phase1_consume(buf, route)) break;
-      if (route) publish(p.rflags, t);
+      if (!phase1_consume(route)) break;
       mark(2);
-      // the shared expert does not depend on the routing: warps 1-15 consume its
-      // gate/up rows while warp 0 already polls for the router partials (top-K's
-      // scratch and the shared rows occupy disjoint parts of the staging area)
-      if (has_sc_) gu_consume(&sc_, 1, buf, 1);
       if (route) {
-        topk(buf, t);
+        topk(t);
         if (hdr->abort_flag) break;
         if (!do_experts) route_weights(t);  // otherwise computed while the rows fly
         mark(4);
       }
       if (do_experts) {
-        if (!experts(buf, route, p.resid + static_cast<size_t>(t) * p.H, p.y + static_cast<size_t>(t) * p.H))
+        if (!experts(route, p.resid + static_cast<size_t>(t) * p.H, p.y + static_cast<size_t>(t) * p.H))
           break;
         mark(9);
       }
