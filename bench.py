@@ -533,6 +533,70 @@ def bench_layer(args, world, rank, config):
             "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms), "max": max(step_ms)}}
 
 
+def bench_tier(args, rank, slots: int = 64, tokens: int = 200):
+    """The full-size layer with its routed experts in pinned host memory behind an HBM
+    cache of `slots` records: single-token calls, each routing on the GPU, reading the
+    routing back, copying the missing records host -> device and running the experts.
+    Reports tokens/s, the host -> device GB/s of the expert copies and the cache hit
+    rate (rank 0, one GPU)."""
+    import torch
+
+    import fmoe_synth as synth
+    from bit_dequant_expert_softmax_b200 import fmoe
+    from fmoe_synth.torch_layer import make_device_layer, make_device_x
+
+    shape = synth.CONFIGS["layer4096"]["shape"]
+    H, E = shape.hidden, shape.n_experts
+    w = make_device_layer(shape, 0, 0)
+    cfg = fmoe.fmoe_config(H, shape.inter, E, shape.top_k, shape.bits, shape.has_shared, shape.router_bias)
+    rb = fmoe.fmoe_record_bytes(H, shape.inter, shape.bits)
+    host = w.experts[:E * rb].cpu().pin_memory()
+    shared = w.experts[E * rb:(E + 1) * rb].clone()
+    router, rbias, gs = w.router, w.router_bias, w.shared_gate
+    del w
+    torch.cuda.empty_cache()
+    tier = fmoe.Tier(cfg, host, shared, router, rbias, gs, slots, 1)
+    x = make_device_x(0, 0, tokens, H)
+    y = torch.empty_like(x)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for t in range(min(32, tokens)):  # warm the cache and the kernels
+            tier.forward(x[t:t + 1], y=y[t:t + 1], stream=stream)
+    torch.cuda.synchronize()
+    s0 = tier.stats()
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for t in range(tokens):
+            tier.forward(x[t:t + 1], y=y[t:t + 1], stream=stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = a.elapsed_time(b)
+    s1 = tier.stats()
+    err = tier.error()
+    tier.close()
+    del tier, host, shared, x, y
+    torch.cuda.empty_cache()
+    if err:
+        raise RuntimeError(f"device-side error bits {err:#x} in the tier benchmark")
+    hits, misses = s1["hits"] - s0["hits"], s1["misses"] - s0["misses"]
+    if rank != 0:
+        return None
+    return {"metric": "host-memory expert tier: MoE-layer decode tokens/s", "value": tokens / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": 1, "warmup": 32, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"layer4096 with its {E} routed expert records in pinned host memory, "
+                                   f"an HBM cache of {slots} records (LRU), {tokens} single-token calls",
+                       "tokens_per_step": tokens},
+            "tier": {"h2d_gbs": round((s1["bytes_h2d"] - s0["bytes_h2d"]) / (ms / 1e3) / 1e9, 2),
+                     "hit_rate": round(hits / max(1, hits + misses), 4), "hits": hits, "misses": misses,
+                     "record_bytes": rb},
+            "gpu_launches": 2 * tokens, "clocks": clocks}
+
+
 SUB_CONFIGS = ("stack24_4bit", "stack60_2bit", "stack16_batched")
 
 
@@ -566,6 +630,7 @@ def main():
         if world == 1 and args.config == "layer4096" and not args.no_sub and args.tokens is None:
             line["sub_records"] = [bench_stack(args, world, rank, c, args.sub_steps, 3,
                                                0 if args.no_cpu_baseline else 2) for c in SUB_CONFIGS]
+            line["sub_records"].append(bench_tier(args, rank))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

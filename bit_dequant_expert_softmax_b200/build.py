@@ -8,6 +8,7 @@ ROOT = os.path.dirname(HERE)
 SO = os.path.join(HERE, "libfmoe.so")
 CSRC = os.path.join(HERE, "csrc")
 MAIN = os.path.join(CSRC, "fmoe_api.cu")
+TIER = os.path.join(CSRC, "fmoe_tier.cpp")  # host-memory expert tier (host code on the C ABI)
 
 # -ftz=false is explicit: the single-token dot products read 4-/2-bit codes masked in
 # place as subnormal floats (code * 2^(s - 149)); flushing subnormals to zero would turn
@@ -35,7 +36,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if os.path.getmtime(SO) >= newest:
             return SO
     check_flags(NVCC_FLAGS)
-    cmd = ["nvcc", *NVCC_FLAGS, MAIN, "-o", SO]
+    cmd = ["nvcc", *NVCC_FLAGS, MAIN, TIER, "-o", SO]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)

@@ -53,14 +53,15 @@ int router_splits(int H) {
 }
 
 // Single-token workspace: the error word, the token counter (the tag base of the
-// exchanges), the router logits and the h values as tagged 64-bit words.
+// exchanges), the router logits and the h values as tagged 64-bit words, two buffers
+// of each (token parity).
 WsLayout ws_layout(const fmoe_config& c) {
   WsLayout w;
   w.err = 0;
   w.tokens = 128;
   w.lx = 256;
-  w.hx = al256(w.lx + (size_t)(c.n_experts + 1) * 2 * sizeof(uint64_t));
-  w.size = al256(w.hx + (size_t)(c.top_k + 1) * c.inter * sizeof(uint64_t));
+  w.hx = al256(w.lx + 2 * (size_t)(c.n_experts + 1) * 2 * sizeof(uint64_t));
+  w.size = al256(w.hx + 2 * (size_t)(c.top_k + 1) * c.inter * sizeof(uint64_t));
   return w;
 }
 

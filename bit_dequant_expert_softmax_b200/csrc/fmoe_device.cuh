@@ -101,6 +101,14 @@ __device__ __forceinline__ ulonglong2 ld_volatile_v2_u64(const unsigned long lon
   return v;
 }
 
+// 16-byte load of two 64-bit words, each read single-copy atomically at GPU scope
+// (served by L2).
+__device__ __forceinline__ ulonglong2 ld_relaxed_v2_u64(const unsigned long long* p) {
+  ulonglong2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
+  return v;
+}
+
 // 16-byte store of two 64-bit words, each written single-copy atomically.
 __device__ __forceinline__ void st_relaxed_v2_u64(unsigned long long* p, unsigned long long a, unsigned long long b) {
   asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(a), "l"(b) : "memory");

@@ -208,30 +208,36 @@ struct LayerKernel {
   // ---------------------------------------------------------------- exchanges
   // Values every block needs from all others (router logits, h rows) travel as 64-bit
   // words carrying the token's tag in their high half (fmoe::tagged).  Each word is
-  // written and read single-copy atomically (relaxed stores, volatile loads served by
-  // L2), so a reader polls the very words it needs until they carry its token's tag:
-  // no flags, no fences, no second read.  One buffer serves every token: a block
-  // overwrites its words with the next token's only after every block has read this
-  // token's (the next token's values need every block's values of this one).  Every
-  // wait is bounded by the layer's time limit.
+  // written and read single-copy atomically (relaxed stores and loads at GPU scope,
+  // served by L2), so a reader polls the very words it needs until they carry its token's tag:
+  // no flags and no second read (the writers only fence once after their last words,
+  // so that the stores are performed at once).  The buffers alternate by token parity: a
+  // block writes token t+2's words only after every block has written token t+1's,
+  // which each does after it has read token t's.  Polls back off (64 ns doubling to
+  // about 1 us between retries, so that waiting blocks do not flood L2) and are
+  // bounded by the layer's time limit.
   uint32_t tbase_;
   __device__ __forceinline__ uint32_t tag32(int t) const {
     return (tbase_ + static_cast<uint32_t>(t)) % 0xFFFFFFFFu + 1u;
   }
+  __device__ __forceinline__ unsigned long long* lx_of(int t) const {
+    return p.lx + static_cast<size_t>(t & 1) * 2 * (p.E + 1);
+  }
+  __device__ __forceinline__ unsigned long long* hx_of(int t) const {
+    return p.hx + static_cast<size_t>(t & 1) * (p.K + 1) * p.I;
+  }
 
-  // One step of a bounded poll: sleeps briefly; false (error bit set) once the limit
-  // has passed or another thread has given up already.
+  // One step of a bounded poll: sleeps (backing off); false (error bit set) once the
+  // limit has passed.
   __device__ __forceinline__ bool poll_tick(uint64_t& t0, int& it) const {
-    if ((++it & 15) == 0) {
-      const uint64_t now = global_timer_ns();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > p.wait_ns || (ld_relaxed_u32(p.err) & FMOE_DEVERR_BARRIER_TIMEOUT)) {
-        atomicOr(p.err, FMOE_DEVERR_BARRIER_TIMEOUT);
-        return false;
-      }
+    const uint64_t now = global_timer_ns();
+    if (it == 0) t0 = now;
+    if (now - t0 > p.wait_ns) {
+      atomicOr(p.err, FMOE_DEVERR_BARRIER_TIMEOUT);
+      return false;
     }
-    __nanosleep(32);
+    __nanosleep(64u << min(it, 4));
+    ++it;
     return true;
   }
 
@@ -293,6 +299,7 @@ struct LayerKernel {
 #pragma unroll
         for (int k = 0; k < 2; ++k) nat[k] = normed(nat[k], rn);
       }
+      if (base == 0 && (nat[0].x | nat[1].y | 1u)) mark(14);
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
@@ -331,7 +338,7 @@ struct LayerKernel {
     const int per_slot = p.I / 4, nch = p.I / C::kCols;
     const int n4 = nslots * per_slot;
     const uint32_t want = tag32(tok_);
-    const unsigned long long* src = p.hx;
+    const unsigned long long* src = hx_of(tok_);
     bool ok = true;
     for (int base = 0; base < n4; base += 4 * kThreads) {  // block-uniform trip count
       ulonglong2 a[4], b[4];
@@ -339,8 +346,8 @@ struct LayerKernel {
       for (int k = 0; k < 4; ++k) {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
         if (q < n4) {
-          a[k] = ld_volatile_v2_u64(src + 4 * q);
-          b[k] = ld_volatile_v2_u64(src + 4 * q + 2);
+          a[k] = ld_relaxed_v2_u64(src + 4 * q);
+          b[k] = ld_relaxed_v2_u64(src + 4 * q + 2);
         } else {
           a[k] = b[k] = make_ulonglong2(tagged(0u, want), tagged(0u, want));
         }
@@ -361,8 +368,8 @@ struct LayerKernel {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
-          if (!(has_tag(a[k].x, want) && has_tag(a[k].y, want))) a[k] = ld_volatile_v2_u64(src + 4 * q);
-          if (!(has_tag(b[k].x, want) && has_tag(b[k].y, want))) b[k] = ld_volatile_v2_u64(src + 4 * q + 2);
+          if (!(has_tag(a[k].x, want) && has_tag(a[k].y, want))) a[k] = ld_relaxed_v2_u64(src + 4 * q);
+          if (!(has_tag(b[k].x, want) && has_tag(b[k].y, want))) b[k] = ld_relaxed_v2_u64(src + 4 * q + 2);
         }
       }
 #pragma unroll
@@ -389,9 +396,7 @@ struct LayerKernel {
           if (q % TPC == 0) hsum[slot * nch + c0 / C::kCols] = make_float2(sum, chunk_unscale(pre));
         }
       }
-      if (base == 0) mark(14);
     }
-    mark(15);
     return ok;
   }
 
@@ -500,7 +505,7 @@ struct LayerKernel {
         static_cast<uint32_t>((p.o_gu_sb + static_cast<unsigned long long>(c.ra) * 2u * p.sh) & 15ull);
     const uint32_t* sg = reinterpret_cast<const uint32_t*>(stage + c.off + g.gu_q(n) + lead) + i * 2 * (p.sh / 4);
     const int sw = p.sh / 4;
-    unsigned long long* hout = p.hx + static_cast<size_t>(c.slot) * p.I + r;
+    unsigned long long* hout = hx_of(tok_) + static_cast<size_t>(c.slot) * p.I + r;
     const uint32_t tag = tag32(tok_);
     if (np == 2) {
       const uint8_t* const q[4] = {qg, qg + p.qh, qg + 2 * p.qh, qg + 3 * p.qh};
@@ -547,6 +552,7 @@ struct LayerKernel {
       }
       base += nu;
     }
+    __threadfence();  // push the h words out now: every block will wait for them
   }
 
   // Gate/up of routed units [v0, v1) (unit = slot*I + r) in rounds that fit the
@@ -698,6 +704,7 @@ struct LayerKernel {
     // load; in a stack block y is the residual buffer itself, rows of this block only)
     const float rj = threadIdx.x < n ? bf16_to_f32(resid_t[ja + threadIdx.x]) : 0.f;
     const bool ok = wait_item(item);
+    mark(15);
     if (!ok) hdr->abort_flag = 1;
     if (ok) down_cells(off, n, hs, hsum, lead, ob);
     __syncthreads();
@@ -805,8 +812,9 @@ struct LayerKernel {
           for (int q = 0; q < p.nq; ++q) l += rp[q];
         }
         const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(l));
-        st_relaxed_v2_u64(p.lx + 2 * (row0_ + i), tagged(static_cast<uint32_t>(bits >> 32), tag),
+        st_relaxed_v2_u64(lx_of(tok_) + 2 * (row0_ + i), tagged(static_cast<uint32_t>(bits >> 32), tag),
                           tagged(static_cast<uint32_t>(bits), tag));
+        __threadfence();  // push the words out now: every block is about to wait for them
       }
     }
     __syncthreads();
@@ -831,13 +839,14 @@ struct LayerKernel {
     // every thread polls the logits it ranks (all of its loads in flight together) and
     // ranks each within its warp's group of 32 consecutive experts by shuffles
     const uint32_t want = tag32(t);
+    const unsigned long long* lx = lx_of(t);
     bool ok = true;
     for (int e0 = 0; e0 < rows; e0 += 2 * kThreads) {  // block-uniform trip count
       ulonglong2 v[2];
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int e = e0 + static_cast<int>(threadIdx.x) + k * kThreads;
-        v[k] = e < rows ? ld_volatile_v2_u64(p.lx + 2 * e) : make_ulonglong2(tagged(0u, want), tagged(0u, want));
+        v[k] = e < rows ? ld_relaxed_v2_u64(lx + 2 * e) : make_ulonglong2(tagged(0u, want), tagged(0u, want));
       }
       {  // every retry re-reads all logits still missing, their loads in flight together
         uint64_t t0 = 0;
@@ -851,7 +860,7 @@ struct LayerKernel {
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
             const int e = e0 + static_cast<int>(threadIdx.x) + k * kThreads;
-            if (!(has_tag(v[k].x, want) && has_tag(v[k].y, want))) v[k] = ld_volatile_v2_u64(p.lx + 2 * e);
+            if (!(has_tag(v[k].x, want) && has_tag(v[k].y, want))) v[k] = ld_relaxed_v2_u64(lx + 2 * e);
           }
         }
       }

@@ -31,7 +31,9 @@ EXPORTS = ["fmoe_record_bytes", "fmoe_workspace_bytes", "fmoe_layer_create", "fm
            "fmoe_layer_forward_noalloc", "fmoe_status_string", "fmoe_block_forward", "fmoe_stack_create",
            "fmoe_stack_destroy", "fmoe_stack_forward", "fmoe_stack_graph_create", "fmoe_graph_launch",
            "fmoe_graph_destroy", "fmoe_batch_workspace_bytes", "fmoe_layer_set_batch_workspace",
-           "fmoe_route_batched", "fmoe_layer_forward_batched", "fmoe_block_forward_batched"]
+           "fmoe_route_batched", "fmoe_layer_forward_batched", "fmoe_block_forward_batched",
+           "fmoe_tier_buffer_bytes", "fmoe_tier_create", "fmoe_tier_forward", "fmoe_tier_stats",
+           "fmoe_tier_get_error", "fmoe_tier_destroy"]
 
 
 class FmoeError(RuntimeError):
@@ -93,6 +95,14 @@ def lib():
         L.fmoe_layer_debug_timeline.argtypes = [vp, vp, i32]
         L.fmoe_layer_grid_size.argtypes = [vp]
         L.fmoe_layer_grid_size.restype = i32
+        L.fmoe_tier_buffer_bytes.restype = sz
+        L.fmoe_tier_buffer_bytes.argtypes = [ctypes.POINTER(fmoe_config), i32, i32]
+        L.fmoe_tier_create.argtypes = [ctypes.POINTER(fmoe_config), vp, vp, vp, vp, vp, vp, sz, i32, i32,
+                                       ctypes.POINTER(vp)]
+        L.fmoe_tier_forward.argtypes = [vp, vp, vp, i32, vp, vp]
+        L.fmoe_tier_stats.argtypes = [vp, ctypes.POINTER(u64), ctypes.POINTER(u64), ctypes.POINTER(u64)]
+        L.fmoe_tier_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.fmoe_tier_destroy.argtypes = [vp]
         L.fmoe_status_string.argtypes = [i32]
         L.fmoe_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -336,6 +346,57 @@ class Layer:
     def close(self):
         if self.handle:
             fmoe_layer_destroy(self.handle)
+            self.handle = 0
+
+
+def fmoe_tier_buffer_bytes(cfg: fmoe_config, slots: int, max_tokens: int) -> int:
+    return lib().fmoe_tier_buffer_bytes(ctypes.byref(cfg), slots, max_tokens)
+
+
+class Tier:
+    """A layer whose routed experts live in host memory behind an HBM cache of `slots`
+    records (see include/fmoe.h).  Keeps the host records, the device buffer and the
+    router tensors alive."""
+
+    def __init__(self, cfg: fmoe_config, host_experts, shared_record, router, router_bias, shared_gate,
+                 slots: int, max_tokens: int = 1):
+        import torch
+        self.cfg = cfg
+        self.keep = (host_experts, shared_record, router, router_bias, shared_gate)
+        n = fmoe_tier_buffer_bytes(cfg, slots, max_tokens)
+        if n == 0:
+            raise FmoeError(1, "fmoe_tier_buffer_bytes")
+        self.buf = torch.empty(n, dtype=torch.uint8, device=router.device)
+        h = ctypes.c_void_p()
+        _check(lib().fmoe_tier_create(ctypes.byref(cfg), _ptr(host_experts), _ptr(shared_record), _ptr(router),
+                                      _ptr(router_bias), _ptr(shared_gate), self.buf.data_ptr(), n, slots,
+                                      max_tokens, ctypes.byref(h)), "fmoe_tier_create")
+        self.handle = h.value
+
+    def forward(self, x, resid=None, y=None, stream=None):
+        import torch
+        resid = x if resid is None else resid
+        y = torch.empty_like(x) if y is None else y
+        _check(lib().fmoe_tier_forward(self.handle, _ptr(x), _ptr(resid), x.shape[0], _ptr(y), _stream(stream)),
+               "fmoe_tier_forward")
+        return y
+
+    def stats(self):
+        a, b, c = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
+        _check(lib().fmoe_tier_stats(self.handle, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+               "fmoe_tier_stats")
+        return {"hits": a.value, "misses": b.value, "bytes_h2d": c.value}
+
+    def error(self) -> int:
+        e = ctypes.c_uint32(0)
+        st = lib().fmoe_tier_get_error(self.handle, ctypes.byref(e))
+        if st not in (0, 5):
+            raise FmoeError(st, "fmoe_tier_get_error")
+        return e.value
+
+    def close(self):
+        if self.handle:
+            lib().fmoe_tier_destroy(self.handle)
             self.handle = 0
 
 

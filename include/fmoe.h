@@ -269,11 +269,61 @@ fmoe_status fmoe_layer_debug_hold_block(fmoe_layer_t layer, int cta);
  * done, 5 gate/up done, 6 h rows of all blocks visible, 7 h staged, 8 down rows done,
  * 9 token done, 10 router logits of all blocks visible, 11 expert ranks start, 12 expert
  * ranks done, 13 the launch's start (token 0 only, before the wait for the previous
- * grid), 14 first batch of h loaded, 15 h loaded.  NULL (default) disables it. */
+ * grid), 14 the activations' loads returned, 15 the first down rows landed.  NULL
+ * (default) disables it. */
 fmoe_status fmoe_layer_debug_timeline(fmoe_layer_t layer, uint64_t* dev_buf, int token);
 
 /* Number of thread blocks one forward launch uses (one per SM of the device). */
 int fmoe_layer_grid_size(fmoe_layer_t layer);
+
+/* ---- Host-memory expert tier ------------------------------------------------------
+ * A layer whose routed experts do not all stay in HBM: their records live in host
+ * memory and a cache of `slots` records in HBM holds the experts used most recently
+ * (least recently used evicted).  The Flash-MoE pages keep the experts on SSD and read
+ * the selected ones per token (hotdry.top "SSD流式加载": parallel pread of the K
+ * experts, the OS page cache as the only cache); here the slow tier is host memory
+ * over the host link and the cache is explicit, in HBM.
+ *
+ * Per call (T tokens): the routing runs on the GPU (router in HBM, as fmoe_route), the
+ * indices come back to the host, every expert not in the cache is copied host -> device
+ * into a free or least-recently-used slot, and the experts run on the cache with the
+ * routing remapped to slots (as fmoe_expert_forward).  The outputs equal
+ * fmoe_layer_forward's bit for bit (the same kernels on byte-identical records).
+ *
+ * Ownership: host_experts (E routed records, format as fmoe_weights.experts) is
+ * caller-owned host memory, pinned (cudaHostRegister or cudaMallocHost) for
+ * asynchronous copies; the router, its bias and the shared gate are device memory;
+ * dev_buf is a caller-owned device buffer of fmoe_tier_buffer_bytes() bytes (256-byte
+ * aligned) holding the cache, the shared expert's record (copied in at creation from
+ * `shared_record`, a device or host pointer to one record) and the workspaces.  The
+ * tier keeps pointers, not copies.  Calls on one tier must be serialised by the
+ * caller.  Errors: INVALID_ARG, UNSUPPORTED (slots < top_k * max_tokens, or shapes the
+ * kernels cannot hold), CUDA. */
+typedef struct fmoe_tier* fmoe_tier_t;
+
+/* Device bytes of a tier's buffer (cache of `slots` records, the shared record, the
+ * two layers' workspaces and the routing buffers for max_tokens tokens); 0 if invalid. */
+size_t fmoe_tier_buffer_bytes(const fmoe_config* cfg, int slots, int max_tokens);
+
+fmoe_status fmoe_tier_create(const fmoe_config* cfg, const void* host_experts, const void* shared_record,
+                             const float* router, const float* router_bias, const float* shared_gate,
+                             void* dev_buf, size_t buf_bytes, int slots, int max_tokens, fmoe_tier_t* out);
+
+/* y = resid + sum_k w_k o_k(x) + sigma o_s(x) for T <= max_tokens tokens, as
+ * fmoe_layer_forward.  Synchronises `stream` once (the routing is read back to place
+ * the experts); the expert copies and the expert kernel are then enqueued on `stream`. */
+fmoe_status fmoe_tier_forward(fmoe_tier_t tier, const uint16_t* x, const uint16_t* resid, int T, uint16_t* y,
+                              void* stream);
+
+/* Counters since creation: expert lookups that hit the cache, those that missed (each
+ * miss copies one record host -> device) and the bytes copied. */
+fmoe_status fmoe_tier_stats(fmoe_tier_t tier, uint64_t* hits, uint64_t* misses, uint64_t* bytes_h2d);
+
+/* Device error bits of the tier's two layers (as fmoe_layer_get_error). */
+fmoe_status fmoe_tier_get_error(fmoe_tier_t tier, uint32_t* device_error);
+
+/* Releases the tier (host memory only).  NULL is accepted. */
+fmoe_status fmoe_tier_destroy(fmoe_tier_t tier);
 
 /* Size in bytes of the fixed device scratch array of fmoe_layer_forward_noalloc. */
 #define FMOE_NOALLOC_SCRATCH_BYTES (128 * 1024)

@@ -26,7 +26,7 @@ def _declared():
 
 def test_exports_every_declared_symbol(lib):
     names = _declared()
-    assert len(names) == 28
+    assert len(names) == 34
     L = lib.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -142,3 +142,21 @@ def test_build_keeps_subnormals():
     for bad in ("--use_fast_math", "-ftz=true"):
         with pytest.raises(ValueError):
             b.check_flags(b.NVCC_FLAGS + [bad])
+
+
+def test_tier_buffer_bytes_and_host_checks(lib):
+    """The host-memory tier's buffer size (cache of `slots` records, the shared record,
+    two workspaces, routing buffers) and its argument checks, without a device."""
+    cfg = lib.fmoe_config(512, 128, 32, 4, 4, 1, 0)
+    rb = lib.fmoe_record_bytes(512, 128, 4)
+    n8 = lib.fmoe_tier_buffer_bytes(cfg, 8, 1)
+    n16 = lib.fmoe_tier_buffer_bytes(cfg, 16, 1)
+    assert n8 > 9 * rb and 8 * rb <= n16 - n8 <= 8 * rb + 4096  # the cache layer's workspace grows a little
+    assert lib.fmoe_tier_buffer_bytes(cfg, 0, 1) == 0
+    assert lib.fmoe_tier_buffer_bytes(cfg, 33, 1) == 0   # more slots than experts
+    assert lib.fmoe_tier_buffer_bytes(cfg, 8, 0) == 0
+    L = lib.lib()
+    h = ctypes.c_void_p()
+    # NULL host records, NULL buffer: rejected before any device call
+    assert L.fmoe_tier_create(ctypes.byref(cfg), None, None, None, None, None, None, n8, 8, 1, ctypes.byref(h)) == 1
+    assert L.fmoe_tier_destroy(None) == 0
