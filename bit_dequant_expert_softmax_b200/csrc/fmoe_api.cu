@@ -42,7 +42,7 @@ bool record_layout(int H, int I, int bits, RecordLayout* L) {
 }
 
 struct WsLayout {
-  size_t err, tokens, lx, hx, size;
+  size_t err, tokens, rflags, hflags, lpart, hbuf, size;
 };
 
 int router_splits(int H) {
@@ -52,16 +52,17 @@ int router_splits(int H) {
   return nq;
 }
 
-// Single-token workspace: the error word, the token counter (the tag base of the
-// exchanges), the router logits and the h values as tagged 64-bit words, two buffers
-// of each (token parity).
 WsLayout ws_layout(const fmoe_config& c) {
   WsLayout w;
+  const int nq = router_splits(c.hidden);
+  const size_t flag_bytes = (size_t)kMaxGrid * kFlagStride * sizeof(uint32_t);
   w.err = 0;
   w.tokens = 128;
-  w.lx = 256;
-  w.hx = al256(w.lx + 2 * (size_t)(c.n_experts + 1) * 2 * sizeof(uint64_t));
-  w.size = al256(w.hx + 2 * (size_t)(c.top_k + 1) * c.inter * sizeof(uint64_t));
+  w.rflags = 256;
+  w.hflags = w.rflags + flag_bytes;
+  w.lpart = w.hflags + flag_bytes;
+  w.hbuf = al256(w.lpart + 2 * (size_t)(c.n_experts + 1) * nq * sizeof(double));
+  w.size = al256(w.hbuf + 2 * (size_t)(c.top_k + 1) * c.inter * sizeof(float));
   return w;
 }
 
@@ -178,19 +179,18 @@ fmoe_status plan(fmoe_layer* L) {
   if (fixed >= (uint32_t)kMaxSmem) return FMOE_ERR_UNSUPPORTED;
   const uint32_t staging = (uint32_t)kMaxSmem - fixed;
   const int G = L->sms;
-  // P1: x in doubles, the block's whole router rows and their split sums from the
-  // start of the staging area, its shared gate/up rows at the end (both in flight
-  // together); the shared rows are consumed while top-K starts, so its logits and
-  // candidates must not reach them either
-  const uint32_t rows_max = (uint32_t)((c.n_experts + c.has_shared + G - 1) / G);
+  // P1: x in doubles and the router rows a block touches from the start of the
+  // staging area, its shared gate/up rows at the end (both in flight together); the
+  // shared rows are consumed while top-K starts, so its logits and candidates must
+  // not reach them either
+  const long long U = (long long)(c.n_experts + c.has_shared) * L->nq;
+  const uint32_t rows_touched = (uint32_t)(((U + G - 1) / G + L->nq - 1) / L->nq + 1);
   const int shared_rows = (c.inter + G - 1) / G;
   const uint32_t sc_off = c.has_shared ? ((staging - g.gu_bytes(shared_rows)) & ~127u) : staging;
-  const uint64_t p1 = (uint64_t)r128(r128((uint32_t)c.hidden * 8u) + rows_max * g.router_item()) +
-                      (uint64_t)rows_max * L->nq * 8u;
-  const uint32_t p1_items = rows_max + (c.has_shared ? (uint32_t)g.gu_items(shared_rows) : 0u);
+  const uint64_t p1 = r128((uint32_t)c.hidden * 8u) + (uint64_t)rows_touched * g.router_item();
+  const uint32_t p1_items = rows_touched + (c.has_shared ? (uint32_t)g.gu_items(shared_rows) : 0u);
   if (c.has_shared && g.gu_bytes(shared_rows) >= staging) return FMOE_ERR_UNSUPPORTED;
   if (p1 > sc_off || p1_items > (uint32_t)kMaxRoundItems) return FMOE_ERR_UNSUPPORTED;
-  // top-K: the candidates of the groups of 32 experts (keys, logits, indices)
   const uint32_t ncand = (uint32_t)((c.n_experts + 31) / 32 * c.top_k);
   if ((uint64_t)2 * r128(ncand * 8u) + (uint64_t)ncand * 4u > sc_off) return FMOE_ERR_UNSUPPORTED;
   // P2: at least one gate/up row pair per round
@@ -198,8 +198,6 @@ fmoe_status plan(fmoe_layer* L) {
   // P3: h of every slot plus one down item; shrink the down item until it fits
   int db = kMaxDownBlock;
   while (db > 1 && (uint64_t)g.h_bytes() + g.dn_item(db) > staging) --db;
-  // the down rows' results of every slot are gathered over the activations x
-  while (db > 1 && (uint64_t)nslots * db > g.padded(c.hidden)) --db;
   if ((uint64_t)g.h_bytes() + g.dn_item(db) > staging) return FMOE_ERR_UNSUPPORTED;
   L->db = db;
   L->staging_bytes = (int)staging;
@@ -212,8 +210,10 @@ fmoe_status plan(fmoe_layer* L) {
 void set_workspace_ptrs(Params& p, const WsLayout& w, uint8_t* ws) {
   p.err = reinterpret_cast<uint32_t*>(ws + w.err);
   p.tokens = reinterpret_cast<uint32_t*>(ws + w.tokens);
-  p.lx = reinterpret_cast<unsigned long long*>(ws + w.lx);
-  p.hx = reinterpret_cast<unsigned long long*>(ws + w.hx);
+  p.rflags = reinterpret_cast<uint32_t*>(ws + w.rflags);
+  p.hflags = reinterpret_cast<uint32_t*>(ws + w.hflags);
+  p.lpart = reinterpret_cast<double*>(ws + w.lpart);
+  p.hbuf = reinterpret_cast<float*>(ws + w.hbuf);
 }
 
 Params base_params(const fmoe_layer* L, int mode, int T) {
@@ -459,7 +459,7 @@ fmoe_status noalloc_get_error(const fmoe_layer* L, uint32_t* device_error) {
   if (cudaMemcpy(&e, ws + L->wsl.err, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return FMOE_ERR_CUDA;
   *device_error = e;
   if (e == 0) return FMOE_OK;
-  if (cudaMemset(ws, 0, L->wsl.size) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
+  if (cudaMemset(ws, 0, L->wsl.lpart) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
   return FMOE_ERR_DEVICE;
 }
 
@@ -866,9 +866,9 @@ fmoe_status fmoe_layer_forward_noalloc(fmoe_layer_t L, const uint16_t* x, const 
   fmoe_status st = noalloc_scratch(dev, &scratch);
   if (st != FMOE_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(scratch);
-  // every call starts from a clean error word, token counter and exchange words (a
-  // word another layer's call left with the same tag would be taken for this call's)
-  if (cudaMemsetAsync(ws, 0, L->wsl.size, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FMOE_ERR_CUDA;
+  // every call starts from a clean error word, tag base and flags (the values the
+  // previous call left there would otherwise be mistaken for this call's)
+  if (cudaMemsetAsync(ws, 0, L->wsl.lpart, static_cast<cudaStream_t>(stream)) != cudaSuccess) return FMOE_ERR_CUDA;
   Params p = base_params(L, MODE_FULL, T);
   set_workspace_ptrs(p, L->wsl, ws);
   p.x = x;

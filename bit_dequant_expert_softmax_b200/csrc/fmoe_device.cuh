@@ -101,29 +101,6 @@ __device__ __forceinline__ ulonglong2 ld_volatile_v2_u64(const unsigned long lon
   return v;
 }
 
-// 16-byte load of two 64-bit words, each read single-copy atomically at GPU scope
-// (served by L2).
-__device__ __forceinline__ ulonglong2 ld_relaxed_v2_u64(const unsigned long long* p) {
-  ulonglong2 v;
-  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
-  return v;
-}
-
-// 16-byte store of two 64-bit words, each written single-copy atomically.
-__device__ __forceinline__ void st_relaxed_v2_u64(unsigned long long* p, unsigned long long a, unsigned long long b) {
-  asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(a), "l"(b) : "memory");
-}
-
-// Values exchanged between blocks travel with the token's 32-bit tag in the same
-// single-copy-atomic 64-bit word (tag in the high half): a reader that sees its
-// token's tag sees that token's value, with no flag, fence or second read.
-__device__ __forceinline__ unsigned long long tagged(uint32_t value, uint32_t tag) {
-  return (static_cast<unsigned long long>(tag) << 32) | value;
-}
-__device__ __forceinline__ bool has_tag(unsigned long long w, uint32_t tag) {
-  return static_cast<uint32_t>(w >> 32) == tag;
-}
-
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -266,55 +243,38 @@ struct Chunk {
     }
   }
 
-  // Word pairs of NR rows against the same activation pairs: float4 k of the chunk
-  // (xv[k * 32]) holds the activations of positions 2k and 2k+1 of both words; every
-  // row's accumulator takes the positions in the same order.
-  template <int K, int NR>
-  __device__ __forceinline__ static void steps(const unsigned long long (&W)[NR], const unsigned long long (&V)[NR],
-                                               const ulonglong2* xv, unsigned long long (&acc)[NR]) {
-    if constexpr (K < kF4PerPair) {
-      const ulonglong2 x = xv[K * 32];
+  // Word pairs of one or two rows against shared activation pairs.
+  template <bool TWO>
+  __device__ __forceinline__ static void word_pair2(unsigned long long Wa, unsigned long long Wb,
+                                                    const ulonglong2* xv, unsigned long long& acc_a,
+                                                    unsigned long long& acc_b) {
+    const unsigned long long Va = Wa >> 8;
+    const unsigned long long Vb = TWO ? (Wb >> 8) : 0ull;
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        pos<2 * K>(W[r], V[r], x.x, acc[r]);
-        pos<2 * K + 1>(W[r], V[r], x.y, acc[r]);
+    for (int k = 0; k < kF4PerPair; ++k) {
+      const ulonglong2 x = xv[k * 32];
+      // positions 2k (x.x) and 2k+1 (x.y)
+      switch (k) {
+#define FMOE_POS_CASE(K)                                  \
+  case K:                                                 \
+    pos<2 * K>(Wa, Va, x.x, acc_a);                       \
+    pos<2 * K + 1>(Wa, Va, x.y, acc_a);                   \
+    if (TWO) pos<2 * K>(Wb, Vb, x.x, acc_b);              \
+    if (TWO) pos<2 * K + 1>(Wb, Vb, x.y, acc_b);          \
+    break;
+        FMOE_POS_CASE(0)
+        FMOE_POS_CASE(1)
+        FMOE_POS_CASE(2)
+        FMOE_POS_CASE(3)
+        FMOE_POS_CASE(4)
+        FMOE_POS_CASE(5)
+        FMOE_POS_CASE(6)
+        FMOE_POS_CASE(7)
+#undef FMOE_POS_CASE
       }
-      steps<K + 1, NR>(W, V, xv, acc);
     }
   }
-
-  template <int NR>
-  __device__ __forceinline__ static void word_pairs(const unsigned long long (&W)[NR], const ulonglong2* xv,
-                                                    unsigned long long (&acc)[NR]) {
-    unsigned long long V[NR];
-#pragma unroll
-    for (int r = 0; r < NR; ++r) V[r] = W[r] >> 8;
-    steps<0, NR>(W, V, xv, acc);
-  }
-
 };
-
-// Sums of four per-lane values over groups of G consecutive lanes (G = 4, 8, 16 or 32,
-// xor shuffles inside the group): value i ends in the lanes whose position p in the
-// group satisfies p / (G / 4) == i (the lane at p = i * G / 4 among them).  Six
-// shuffles for G = 32 instead of twenty.
-template <int G>
-__device__ __forceinline__ float group_sum4(float v0, float v1, float v2, float v3) {
-  const int p = static_cast<int>(threadIdx.x & 31) & (G - 1);
-  const bool hi1 = p & (G / 2);
-  // halves: the lower half of the group keeps values {0, 1}, the upper {2, 3}
-  const float s0 = hi1 ? v0 : v2, s1 = hi1 ? v1 : v3;
-  float k0 = hi1 ? v2 : v0, k1 = hi1 ? v3 : v1;
-  k0 += __shfl_xor_sync(0xffffffffu, s0, G / 2);
-  k1 += __shfl_xor_sync(0xffffffffu, s1, G / 2);
-  // quarters: keep one of the two
-  const bool hi2 = p & (G / 4);
-  float k = hi2 ? k1 : k0;
-  k += __shfl_xor_sync(0xffffffffu, hi2 ? k0 : k1, G / 4);
-#pragma unroll
-  for (int o = G / 8; o > 0; o >>= 1) k += __shfl_xor_sync(0xffffffffu, k, o);
-  return k;
-}
 
 // 2^(P - shift): the pre-scale of an activation met by codes masked at bit `shift`.
 __device__ __forceinline__ float prescale_factor(int pre, int shift) {

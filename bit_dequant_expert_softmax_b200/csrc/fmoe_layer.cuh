@@ -2,18 +2,17 @@
 //
 // One persistent thread block per SM (cooperative launch).  Per token:
 //
-//   P1  router matvec (fp64 accumulation of exact fp32 x bf16 products) over whole
-//       router rows per block (their copies start before the kernel waits for the
-//       previous grid), logits published as tagged words; while they travel, warps
-//       1-15 consume the block's slice of the shared expert's gate/up rows (they do
-//       not depend on the routing).
-//   P2  every block polls all logits and computes top-K redundantly; thread 0
-//       requests the block's slice of the K routed experts' gate/up row pairs one
-//       copy after another, and its down rows (P3's data) once half of those have
-//       landed; warps 1-15 compute h = silu(g) * u (four rows per activation load),
-//       warp 0 the renormalised softmax weights; h is published as tagged words.
-//   P3  every block polls h of all K+1 experts, computes its slice of output rows of
-//       the K+1 down matvecs (activations held in registers) and the combine
+//   P1  router matvec (fp64 accumulation of exact fp32 x bf16 products) over a
+//       slice of router rows per block, partials published with a per-block flag;
+//       while they travel, warps 1-15 consume the block's slice of the shared
+//       expert's gate/up rows (they do not depend on the routing) and warp 0 polls.
+//   P2  every block computes top-K from the logits redundantly; thread 0 requests
+//       the block's slice of the K routed experts' gate/up row pairs one copy after
+//       another, and its down rows (P3's data) once half of those have landed;
+//       warps 1-15 compute h = silu(g) * u, warp 0 the renormalised softmax
+//       weights; h is published with a per-block flag.
+//   P3  every block stages h of all K+1 experts, computes its slice of output
+//       rows of the K+1 down matvecs and the combine
 //       y = resid + sum_k w_k o_k + sigma o_s, rounded once to bf16.
 //
 // All weight bytes move HBM -> shared memory through the bulk-copy (TMA) engine
@@ -44,7 +43,8 @@ constexpr int kMaxDownBlock = 2 * kWarps;  // output rows per down item (two per
 constexpr int kMaxChunks = 8;              // gate/up chunks per round
 constexpr int kMaxExperts = 2048;          // routed experts a layer may have
 constexpr int kMaxSplits = 4;              // router column splits
-constexpr int kMaxGrid = 256;              // blocks a launch may have
+constexpr int kMaxGrid = 256;              // blocks a launch may have (flag words reserved)
+constexpr int kFlagStride = 8;             // uint32 per flag (one 32-byte sector each)
 
 enum Mode : int { MODE_ROUTE = 1, MODE_EXPERTS = 2, MODE_FULL = 3 };
 
@@ -71,8 +71,10 @@ struct Params {
   const float* sig_in;
   uint32_t* err;
   uint32_t* tokens;  // tokens this workspace has seen (tag base)
-  unsigned long long* lx;  // [E+1][2] router logits as tagged words (high, low half of the double)
-  unsigned long long* hx;  // [(K+1)*I] h values as tagged words
+  uint32_t* rflags;  // [kMaxGrid * kFlagStride] per-block "router partials written" tags
+  uint32_t* hflags;  // [kMaxGrid * kFlagStride] per-block "h rows written" tags
+  double* lpart;     // [2][(E+1)*nq] router partials
+  float* hbuf;       // [2][(K+1)*I]  h values
   int norm;         // 1: the input is a pre-norm block's h (the NORM kernel variant)
   double norm_eps;
   int staging_bytes;
@@ -106,7 +108,6 @@ struct alignas(128) SmemHeader {
   float wsl[kMaxK + 1];  // weight of each slot (w_k; slot K = sigma)
   int abort_flag;
   int skip_token;
-  int shared_done;  // warps that have consumed their share of the shared expert's gate/up rows
   uint32_t tok_base;
   ExpertPlan plan;
 };
@@ -206,39 +207,61 @@ struct LayerKernel {
   }
 
   // ---------------------------------------------------------------- exchanges
-  // Values every block needs from all others (router logits, h rows) travel as 64-bit
-  // words carrying the token's tag in their high half (fmoe::tagged).  Each word is
-  // written and read single-copy atomically (relaxed stores and loads at GPU scope,
-  // served by L2), so a reader polls the very words it needs until they carry its token's tag:
-  // no flags and no second read (the writers only fence once after their last words,
-  // so that the stores are performed at once).  The buffers alternate by token parity: a
-  // block writes token t+2's words only after every block has written token t+1's,
-  // which each does after it has read token t's.  Polls back off (64 ns doubling to
-  // about 1 us between retries, so that waiting blocks do not flood L2) and are
-  // bounded by the layer's time limit.
+  // Values every block needs from all others (router partials, h rows) are written
+  // with plain stores; then the block publishes the token's tag in its own flag word
+  // with a release store.  A reader's warp 0 polls the grid's flags (each lane a few,
+  // all of a lane's loads in flight together, relaxed loads, bounded), fences, and
+  // the block then reads the values once from L2.  Buffers alternate by token parity;
+  // no block can run two tokens ahead of another because each token needs every
+  // block's values.
   uint32_t tbase_;
   __device__ __forceinline__ uint32_t tag32(int t) const {
     return (tbase_ + static_cast<uint32_t>(t)) % 0xFFFFFFFFu + 1u;
   }
-  __device__ __forceinline__ unsigned long long* lx_of(int t) const {
-    return p.lx + static_cast<size_t>(t & 1) * 2 * (p.E + 1);
-  }
-  __device__ __forceinline__ unsigned long long* hx_of(int t) const {
-    return p.hx + static_cast<size_t>(t & 1) * (p.K + 1) * p.I;
+
+  __device__ __forceinline__ void publish(uint32_t* flags, int t) {
+    __syncthreads();
+    if (threadIdx.x == 0) st_release_u32(flags + blockIdx.x * kFlagStride, tag32(t));
   }
 
-  // One step of a bounded poll: sleeps (backing off); false (error bit set) once the
-  // limit has passed.
-  __device__ __forceinline__ bool poll_tick(uint64_t& t0, int& it) const {
-    const uint64_t now = global_timer_ns();
-    if (it == 0) t0 = now;
-    if (now - t0 > p.wait_ns) {
-      atomicOr(p.err, FMOE_DEVERR_BARRIER_TIMEOUT);
-      return false;
+  __device__ bool wait_all(const uint32_t* flags, int t) {
+    int fail = 0;
+    if (threadIdx.x < 32) {
+      const int G = gridDim.x, lane = threadIdx.x;
+      const uint32_t want = tag32(t);
+      constexpr int NF = kMaxGrid / 32;
+      uint32_t got[NF];
+#pragma unroll
+      for (int i = 0; i < NF; ++i) {
+        const int b = lane + 32 * i;
+        got[i] = b < G ? ld_relaxed_u32(flags + b * kFlagStride) : want;
+      }
+      uint64_t t0 = 0;
+      for (int it = 0;; ++it) {
+        bool all = true;
+#pragma unroll
+        for (int i = 0; i < NF; ++i) all &= got[i] == want;
+        if (__all_sync(0xffffffffu, all)) break;
+        if ((it & 15) == 15) {
+          if (t0 == 0) t0 = global_timer_ns();
+          const bool bad =
+              (ld_relaxed_u32(p.err) & FMOE_DEVERR_BARRIER_TIMEOUT) || global_timer_ns() - t0 > p.wait_ns;
+          if (__any_sync(0xffffffffu, bad)) {
+            if (lane == 0) atomicOr(p.err, FMOE_DEVERR_BARRIER_TIMEOUT);
+            fail = 1;
+            break;
+          }
+        }
+        __nanosleep(32);
+#pragma unroll
+        for (int i = 0; i < NF; ++i) {
+          const int b = lane + 32 * i;
+          if (got[i] != want) got[i] = ld_relaxed_u32(flags + b * kFlagStride);
+        }
+      }
+      __threadfence();
     }
-    __nanosleep(64u << min(it, 4));
-    ++it;
-    return true;
+    return __syncthreads_or(fail) == 0;
   }
 
   // ---------------------------------------------------------------- activations
@@ -299,7 +322,6 @@ struct LayerKernel {
 #pragma unroll
         for (int k = 0; k < 2; ++k) nat[k] = normed(nat[k], rn);
       }
-      if (base == 0 && (nat[0].x | nat[1].y | 1u)) mark(14);
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
@@ -327,60 +349,27 @@ struct LayerKernel {
     }
   }
 
-  // h of every slot (fp32 values in tagged words written by other blocks) polled from
-  // L2 until every word carries this token's tag: thread -> 4 consecutive columns (two
-  // 16-byte loads), all of a thread's loads in flight together; chunk sums and largest
-  // magnitudes by shuffles over the kCols/4 threads of a chunk; pre-scaled values
-  // scattered into the interleaved layout.  Returns false (in every thread that timed
-  // out) when a wait ran past the limit.
-  __device__ bool stage_h(float* hs, uint32_t hstride, float2* hsum) {
+  // h of every slot (fp32, written by other blocks, read from L2 once every block
+  // has published): coalesced 16-byte loads (thread -> 4 consecutive columns), all of
+  // a thread's loads in flight together; chunk sums by shuffles over the kCols/4
+  // threads of a chunk; pre-scaled values scattered into the interleaved layout.
+  __device__ void stage_h(const float* hb, float* hs, uint32_t hstride, float2* hsum) {
     constexpr int TPC = C::kCols / 4;
     const int per_slot = p.I / 4, nch = p.I / C::kCols;
     const int n4 = nslots * per_slot;
-    const uint32_t want = tag32(tok_);
-    const unsigned long long* src = hx_of(tok_);
-    bool ok = true;
-    for (int base = 0; base < n4; base += 4 * kThreads) {  // block-uniform trip count
-      ulonglong2 a[4], b[4];
+    const float4* src = reinterpret_cast<const float4*>(hb);
+    for (int base = 0; base < n4; base += 4 * kThreads) {
+      float4 v[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
-        if (q < n4) {
-          a[k] = ld_relaxed_v2_u64(src + 4 * q);
-          b[k] = ld_relaxed_v2_u64(src + 4 * q + 2);
-        } else {
-          a[k] = b[k] = make_ulonglong2(tagged(0u, want), tagged(0u, want));
-        }
-      }
-      // every retry re-reads all words still missing, their loads in flight together
-      uint64_t t0 = 0;
-      int it = 0;
-      while (ok) {
-        bool all = true;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          all &= has_tag(a[k].x, want) && has_tag(a[k].y, want) && has_tag(b[k].x, want) && has_tag(b[k].y, want);
-        if (all) break;
-        if (!poll_tick(t0, it)) {
-          ok = false;
-          break;
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
-          if (!(has_tag(a[k].x, want) && has_tag(a[k].y, want))) a[k] = ld_relaxed_v2_u64(src + 4 * q);
-          if (!(has_tag(b[k].x, want) && has_tag(b[k].y, want))) b[k] = ld_relaxed_v2_u64(src + 4 * q + 2);
-        }
+        v[k] = q < n4 ? __ldcg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int q = base + static_cast<int>(threadIdx.x) + k * kThreads;
-        const float4 v = make_float4(__uint_as_float(static_cast<uint32_t>(a[k].x)),
-                                     __uint_as_float(static_cast<uint32_t>(a[k].y)),
-                                     __uint_as_float(static_cast<uint32_t>(b[k].x)),
-                                     __uint_as_float(static_cast<uint32_t>(b[k].y)));
-        float sum = (v.x + v.y) + (v.z + v.w);
-        uint32_t mx = max_abs_bits(v);
+        float sum = (v[k].x + v[k].y) + (v[k].z + v[k].w);
+        uint32_t mx = max_abs_bits(v[k]);
 #pragma unroll
         for (int o = 1; o < TPC; o <<= 1) {
           sum += __shfl_xor_sync(0xffffffffu, sum, o);
@@ -389,68 +378,46 @@ struct LayerKernel {
         if (q < n4) {
           const int slot = q / per_slot, c0 = (q % per_slot) * 4, pre = chunk_pre(mx);
           float* d = hs + static_cast<size_t>(slot) * hstride;
-          d[phys(c0 + 0)] = v.x * prescale_factor(pre, C::shift_of(c0 + 0));
-          d[phys(c0 + 1)] = v.y * prescale_factor(pre, C::shift_of(c0 + 1));
-          d[phys(c0 + 2)] = v.z * prescale_factor(pre, C::shift_of(c0 + 2));
-          d[phys(c0 + 3)] = v.w * prescale_factor(pre, C::shift_of(c0 + 3));
+          d[phys(c0 + 0)] = v[k].x * prescale_factor(pre, C::shift_of(c0 + 0));
+          d[phys(c0 + 1)] = v[k].y * prescale_factor(pre, C::shift_of(c0 + 1));
+          d[phys(c0 + 2)] = v[k].z * prescale_factor(pre, C::shift_of(c0 + 2));
+          d[phys(c0 + 3)] = v[k].w * prescale_factor(pre, C::shift_of(c0 + 3));
           if (q % TPC == 0) hsum[slot * nch + c0 / C::kCols] = make_float2(sum, chunk_unscale(pre));
         }
       }
+      if (base == 0) mark(14);
     }
-    return ok;
+    mark(15);
   }
 
   __device__ __forceinline__ static int phys(int c) { return C::phys(c); }
 
   // ---------------------------------------------------------------- dot products
-  // Lane partials of sum_c W[r][c] v[c] for NR rows sharing the activation loads (W =
-  // scale*code + bias; v pre-scaled, interleaved).  The lanes stride over chunk parts:
-  // a 4-bit chunk (32 columns) is one part; a 2-bit chunk (64 columns) is two, one word
-  // pair each, so that rows of few chunks still keep every lane busy (the chunk's bias
-  // term goes with its first part).  Every row is summed in the same order whatever NR
-  // is.
-  template <int NR>
-  __device__ __forceinline__ void dotr(const uint8_t* const (&q)[NR], const uint32_t* const (&sb)[NR],
-                                       const float* vs, const float2* vsum, int nch, float (&res)[NR]) const {
-    constexpr int PPC = BITS == 2 ? 2 : 1;  // parts per chunk
+  // Lane partial of sum_c W[r][c] v[c] over the lane's chunks, for one or two rows
+  // sharing the activation loads (W = scale*code + bias; v pre-scaled, interleaved).
+  template <bool TWO>
+  __device__ __forceinline__ void dotn(const uint8_t* q0, const uint32_t* s0, const uint8_t* q1,
+                                       const uint32_t* s1, const float* vs, const float2* vsum, int nch, float& r0,
+                                       float& r1) const {
     const int lane = threadIdx.x & 31;
-#pragma unroll(NR <= 2 ? 2 : 1)
-    for (int u = lane; u < nch * PPC; u += 32) {
-      const int m = u / PPC, half = u % PPC;
-      unsigned long long a0[NR];
+#pragma unroll 2
+    for (int m = lane; m < nch; m += 32) {
+      const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(q0 + 16 * m);
+      ulonglong2 b = make_ulonglong2(0ull, 0ull);
+      if (TWO) b = *reinterpret_cast<const ulonglong2*>(q1 + 16 * m);
+      const ulonglong2* xv0 = C::f4(vs, m, 0);
+      const ulonglong2* xv1 = C::f4(vs, m, C::kF4PerPair);
+      unsigned long long a0 = 0ull, a1 = 0ull, b0 = 0ull, b1 = 0ull;
+      C::template word_pair2<TWO>(a.x, b.x, xv0, a0, b0);
+      C::template word_pair2<TWO>(a.y, b.y, xv1, a1, b1);
       const float2 vm = vsum[m];  // (sum of the chunk's activations, rescale of its products)
-      if constexpr (PPC == 1) {
-        unsigned long long wx[NR], wy[NR], a1[NR];
-#pragma unroll
-        for (int r = 0; r < NR; ++r) {
-          const ulonglong2 w = *reinterpret_cast<const ulonglong2*>(q[r] + 16 * m);
-          wx[r] = w.x;
-          wy[r] = w.y;
-          a0[r] = 0ull;
-          a1[r] = 0ull;
-        }
-        C::template word_pairs<NR>(wx, C::f4(vs, m, 0), a0);
-        C::template word_pairs<NR>(wy, C::f4(vs, m, C::kF4PerPair), a1);
-#pragma unroll
-        for (int r = 0; r < NR; ++r) {
-          const uint32_t sbv = sb[r][C::sb_index(m)];
-          res[r] = fmaf(sb_scale(sbv), (pair_sum(a0[r]) + pair_sum(a1[r])) * vm.y, res[r]);
-          res[r] = fmaf(sb_bias(sbv), vm.x, res[r]);
-        }
-      } else {
-        unsigned long long wx[NR];
-#pragma unroll
-        for (int r = 0; r < NR; ++r) {
-          wx[r] = *reinterpret_cast<const unsigned long long*>(q[r] + 16 * m + 8 * half);
-          a0[r] = 0ull;
-        }
-        C::template word_pairs<NR>(wx, C::f4(vs, m, half * C::kF4PerPair), a0);
-#pragma unroll
-        for (int r = 0; r < NR; ++r) {
-          const uint32_t sbv = sb[r][C::sb_index(m)];
-          res[r] = fmaf(sb_scale(sbv), pair_sum(a0[r]) * vm.y, res[r]);
-          if (half == 0) res[r] = fmaf(sb_bias(sbv), vm.x, res[r]);
-        }
+      const uint32_t sa = s0[C::sb_index(m)];
+      r0 = fmaf(sb_scale(sa), (pair_sum(a0) + pair_sum(a1)) * vm.y, r0);
+      r0 = fmaf(sb_bias(sa), vm.x, r0);
+      if (TWO) {
+        const uint32_t sbv = s1[C::sb_index(m)];
+        r1 = fmaf(sb_scale(sbv), (pair_sum(b0) + pair_sum(b1)) * vm.y, r1);
+        r1 = fmaf(sb_bias(sbv), vm.x, r1);
       }
     }
   }
@@ -493,71 +460,53 @@ struct LayerKernel {
     }
   }
 
-  // h of row pairs r .. r+np-1 (np = 1 or 2) of the chunk -> the tagged h words of the slot (one
-  // warp); two row pairs are four rows sharing the activation loads.
-  __device__ bool gu_unit(const GuChunk& c, int r, int np) {
+  // h of row pair r of the chunk -> hbuf[buf][slot][r]  (one warp)
+  __device__ bool gu_unit(const GuChunk& c, int r, int buf) {
     const int n = c.rb - c.ra, i = r - c.ra;
     if (!wait_item(c.first + i / p.rp)) return false;
-    if ((i + np - 1) / p.rp != i / p.rp && !wait_item(c.first + (i + np - 1) / p.rp)) return false;
     if (i >= p.rp && !wait_item(c.first)) return false;  // (scale,bias) rows ride on item 0
     const uint8_t* qg = stage + c.off + static_cast<uint32_t>(i) * 2u * p.qh;
+    const uint8_t* qu = qg + p.qh;
     const uint32_t lead =
         static_cast<uint32_t>((p.o_gu_sb + static_cast<unsigned long long>(c.ra) * 2u * p.sh) & 15ull);
     const uint32_t* sg = reinterpret_cast<const uint32_t*>(stage + c.off + g.gu_q(n) + lead) + i * 2 * (p.sh / 4);
-    const int sw = p.sh / 4;
-    unsigned long long* hout = hx_of(tok_) + static_cast<size_t>(c.slot) * p.I + r;
-    const uint32_t tag = tag32(tok_);
-    if (np == 2) {
-      const uint8_t* const q[4] = {qg, qg + p.qh, qg + 2 * p.qh, qg + 3 * p.qh};
-      const uint32_t* const sb[4] = {sg, sg + sw, sg + 2 * sw, sg + 3 * sw};
-      float v[4] = {0.f, 0.f, 0.f, 0.f};
-      dotr<4>(q, sb, xs, xsum, p.H / C::kCols, v);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) v[k] = warp_sum(v[k]);
-      if ((threadIdx.x & 31) == 0) {
-        st_relaxed_u64(hout, tagged(__float_as_uint((v[0] / (1.0f + expf(-v[0]))) * v[1]), tag));
-        st_relaxed_u64(hout + 1, tagged(__float_as_uint((v[2] / (1.0f + expf(-v[2]))) * v[3]), tag));
-      }
-    } else {
-      const uint8_t* const q[2] = {qg, qg + p.qh};
-      const uint32_t* const sb[2] = {sg, sg + sw};
-      float v[2] = {0.f, 0.f};
-      dotr<2>(q, sb, xs, xsum, p.H / C::kCols, v);
-      v[0] = warp_sum(v[0]);
-      v[1] = warp_sum(v[1]);
-      if ((threadIdx.x & 31) == 0)
-        st_relaxed_u64(hout, tagged(__float_as_uint((v[0] / (1.0f + expf(-v[0]))) * v[1]), tag));
+    const uint32_t* su = sg + p.sh / 4;
+    float gv = 0.f, uv = 0.f;
+    dotn<true>(qg, sg, qu, su, xs, xsum, p.H / C::kCols, gv, uv);
+    gv = warp_sum(gv);
+    uv = warp_sum(uv);
+    if ((threadIdx.x & 31) == 0) {
+      const float hval = (gv / (1.0f + expf(-gv))) * uv;
+      p.hbuf[static_cast<size_t>(buf) * (p.K + 1) * p.I + static_cast<size_t>(c.slot) * p.I + r] = hval;
     }
     return true;
   }
 
-  // Consume every row pair of `nc` chunks in units of `upairs` (1 or 2) row pairs, spread
-  // over warps w0 .. kWarps-1 (unit u -> warp w0 + u % (kWarps - w0)); w0 = 1 keeps warp
-  // 0, which issues the copies and computes the routing weights meanwhile, out of the
-  // routed rows.
-  __device__ void gu_consume(const GuChunk* ch, int nc, int w0 = 0, int upairs = 2) {
+  // Consume every row pair of `nc` chunks, spread over warps w0 .. kWarps-1 (unit u ->
+  // warp w0 + u % (kWarps - w0)); w0 = 1 keeps warp 0, which issues the copies and
+  // computes the routing weights meanwhile, out of the routed rows.
+  __device__ void gu_consume(const GuChunk* ch, int nc, int buf, int w0 = 0) {
     const int warp = threadIdx.x >> 5;
     if (warp < w0) return;
     const int nw = kWarps - w0;
     int base = 0;
     for (int k = 0; k < nc; ++k) {
-      const int n = ch[k].rb - ch[k].ra, nu = (n + upairs - 1) / upairs;
+      const int n = ch[k].rb - ch[k].ra;
       int first = (warp - w0 - base) % nw;
       if (first < 0) first += nw;
-      for (int u = first; u < nu; u += nw) {
-        if (!gu_unit(ch[k], ch[k].ra + upairs * u, min(upairs, n - upairs * u))) {
+      for (int i = first; i < n; i += nw) {
+        if (!gu_unit(ch[k], ch[k].ra + i, buf)) {
           hdr->abort_flag = 1;
           return;
         }
       }
-      base += nu;
+      base += n;
     }
-    __threadfence();  // push the h words out now: every block will wait for them
   }
 
   // Gate/up of routed units [v0, v1) (unit = slot*I + r) in rounds that fit the
   // whole staging area (used when the block's share does not fit at once).
-  __device__ bool gu_rounds(int v0, int v1) {
+  __device__ bool gu_rounds(int v0, int v1, int buf) {
     GuChunk ch[kMaxChunks];
     int nc = 0, items = 0;
     uint32_t used = 0;
@@ -584,7 +533,7 @@ struct LayerKernel {
         }
         issue_gu(ch, nc);
         nitem += static_cast<uint32_t>(items);
-        gu_consume(ch, nc);
+        gu_consume(ch, nc, buf);
         __syncthreads();
         if (hdr->abort_flag) return false;
         nc = 0;
@@ -634,114 +583,83 @@ struct LayerKernel {
     }
   }
 
-  // Down rows of an item as cells (group of up to four rows, slot): each warp takes a
-  // contiguous range of cells in group-major order, four rows sharing each activation
-  // load; its lanes accumulate w_s * o_s over the slots of a group and reduce the four
-  // rows once per group (group_sum4).  The weighted sum of a warp's run of slots
-  // [s0, s1) of group g goes to ob[s0 * n + j], zeros to the other slots of the run, so
-  // that every (slot, row) entry is written exactly once.
-  __device__ void down_cells(uint32_t off, int n, const float* hs, const float2* hsum, uint32_t lead, float* ob) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nch = p.I / C::kCols, sw = p.si / 4;
-    const int ng = (n + 3) >> 2, cells = ng * nslots;
-    const int c0 = cells * warp / kWarps, c1 = cells * (warp + 1) / kWarps;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    int cg = -1, s0 = 0;
-    auto flush = [&](int s1) {
-      const float r = group_sum4<32>(acc[0], acc[1], acc[2], acc[3]);
-      const int q = lane >> 3, j = 4 * cg + q;
-      if ((lane & 7) == 0 && j < n) {
-        ob[s0 * n + j] = r;
-        for (int sl = s0 + 1; sl < s1; ++sl) ob[sl * n + j] = 0.f;
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] = 0.f;
-    };
-    for (int c = c0; c < c1; ++c) {
-      const int gi = c / nslots, sl = c % nslots;
-      if (gi != cg) {
-        if (cg >= 0) flush(nslots);
-        cg = gi;
-        s0 = sl;
-      }
-      const int j0 = 4 * gi, nr = min(4, n - j0);
-      const uint8_t* blk = stage + off + sl * g.dn_slot(n);
-      const uint8_t* q0 = blk + static_cast<uint32_t>(j0) * p.qi;
-      const uint32_t* sp = reinterpret_cast<const uint32_t*>(blk + g.dn_q(n) + lead) + j0 * sw;
-      const float* hsl = hs + static_cast<size_t>(sl) * g.padded(p.I);
-      const float2* hsm = hsum + static_cast<size_t>(sl) * nch;
-      const float ws = hdr->wsl[sl];
-      float v[4] = {0.f, 0.f, 0.f, 0.f};
-      if (nr > 2) {  // a group of three repeats its last row (the fourth result is dropped)
-        const int r3 = nr - 1;
-        const uint8_t* const q[4] = {q0, q0 + p.qi, q0 + 2 * p.qi, q0 + r3 * p.qi};
-        const uint32_t* const sb[4] = {sp, sp + sw, sp + 2 * sw, sp + r3 * sw};
-        dotr<4>(q, sb, hsl, hsm, nch, v);
-      } else {
-        const int r1 = nr - 1;
-        const uint8_t* const q[2] = {q0, q0 + r1 * p.qi};
-        const uint32_t* const sb[2] = {sp, sp + r1 * sw};
-        float v2[2] = {0.f, 0.f};
-        dotr<2>(q, sb, hsl, hsm, nch, v2);
-        v[0] = v2[0];
-        v[1] = v2[1];
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] = fmaf(ws, v[k], acc[k]);
-    }
-    if (cg >= 0) flush(min(nslots, c1 - cg * nslots));
-  }
-
-  // Consume a down item (rows [ja, ja+n) of every slot): the weighted contributions
-  // are gathered in shared memory over the activations x (no longer read in this
-  // phase), then y = resid + their sum in slot order, rounded once.  Called by every
-  // thread; returns false for all on an abort.
+  // Consume a down item (rows [ja, ja+n)): y = resid + sum_s w_s o_s.  In a pre-norm
+  // block (NORM) y is the residual buffer itself: the block's residual rows are loaded
+  // before the dot products, so that the late loads do not queue behind other warps'
+  // stores to the same sectors.
   __device__ bool down_item(uint32_t item, uint32_t off, int ja, int n, const float* hs, const float2* hsum,
                             const uint16_t* resid_t, uint16_t* y_t) {
-    const uint32_t lead = static_cast<uint32_t>((p.o_d_sb + static_cast<unsigned long long>(ja) * p.si) & 15ull);
-    float* ob = xs;  // [nslots][n]
-    // the residual of the item's rows, loaded before the dot products (one coalesced
-    // load; in a stack block y is the residual buffer itself, rows of this block only)
-    const float rj = threadIdx.x < n ? bf16_to_f32(resid_t[ja + threadIdx.x]) : 0.f;
-    const bool ok = wait_item(item);
-    mark(15);
-    if (!ok) hdr->abort_flag = 1;
-    if (ok) down_cells(off, n, hs, hsum, lead, ob);
-    __syncthreads();
-    if (hdr->abort_flag) return false;
-    if (threadIdx.x < n) {
-      const int j = threadIdx.x;
-      float pa = 0.f;
-      for (int sl = 0; sl < nslots; ++sl) pa += ob[sl * n + j];
-      y_t[ja + j] = f32_to_bf16(rj + pa);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ia = warp, ib = warp + kWarps;
+    if (ia >= n) return true;
+    const bool two = ib < n;
+    float ra = 0.f, rb = 0.f;
+    if (NORM && lane == 0) {
+      ra = bf16_to_f32(resid_t[ja + ia]);
+      if (two) rb = bf16_to_f32(resid_t[ja + ib]);
     }
-    __syncthreads();
+    if (!wait_item(item)) {
+      hdr->abort_flag = 1;
+      return false;
+    }
+    const uint32_t lead = static_cast<uint32_t>((p.o_d_sb + static_cast<unsigned long long>(ja) * p.si) & 15ull);
+    const int nch = p.I / C::kCols;
+    float pa = 0.f, pb = 0.f;
+    for (int s = 0; s < nslots; ++s) {
+      const uint8_t* blk = stage + off + s * g.dn_slot(n);
+      const uint32_t* sbase = reinterpret_cast<const uint32_t*>(blk + g.dn_q(n) + lead);
+      float oa = 0.f, ob = 0.f;
+      const float* hsl = hs + static_cast<size_t>(s) * g.padded(p.I);
+      const float2* hsm = hsum + static_cast<size_t>(s) * nch;
+      if (two)
+        dotn<true>(blk + static_cast<uint32_t>(ia) * p.qi, sbase + ia * (p.si / 4),
+                   blk + static_cast<uint32_t>(ib) * p.qi, sbase + ib * (p.si / 4), hsl, hsm, nch, oa, ob);
+      else
+        dotn<false>(blk + static_cast<uint32_t>(ia) * p.qi, sbase + ia * (p.si / 4), nullptr, nullptr, hsl, hsm,
+                    nch, oa, ob);
+      const float ws = hdr->wsl[s];
+      pa = fmaf(ws, oa, pa);
+      pb = fmaf(ws, ob, pb);
+    }
+    pa = warp_sum(pa);
+    pb = warp_sum(pb);
+    if (lane == 0) {
+      if (!NORM) {
+        ra = bf16_to_f32(resid_t[ja + ia]);
+        if (two) rb = bf16_to_f32(resid_t[ja + ib]);
+      }
+      y_t[ja + ia] = f32_to_bf16(ra + pa);
+      if (two) y_t[ja + ib] = f32_to_bf16(rb + pb);
+    }
     return true;
   }
 
   // ---------------------------------------------------------------- P1
-  // Router rows [row0, row1) of the (E + has_shared) rows (the shared gate vector is the
-  // last row), whole rows per block, staged after the router's doubles; the block's
-  // slice of the shared expert's gate/up rows staged at the end of the staging area, to
-  // be consumed while the router logits travel.  These are weights only: the copies are
-  // issued before the kernel waits for the previous grid, and before the activations.
-  int row0_, row1_;
-  uint32_t p1first_, rbase_, rpart_;
+  // Router units [u0, u1) over (E + has_shared) rows x nq splits (the shared gate
+  // vector is the last row) staged after the router's doubles; the block's slice of
+  // the shared expert's gate/up rows staged at the end of the staging area, to be
+  // consumed after top-K while the routed rows are in flight.  All copies are issued
+  // before the activations are staged (they do not depend on them).
+  int u0_, u1_, row0_, row1_;
+  uint32_t p1first_, rbase_;
   GuChunk sc_;
   bool has_sc_;
 
   __device__ void phase1_issue(bool route, bool shared_gu) {
     const int rows = p.E + (p.has_shared ? 1 : 0);
     const int G = gridDim.x, b = blockIdx.x;
-    row0_ = row1_ = 0;
+    u0_ = u1_ = row0_ = row1_ = 0;
     if (route) {
-      row0_ = static_cast<int>(static_cast<long long>(rows) * b / G);
-      row1_ = static_cast<int>(static_cast<long long>(rows) * (b + 1) / G);
+      const long long U = static_cast<long long>(rows) * p.nq;
+      u0_ = static_cast<int>(U * b / G);
+      u1_ = static_cast<int>(U * (b + 1) / G);
+      row0_ = u0_ / p.nq;
+      row1_ = (u1_ + p.nq - 1) / p.nq;
     }
+    const int hc = p.H / p.nq;
     const uint32_t rib = g.router_item();
     rbase_ = route ? r128(static_cast<uint32_t>(p.H) * 8u) : 0u;
     const int nrouter = row1_ - row0_;
-    rpart_ = r128(rbase_ + static_cast<uint32_t>(nrouter) * rib);
     p1first_ = nitem;
     sc_ = GuChunk{p.K, 0, 0, 0, p1first_ + static_cast<uint32_t>(nrouter)};
     if (shared_gu) {
@@ -754,10 +672,14 @@ struct LayerKernel {
     if (threadIdx.x < 32) {
       fence_proxy_async_smem();
       for (int r = row0_ + static_cast<int>(threadIdx.x); r < row1_; r += 32) {
+        const int ua = max(u0_, r * p.nq), ub = min(u1_, r * p.nq + p.nq);
         uint64_t* bar = bar_of(p1first_ + (r - row0_));
+        const uint32_t bytes = static_cast<uint32_t>(ub - ua) * hc * 4u;
         const float* src = (r < p.E) ? p.router + static_cast<size_t>(r) * p.H : p.sgate;
-        mbar_arrive_expect_tx(bar, rib);
-        bulk_g2s(stage + rbase_ + (r - row0_) * rib, src, rib, bar);
+        src += static_cast<size_t>(ua - r * p.nq) * hc;
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(stage + rbase_ + (r - row0_) * rib + static_cast<uint32_t>(ua - r * p.nq) * hc * 4u, src, bytes,
+                 bar);
       }
       for (int i = static_cast<int>(threadIdx.x) - (nrouter % 32); i < nsh; i += 32)
         if (i >= 0) issue_gu_item(sc_, i);
@@ -765,21 +687,18 @@ struct LayerKernel {
     nitem += static_cast<uint32_t>(nrouter + nsh);
   }
 
-  // Router logits of this block's rows: every (row, column split) unit is a warp's fp64
-  // sum of exact fp32 x bf16 products, lanes striding the split; the splits' sums are
-  // added in split order (the batched router's order too, so both give the same bits)
-  // and published for every block to read.
-  __device__ bool phase1_consume(bool route) {
+  // Router dot products of this block's units: fp64 sums of exact fp32 x bf16 products.
+  __device__ bool phase1_consume(int buf, bool route) {
     if (route) {
+      const int rows = p.E + (p.has_shared ? 1 : 0);
       const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
       const int hc = p.H / p.nq;
       const uint32_t rib = g.router_item();
       const double2* xa = reinterpret_cast<const double2*>(stage);
       const double2* xb = xa + p.H / 4;
-      double* rpart = reinterpret_cast<double*>(stage + rpart_);
-      const int nu = (row1_ - row0_) * p.nq;
-      for (int u = warp; u < nu; u += kWarps) {
-        const int r = row0_ + u / p.nq, qq = u % p.nq;
+      double* lpart = p.lpart + static_cast<size_t>(buf) * rows * p.nq;
+      for (int u = u0_ + warp; u < u1_; u += kWarps) {
+        const int r = u / p.nq, qq = u % p.nq;
         if (!wait_item(p1first_ + (r - row0_))) {
           hdr->abort_flag = 1;
           break;
@@ -798,23 +717,7 @@ struct LayerKernel {
           acc1 = fma(static_cast<double>(wv.w), bb.y, acc1);
         }
         const double acc = warp_sum_d(acc0 + acc1);
-        if (lane == 0) rpart[u] = acc;
-      }
-      __syncthreads();
-      const uint32_t tag = tag32(tok_);
-      for (int i = threadIdx.x; i < row1_ - row0_; i += kThreads) {
-        const double* rp = rpart + i * p.nq;
-        double l;
-        if (p.nq == 4) {
-          l = ((rp[0] + rp[1]) + rp[2]) + rp[3];
-        } else {
-          l = 0.0;
-          for (int q = 0; q < p.nq; ++q) l += rp[q];
-        }
-        const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(l));
-        st_relaxed_v2_u64(lx_of(tok_) + 2 * (row0_ + i), tagged(static_cast<uint32_t>(bits >> 32), tag),
-                          tagged(static_cast<uint32_t>(bits), tag));
-        __threadfence();  // push the words out now: every block is about to wait for them
+        if (lane == 0) lpart[u] = acc;
       }
     }
     __syncthreads();
@@ -827,76 +730,47 @@ struct LayerKernel {
   // descending with ties to the lower index (compared through the order-preserving
   // 64-bit key of each fp64 logit), then the renormalised softmax weights of the K
   // and the shared sigmoid gate.
-  __device__ void topk(int t) {
+  __device__ void topk(int buf, int t) {
     mark(3);
-    const int rows = p.E + (p.has_shared ? 1 : 0);
-    const int lane = threadIdx.x & 31;
-    const int ngroups = (p.E + 31) >> 5;
-    // candidates of the first level: per group of 32 experts its K best, in rank order
-    unsigned long long* ckey = reinterpret_cast<unsigned long long*>(stage);
-    double* cval = reinterpret_cast<double*>(stage + r128(static_cast<uint32_t>(ngroups * p.K) * 8u));
-    int* cidx = reinterpret_cast<int*>(stage + 2 * r128(static_cast<uint32_t>(ngroups * p.K) * 8u));
-    // every thread polls the logits it ranks (all of its loads in flight together) and
-    // ranks each within its warp's group of 32 consecutive experts by shuffles
-    const uint32_t want = tag32(t);
-    const unsigned long long* lx = lx_of(t);
-    bool ok = true;
-    for (int e0 = 0; e0 < rows; e0 += 2 * kThreads) {  // block-uniform trip count
-      ulonglong2 v[2];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int e = e0 + static_cast<int>(threadIdx.x) + k * kThreads;
-        v[k] = e < rows ? ld_relaxed_v2_u64(lx + 2 * e) : make_ulonglong2(tagged(0u, want), tagged(0u, want));
-      }
-      {  // every retry re-reads all logits still missing, their loads in flight together
-        uint64_t t0 = 0;
-        int it = 0;
-        while (ok && !(has_tag(v[0].x, want) && has_tag(v[0].y, want) && has_tag(v[1].x, want) &&
-                       has_tag(v[1].y, want))) {
-          if (!poll_tick(t0, it)) {
-            ok = false;
-            break;
-          }
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int e = e0 + static_cast<int>(threadIdx.x) + k * kThreads;
-            if (!(has_tag(v[k].x, want) && has_tag(v[k].y, want))) v[k] = ld_relaxed_v2_u64(lx + 2 * e);
-          }
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int e = e0 + static_cast<int>(threadIdx.x) + k * kThreads;
-        double l = __longlong_as_double(static_cast<long long>((v[k].x << 32) | (v[k].y & 0xFFFFFFFFull)));
-        if (e < p.E && p.has_rbias) l += static_cast<double>(__ldg(p.rbias + e));
-        if (e == p.E && p.has_shared) hdr->selog[p.K] = l;
-        // experts beyond E take key 0, below every logit's key (and never selected)
-        const unsigned long long key = e < p.E ? dkey(l) : 0ull;
-        if (e - static_cast<int>(lane) < p.E) {  // warp-uniform: the group's first expert exists
-          int rank = 0;
-#pragma unroll 8
-          for (int j = 0; j < 32; ++j) {
-            const unsigned long long kj = __shfl_sync(0xffffffffu, key, j);
-            rank += static_cast<int>(kj > key) | (static_cast<int>(kj == key) & static_cast<int>(j < lane));
-          }
-          if (rank < p.K) {
-            const int slot = (e >> 5) * p.K + rank;
-            ckey[slot] = key;
-            cval[slot] = l;
-            cidx[slot] = e < p.E ? e : 0x7fffffff;
-          }
-        }
-      }
-    }
-    if (__syncthreads_or(!ok)) {
+    if (!wait_all(p.rflags, t)) {
       if (threadIdx.x == 0) hdr->abort_flag = 1;
       __syncthreads();
       return;
     }
     mark(10);
+    const int rows = p.E + (p.has_shared ? 1 : 0);
+    const int lane = threadIdx.x & 31;
+    const int ngroups = (p.E + 31) >> 5;
+    unsigned long long* ckey = reinterpret_cast<unsigned long long*>(stage);
+    double* cval = reinterpret_cast<double*>(stage + r128(static_cast<uint32_t>(ngroups * p.K) * 8u));
+    int* cidx = reinterpret_cast<int*>(stage + 2 * r128(static_cast<uint32_t>(ngroups * p.K) * 8u));
+    const double* lpart = p.lpart + static_cast<size_t>(buf) * rows * p.nq;
+    for (int e0 = 0; e0 < rows; e0 += kThreads) {  // block-uniform trip count
+      const int e = e0 + static_cast<int>(threadIdx.x);
+      double l = 0.0;
+      if (e < rows) {
+        l = router_logit(lpart + static_cast<size_t>(e) * p.nq, p.nq);
+        if (e < p.E && p.has_rbias) l += static_cast<double>(__ldg(p.rbias + e));
+        if (e == p.E && p.has_shared) hdr->selog[p.K] = l;
+      }
+      const unsigned long long key = e < p.E ? dkey(l) : 0ull;
+      if (e - static_cast<int>(lane) < p.E) {  // warp-uniform: the group's first expert exists
+        int rank = 0;
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+          const unsigned long long kj = __shfl_sync(0xffffffffu, key, j);
+          rank += static_cast<int>(kj > key) | (static_cast<int>(kj == key) & static_cast<int>(j < lane));
+        }
+        if (rank < p.K) {
+          const int slot = (e >> 5) * p.K + rank;
+          ckey[slot] = key;
+          cval[slot] = l;
+          cidx[slot] = e < p.E ? e : 0x7fffffff;
+        }
+      }
+    }
+    __syncthreads();
     mark(11);
-    // second level: every candidate's rank among all groups' candidates, counted by
-    // kStripe consecutive lanes (each over every kStripe-th candidate), summed by shuffles
     constexpr int kStripe = 8;
     const int ncand = ngroups * p.K;
     for (int base = 0; base < ncand * kStripe; base += kThreads) {  // block-uniform trip count
@@ -987,19 +861,11 @@ struct LayerKernel {
     pl.doff = gtotal;
     const uint32_t dtotal = g.dn_total(pl.j1 - pl.j0);
     pl.hoff = g.h_bytes() <= pl.doff ? 0u : r128(pl.doff + dtotal);
-    // the shared expert's rows (staged at the end of the staging area in P1) are
-    // consumed while the routed rows fly in: the routed chunks must stop before them
-    uint32_t sc_off = cap;
-    if (p.has_shared) {
-      const int sa = static_cast<int>(static_cast<long long>(p.I) * b / G);
-      const int sb = static_cast<int>(static_cast<long long>(p.I) * (b + 1) / G);
-      if (sb > sa) sc_off = (cap - g.gu_bytes(sb - sa)) & ~127u;
-    }
-    pl.prefetch = (vend >= pl.v1) && (pl.doff <= sc_off) && (pl.doff + dtotal <= cap) &&
-                  (pl.hoff + g.h_bytes() <= cap) && (gitems + pl.ndown <= kMaxRoundItems);
+    pl.prefetch = (vend >= pl.v1) && (pl.doff + dtotal <= cap) && (pl.hoff + g.h_bytes() <= cap) &&
+                  (gitems + pl.ndown <= kMaxRoundItems);
   }
 
-  __device__ bool experts(bool route, const uint16_t* resid_t, uint16_t* y_t) {
+  __device__ bool experts(int buf, bool route, const uint16_t* resid_t, uint16_t* y_t) {
     const ExpertPlan& pl = hdr->plan;
     const int j0 = pl.j0, j1 = pl.j1, ndown = pl.ndown;
     const bool prefetch = pl.prefetch != 0;
@@ -1017,46 +883,34 @@ struct LayerKernel {
       // the down rows are requested once the first half of the gate/up rows has
       // landed (thread 0 consumes none of them): requested together, both streams are
       // served interleaved and the gate/up rows complete late, while the down rows are
-      // needed only after the h exchange.  They overwrite the shared expert's rows, so
-      // they also wait (bounded) for warps 1-15 to have consumed those.  The copies are
-      // issued whatever the waits return.
+      // needed only after the h exchange.  The copies are issued whatever the wait
+      // returns.
       if (threadIdx.x == 0) {
         if (pl.gitems > 0) (void)wait_item(down_first - static_cast<uint32_t>(pl.gitems - (pl.gitems - 1) / 2));
-        if (has_sc_) {
-          const uint64_t t0 = global_timer_ns();
-          while (atomicAdd(&hdr->shared_done, 0) < kWarps - 1 && global_timer_ns() - t0 < p.wait_ns) __nanosleep(64);
-        }
         issue_down_items(j0, j1, 0, ndown, down_first, doff);
       }
-      // warps 1-15: the shared expert's gate/up rows first (in shared memory since P1),
-      // while the first routed rows are in flight
-      if (has_sc_ && threadIdx.x >= 32) {
-        gu_consume(&sc_, 1, 1, 1);
-        __syncwarp();
-        if ((threadIdx.x & 31) == 0) atomicAdd(&hdr->shared_done, 1);
-      }
-      gu_consume(ch, pl.nc, 1);
+      gu_consume(ch, pl.nc, buf, 1);
       __syncthreads();
       if (hdr->abort_flag) return false;
     } else {
       if (route) route_weights(tok_);
-      if (has_sc_) gu_consume(&sc_, 1, 0, 1);
-      __syncthreads();
-      if (hdr->abort_flag || !gu_rounds(pl.v0, pl.v1)) return false;
+      if (!gu_rounds(pl.v0, pl.v1, buf)) return false;
     }
+    publish(p.hflags, tok_);
     mark(5);
-    // ---- P3: stage h of every slot (polled from every block's tagged words), then the
-    // down rows
+    // ---- P3: stage h of every slot, then the down rows
     const uint32_t hbase = prefetch ? hoff : 0u;
     float* hs = reinterpret_cast<float*>(stage + hbase);
     const uint32_t hstride = g.padded(p.I);
     float2* hsum = reinterpret_cast<float2*>(hs + static_cast<size_t>(nslots) * hstride);
-    if (__syncthreads_or(!stage_h(hs, hstride, hsum))) {
+    if (!wait_all(p.hflags, tok_)) {
       if (threadIdx.x == 0) hdr->abort_flag = 1;
       __syncthreads();
       return false;
     }
     mark(6);
+    stage_h(p.hbuf + static_cast<size_t>(buf) * (p.K + 1) * p.I, hs, hstride, hsum);
+    __syncthreads();
     mark(7);
     if (prefetch) {
       for (int k = 0; k < ndown; ++k) {
@@ -1098,39 +952,26 @@ struct LayerKernel {
     } else if (threadIdx.x == 32 && p.mode != MODE_ROUTE) {
       plan_experts();
     }
-    __syncthreads();
-    if (p.timeline_token == 0) {  // diagnostic: the launch's start, before the grid dependency wait
-      tok_ = 0;
-      mark(13);
-      tok_ = -1;
-    }
-    const bool route = p.mode != MODE_EXPERTS;
-    const bool do_experts = p.mode != MODE_ROUTE;
-    // the first token's router rows and shared gate/up rows are weights, which no
-    // grid writes: their copies start before the wait for the previous grid
-    if (route) phase1_issue(route, do_experts && p.has_shared);
-    // everything above reads only weights, shared memory and the parameters; from here
-    // on the kernel reads what the previous grid may have written
+    // everything above touches only shared memory and the parameters; from here on
+    // the kernel reads what the previous grid may have written
     grid_dependency_wait();
     if (threadIdx.x == 0) hdr->tok_base = ld_relaxed_u32(p.tokens);
     const uint32_t err0 = ld_relaxed_u32(p.err);
     __syncthreads();
     tbase_ = hdr->tok_base;
-    if (err0 != 0) {  // sticky error from an earlier call
-      drain();
-      return;
-    }
+    if (err0 != 0) return;  // sticky error from an earlier call
+    const bool route = p.mode != MODE_EXPERTS;
+    const bool do_experts = p.mode != MODE_ROUTE;
     for (int t = 0; t < p.T; ++t) {
+      const int buf = t & 1;
       tok_ = t;
       mark(0);
-      if (threadIdx.x == 0) hdr->shared_done = 0;  // first read after the barriers of P1
       if (!route) {
         given_routing(t);
         if (hdr->skip_token) continue;
       }
-      // weight copies first (the first token's are in flight already), activations
-      // while they fly
-      if (!route || t > 0) phase1_issue(route, do_experts && p.has_shared);
+      // weight copies first, activations while they fly
+      phase1_issue(route, do_experts && p.has_shared);
       double2* xa = route ? reinterpret_cast<double2*>(stage) : nullptr;
       stage_x(p.x + static_cast<size_t>(t) * p.H, xa, xa ? xa + p.H / 4 : nullptr);
       __syncthreads();
@@ -1139,16 +980,21 @@ struct LayerKernel {
         drain();
         return;
       }
-      if (!phase1_consume(route)) break;
+      if (!phase1_consume(buf, route)) break;
+      if (route) publish(p.rflags, t);
       mark(2);
+      // the shared expert does not depend on the routing: warps 1-15 consume its
+      // gate/up rows while warp 0 already polls for the router partials (top-K's
+      // scratch and the shared rows occupy disjoint parts of the staging area)
+      if (has_sc_) gu_consume(&sc_, 1, buf, 1);
       if (route) {
-        topk(t);
+        topk(buf, t);
         if (hdr->abort_flag) break;
         if (!do_experts) route_weights(t);  // otherwise computed while the rows fly
         mark(4);
       }
       if (do_experts) {
-        if (!experts(route, p.resid + static_cast<size_t>(t) * p.H, p.y + static_cast<size_t>(t) * p.H))
+        if (!experts(buf, route, p.resid + static_cast<size_t>(t) * p.H, p.y + static_cast<size_t>(t) * p.H))
           break;
         mark(9);
       }

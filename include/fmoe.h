@@ -268,9 +268,7 @@ fmoe_status fmoe_layer_debug_hold_block(fmoe_layer_t layer, int cta);
  * staged, 2 router rows done, 3 top-K start (the shared expert's gate/up done), 4 top-K
  * done, 5 gate/up done, 6 h rows of all blocks visible, 7 h staged, 8 down rows done,
  * 9 token done, 10 router logits of all blocks visible, 11 expert ranks start, 12 expert
- * ranks done, 13 the launch's start (token 0 only, before the wait for the previous
- * grid), 14 the activations' loads returned, 15 the first down rows landed.  NULL
- * (default) disables it. */
+ * ranks done, 14 first batch of h loaded, 15 h loaded.  NULL (default) disables it. */
 fmoe_status fmoe_layer_debug_timeline(fmoe_layer_t layer, uint64_t* dev_buf, int token);
 
 /* Number of thread blocks one forward launch uses (one per SM of the device). */
