@@ -597,6 +597,72 @@ def bench_tier(args, rank, slots: int = 64, tokens: int = 200):
             "gpu_launches": 2 * tokens, "clocks": clocks}
 
 
+def bench_gdn(args, rank, layers: int = 45, heads: int = 64, dk: int = 128, dv: int = 128, steps: int = 50):
+    """GatedDeltaNet steps (the linear-attention layers beside the MoE: 45 of the 60
+    layers of the pages' model, 64 heads of 128 x 128 fp32 state each): one token through
+    all layers per step from a CUDA graph; the states (189 MB) exceed L2.  Roofline: the
+    state is read and written once per layer (8.39 MB)."""
+    import numpy as np
+    import torch
+
+    from bit_dequant_expert_softmax_b200 import fmoe
+
+    rng = np.random.default_rng(0)
+    S = torch.from_numpy((0.1 * rng.standard_normal((layers, heads, dv, dk))).astype(np.float32)).cuda()
+    q = torch.nn.functional.normalize(torch.from_numpy(rng.standard_normal((layers, heads, dk)).astype(np.float32)),
+                                      dim=-1).cuda()
+    k = torch.nn.functional.normalize(torch.from_numpy(rng.standard_normal((layers, heads, dk)).astype(np.float32)),
+                                      dim=-1).cuda()
+    v = torch.from_numpy(rng.standard_normal((layers, heads, dv)).astype(np.float32)).cuda()
+    alpha = torch.from_numpy(rng.uniform(0.5, 1.0, (layers, heads)).astype(np.float32)).cuda()
+    beta = torch.from_numpy(rng.uniform(0.0, 1.0, (layers, heads)).astype(np.float32)).cuda()
+    o = torch.empty(layers, heads, dv, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def token():
+        for l in range(layers):
+            fmoe.fmoe_gdn_step(S[l], q[l], k[l], v[l], alpha[l], beta[l], o[l], stream=stream)
+
+    with torch.cuda.stream(stream):
+        token()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        token()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = a.elapsed_time(b)
+    del g, S, q, k, v, alpha, beta, o
+    torch.cuda.empty_cache()
+    if rank != 0:
+        return None
+    per_launch_bytes = heads * dv * dk * 4 * 2 + heads * (2 * dk + 2 * dv + 2) * 4
+    launch_s = ms / 1e3 / (steps * layers)
+    peak, peak_kind = measured_peaks()
+    achieved = per_launch_bytes / launch_s / 1e9
+    return {"metric": f"GatedDeltaNet step, {layers} layers x {heads} heads x {dv}x{dk} state: tokens/s",
+            "value": steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": 3,
+            "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"gdn: {layers} layers, {heads} heads, state {dv}x{dk} fp32 ({layers * heads * dv * dk * 4 / 1e6:.0f} MB), "
+                                   "one token per step through all layers (CUDA graph)"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "gdn_step_kernel", "bytes_per_launch": per_launch_bytes,
+                         "avg_launch_us": round(launch_s * 1e6, 3)},
+            "gpu_launches": steps * layers, "clocks": clocks}
+
+
 SUB_CONFIGS = ("stack24_4bit", "stack60_2bit", "stack16_batched")
 
 
@@ -631,6 +697,7 @@ def main():
             line["sub_records"] = [bench_stack(args, world, rank, c, args.sub_steps, 3,
                                                0 if args.no_cpu_baseline else 2) for c in SUB_CONFIGS]
             line["sub_records"].append(bench_tier(args, rank))
+            line["sub_records"].append(bench_gdn(args, rank))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

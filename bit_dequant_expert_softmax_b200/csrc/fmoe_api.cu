@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/fmoe.h"
+#include "fmoe_gdn.cuh"
 #include "fmoe_grouped.cuh"
 #include "fmoe_layer.cuh"
 
@@ -675,6 +676,20 @@ fmoe_status fmoe_block_forward_batched(fmoe_layer_t L, const uint16_t* h, int T,
   p.resid = h;
   p.y = h_out;
   return launch_batched(L, p, true, s);
+}
+
+fmoe_status fmoe_gdn_step(float* state, const float* q, const float* k, const float* v, const float* alpha,
+                          const float* beta, float* o, int heads, int dk, int dv, void* stream) {
+  if (heads < 0 || dv < 1 || dk < 4 || dk % 4 != 0 || dk > 128 * kGdnMaxChunks) return FMOE_ERR_INVALID_ARG;
+  if (heads == 0) return FMOE_OK;
+  if (!state || !q || !k || !v || !alpha || !beta || !o) return FMOE_ERR_INVALID_ARG;
+  if (!aligned(state, 16) || !aligned(q, 16) || !aligned(k, 16)) return FMOE_ERR_INVALID_ARG;
+  const long long rows = (long long)heads * dv;
+  const long long blocks = (rows + kGdnWarps - 1) / kGdnWarps;
+  if (blocks > 0x7fffffffLL) return FMOE_ERR_UNSUPPORTED;
+  gdn_step_kernel<<<(unsigned)blocks, kGdnWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(state, q, k, v, alpha,
+                                                                                            beta, o, heads, dk, dv);
+  return cudaGetLastError() == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
 }
 
 fmoe_status fmoe_rmsnorm(const uint16_t* h, uint16_t* out, int T, int H, double eps, void* stream) {

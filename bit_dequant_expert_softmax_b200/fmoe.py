@@ -33,7 +33,7 @@ EXPORTS = ["fmoe_record_bytes", "fmoe_workspace_bytes", "fmoe_layer_create", "fm
            "fmoe_graph_destroy", "fmoe_batch_workspace_bytes", "fmoe_layer_set_batch_workspace",
            "fmoe_route_batched", "fmoe_layer_forward_batched", "fmoe_block_forward_batched",
            "fmoe_tier_buffer_bytes", "fmoe_tier_create", "fmoe_tier_forward", "fmoe_tier_stats",
-           "fmoe_tier_get_error", "fmoe_tier_destroy"]
+           "fmoe_tier_get_error", "fmoe_tier_destroy", "fmoe_gdn_step"]
 
 
 class FmoeError(RuntimeError):
@@ -103,6 +103,7 @@ def lib():
         L.fmoe_tier_stats.argtypes = [vp, ctypes.POINTER(u64), ctypes.POINTER(u64), ctypes.POINTER(u64)]
         L.fmoe_tier_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.fmoe_tier_destroy.argtypes = [vp]
+        L.fmoe_gdn_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp]
         L.fmoe_status_string.argtypes = [i32]
         L.fmoe_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -168,6 +169,14 @@ def fmoe_layer_forward_noalloc(handle, x, resid, T, y, stream=None):
     allocation); see include/fmoe.h."""
     _check(lib().fmoe_layer_forward_noalloc(handle, _ptr(x), _ptr(resid), T, _ptr(y), _stream(stream)),
            "fmoe_layer_forward_noalloc")
+
+
+def fmoe_gdn_step(state, q, k, v, alpha, beta, o, stream=None):
+    """One GatedDeltaNet token step in place on state [heads, dv, dk] (fp32 CUDA tensors);
+    o [heads, dv] gets the read-out (see include/fmoe.h)."""
+    heads, dv, dk = state.shape
+    _check(lib().fmoe_gdn_step(_ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o), heads, dk,
+                               dv, _stream(stream)), "fmoe_gdn_step")
 
 
 def fmoe_rmsnorm(h, out, T, H, eps=1e-6, stream=None):

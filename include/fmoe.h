@@ -274,6 +274,19 @@ fmoe_status fmoe_layer_debug_timeline(fmoe_layer_t layer, uint64_t* dev_buf, int
 /* Number of thread blocks one forward launch uses (one per SM of the device). */
 int fmoe_layer_grid_size(fmoe_layer_t layer);
 
+/* ---- GatedDeltaNet step (the linear-attention layers beside the MoE) ---------------
+ * One token of `heads` GatedDeltaNet heads, in place on the state:
+ *   S_h <- alpha_h S_h;  u = S_h k_h;  S_h <- S_h + beta_h (v_h - u) k_h^T;  o_h = S_h q_h
+ * (hotdry.top "Metal GPU管线", linear-attention paragraph: the pages run a scaling,
+ * matrix-vector products and a rank-1 update with BLAS on 64 heads x 128 x 128; the
+ * composition is GatedDeltaNet's gated delta rule).  All fp32 device pointers:
+ * state [heads][dv][dk] row-major (updated in place), q, k [heads][dk], v [heads][dv],
+ * alpha, beta [heads], o [heads][dv].  state, q and k 16-byte aligned; 4 <= dk <= 512,
+ * dk a multiple of 4; dv >= 1.  heads == 0 is a no-op.  Asynchronous on `stream`.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+fmoe_status fmoe_gdn_step(float* state, const float* q, const float* k, const float* v, const float* alpha,
+                          const float* beta, float* o, int heads, int dk, int dv, void* stream);
+
 /* ---- Host-memory expert tier ------------------------------------------------------
  * A layer whose routed experts do not all stay in HBM: their records live in host
  * memory and a cache of `slots` records in HBM holds the experts used most recently

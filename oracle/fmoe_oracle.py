@@ -376,3 +376,31 @@ def bf16_agreement(gpu: np.ndarray, ref: np.ndarray, min_rel_rms: float = 0.0):
     ulp = 2.0 * bf16_half_ulp(ref)
     d = np.abs(gpu - rb) / np.where(ulp > 0, ulp, 1.0)
     return float(np.mean(gpu == rb)), float(np.max(d))
+
+
+# ----------------------------------------------------------------------------
+# GatedDeltaNet step (the linear-attention layers' state update)
+# ----------------------------------------------------------------------------
+def gdn_step(S: np.ndarray, q: np.ndarray, k: np.ndarray, v: np.ndarray, alpha: float, beta: float):
+    """One token of a GatedDeltaNet head: the state S [dv, dk] is scaled by the gate
+    alpha, read at the key k, moved towards the value v by a rank-1 update of strength
+    beta, and read at the query q.  Returns (S_new, o), float64.
+
+    The pages implement this step with BLAS on a 64-head x 128 x 128 state: a scaling,
+    matrix-vector products and a rank-1 update (hotdry.top, "Metal GPU管线", the
+    linear-attention paragraph: cblas_sscal, cblas_sgemv, cblas_sger).  The update they
+    compose is the gated delta rule of GatedDeltaNet (Yang, Kautz, Hatamizadeh, "Gated
+    Delta Networks", ICLR 2025), taken here in the pages' order:
+      S <- alpha * S            (scale)
+      u  = S k                  (matrix-vector)
+      S <- S + beta (v - u) k^T (rank-1 update)
+      o  = S q                  (matrix-vector)"""
+    S = np.asarray(S, dtype=np.float64)
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    S = float(alpha) * S
+    u = S @ k
+    S = S + float(beta) * np.outer(v - u, k)
+    o = S @ q
+    return S, o

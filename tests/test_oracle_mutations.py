@@ -170,7 +170,25 @@ MUTATIONS = {
         lambda n: layer.forward(n, resid=n))(fo.bf16_to_f64(fo.rmsnorm_bf16(np.asarray(h, np.float64), eps)))},
     "block without the norm": {"block_forward": lambda layer, h, eps=1e-6: layer.forward(
         np.asarray(h, np.float64), resid=np.asarray(h, np.float64))},
+    # GatedDeltaNet step
+    "delta rule with the sign flipped": {"gdn_step": lambda S, q, k, v, a, b: _gdn_with(S, q, k, v, a, b, sign=-1.0)},
+    "key read before the decay": {"gdn_step": lambda S, q, k, v, a, b: _gdn_with(S, q, k, v, a, b, read_first=True)},
+    "rank-1 update transposed": {"gdn_step": lambda S, q, k, v, a, b: _gdn_with(S, q, k, v, a, b, transpose=True)},
+    "query read from the old state": {"gdn_step": lambda S, q, k, v, a, b: _gdn_with(S, q, k, v, a, b, old_read=True)},
 }
+
+
+def _gdn_with(S, q, k, v, alpha, beta, sign=1.0, read_first=False, transpose=False, old_read=False):
+    S0 = np.asarray(S, np.float64)
+    S = alpha * S0
+    u = (S0 if read_first else S) @ np.asarray(k, np.float64)
+    d = sign * (np.asarray(v, np.float64) - u) if sign > 0 else (np.asarray(v, np.float64) + u)
+    upd = np.outer(k, d) if transpose and S.shape[0] == S.shape[1] else np.outer(d, k)
+    if transpose and S.shape[0] != S.shape[1]:
+        upd = np.outer(d[::-1], k)
+    Sn = S + beta * upd
+    o = (S0 if old_read else Sn) @ np.asarray(q, np.float64)
+    return Sn, o
 
 
 @pytest.fixture(scope="module")

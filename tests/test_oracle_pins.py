@@ -468,3 +468,65 @@ def test_golden_tiny_regression():
         assert [int(i) for i in r.idx] == tok["idx"]
         assert np.allclose(r.w, tok["w"], rtol=1e-14, atol=0)
         assert np.allclose(r.y, tok["y"], rtol=1e-13, atol=1e-15)
+
+
+# ------------------------------------------------------------ GatedDeltaNet step ----
+def _gdn_case(dv=7, dk=5, seed=0):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((dv, dk)), rng.standard_normal(dk), rng.standard_normal(dk),
+            rng.standard_normal(dv))
+
+
+def test_gdn_identity_and_pure_decay():
+    """alpha = 1, beta = 0 leaves the state and reads S q; beta = 0 is a pure decay."""
+    S, q, k, v = _gdn_case()
+    S1, o1 = oracle.gdn_step(S, q, k, v, 1.0, 0.0)
+    assert np.array_equal(S1, S) and np.allclose(o1, S @ q, rtol=1e-15, atol=1e-15)
+    S2, o2 = oracle.gdn_step(S, q, k, v, 0.25, 0.0)
+    assert np.array_equal(S2, 0.25 * S) and np.allclose(o2, 0.25 * (S @ q), rtol=1e-15, atol=1e-15)
+
+
+def test_gdn_delta_rule_stores_the_value_at_a_unit_key():
+    """With |k| = 1 and beta = 1 the updated state maps k exactly to v (the delta
+    rule's defining property), whatever alpha and S."""
+    S, q, k, v = _gdn_case(9, 6, 1)
+    k = k / np.linalg.norm(k)
+    for alpha in (1.0, 0.7, 0.01):
+        S1, _ = oracle.gdn_step(S, q, k, v, alpha, 1.0)
+        assert np.allclose(S1 @ k, v, rtol=1e-12, atol=1e-12)
+
+
+def test_gdn_matches_closed_form_and_is_rank_one():
+    """S' = alpha S (I - beta k k^T) + beta v k^T (the same update as a matrix product);
+    S' - alpha S has rank one; o = S' q.  Also a one-hot key and query select a column."""
+    S, q, k, v = _gdn_case(6, 8, 2)
+    alpha, beta = 0.83, 0.37
+    S1, o1 = oracle.gdn_step(S, q, k, v, alpha, beta)
+    closed = alpha * S @ (np.eye(8) - beta * np.outer(k, k)) + beta * np.outer(v, k)
+    assert np.allclose(S1, closed, rtol=1e-12, atol=1e-12)
+    assert np.linalg.matrix_rank(S1 - alpha * S) == 1
+    assert np.allclose(o1, closed @ q, rtol=1e-12, atol=1e-12)
+    e = np.zeros(8)
+    e[3] = 1.0
+    S2, o2 = oracle.gdn_step(S, e, e, v, alpha, beta)
+    col = alpha * S[:, 3] + beta * (v - alpha * S[:, 3])
+    assert np.allclose(o2, col, rtol=1e-14, atol=1e-14) and np.allclose(S2[:, 3], col, rtol=1e-14, atol=1e-14)
+
+
+def test_gdn_brute_force_loops():
+    """A 3 x 2 head by scalar loops (no library products), two steps in sequence."""
+    S, q, k, v = _gdn_case(3, 2, 3)
+    Sb = S.copy()
+    St = S.copy()
+    for step, (alpha, beta) in enumerate([(0.9, 0.5), (0.6, 0.2)]):
+        qq, kk, vv = q * (step + 1), k - step, v + step
+        St, ot = oracle.gdn_step(St, qq, kk, vv, alpha, beta)
+        for i in range(3):
+            for j in range(2):
+                Sb[i][j] *= alpha
+        u = [sum(Sb[i][j] * kk[j] for j in range(2)) for i in range(3)]
+        for i in range(3):
+            for j in range(2):
+                Sb[i][j] += beta * (vv[i] - u[i]) * kk[j]
+        ob = [sum(Sb[i][j] * qq[j] for j in range(2)) for i in range(3)]
+        assert np.allclose(St, Sb, rtol=1e-13, atol=1e-13) and np.allclose(ot, ob, rtol=1e-13, atol=1e-13)
