@@ -1,5 +1,6 @@
 // Host side of libfmoe.so: validation, the layer handle, workspace layout and
 // kernel launches for the C ABI declared in include/fmoe.h.
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstdlib>
@@ -13,6 +14,7 @@
 #include "../../include/fmoe.h"
 #include "fmoe_gdn.cuh"
 #include "fmoe_grouped.cuh"
+#include "fmoe_umma.cuh"
 #include "fmoe_layer.cuh"
 
 using namespace fmoe;
@@ -69,10 +71,25 @@ WsLayout ws_layout(const fmoe_config& c) {
 
 // Workspace of the batched path for up to max_tokens tokens per call.
 struct BatchLayout {
-  size_t err, ticket, ntiles, tiles, tcost, pair_token, pidx, idx, w, sig, lpart, hbuf, obuf, xn, size;
+  size_t err, ticket, ntiles, tiles, tcost, pair_token, pidx, idx, w, sig, lpart, hbuf, obuf, xn, xg, hg, size;
 };
 
 int batch_max_tiles(const fmoe_config& c, int T) { return T * c.top_k + (T + kTileTok - 1) / kTileTok; }
+
+// The tcgen05 path takes whole pieces of every row and units of 128 rows.
+bool umma_shape_ok(const fmoe_config& c) {
+  const int pc = c.bits == 4 ? UGeom<4>::kPC : UGeom<2>::kPC;
+  return c.hidden % pc == 0 && c.inter % pc == 0 && c.hidden % kURows == 0;
+}
+
+// 16-pair blocks the activation tiles of one call can need: sum over tiles of
+// ceil(n / 16) <= pairs / 16 + tiles, with tiles of up to kUTileTok pairs.
+size_t umma_max_blocks16(const fmoe_config& c, int T) {
+  const size_t routed = (size_t)T * c.top_k, P = routed + (size_t)T;
+  const size_t tiles = std::min(routed, (size_t)c.n_experts) + (routed + kUTileTok - 1) / kUTileTok +
+                       (size_t)(T + kUTileTok - 1) / kUTileTok;
+  return (P + 15) / 16 + tiles;
+}
 
 BatchLayout batch_layout(const fmoe_config& c, int T) {
   BatchLayout b;
@@ -98,6 +115,12 @@ BatchLayout batch_layout(const fmoe_config& c, int T) {
   b.hbuf = take(P * c.inter * 4);
   b.obuf = take(P * c.hidden * 4);
   b.xn = take((size_t)T * c.hidden * 2);
+  b.xg = b.hg = 0;
+  if (umma_shape_ok(c)) {
+    const size_t nb = umma_max_blocks16(c, T);
+    b.xg = take(nb * xg_bytes_per16(c.hidden));
+    b.hg = take(nb * hg_bytes_per16(c.inter));
+  }
   b.size = o;
   return b;
 }
@@ -139,6 +162,10 @@ struct fmoe_layer {
   int max_tokens;
   BatchLayout bl;
   int g_router_smem, g_topk_smem, g_gu_smem, g_dn_smem;
+  // tcgen05 path of the batched matvecs
+  int umma;
+  int u_gu_slots, u_dn_slots, u_gu_smem, u_dn_smem;
+  uint8_t u_maps[4][sizeof(CUtensorMap)];  // gate/up codes, gate/up words, down codes, down words
 };
 
 namespace {
@@ -293,6 +320,81 @@ fmoe_status launch(const fmoe_layer* L, const Params& p, void* stream, bool allo
   return e == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
 }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// A 3-D byte tensor over one matrix of every expert record: {row bytes, rows,
+// experts}, boxes of `box_bytes` x 128 rows (128B-swizzled for the codes).
+bool encode_rows(uint8_t (&out)[sizeof(CUtensorMap)], const uint8_t* base, uint64_t row_bytes, uint64_t rows,
+                 uint64_t nexp, uint64_t rec_bytes, uint32_t box_bytes, bool swizzle) {
+  const EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn) return false;
+  CUtensorMap m;
+  const cuuint64_t dims[3] = {row_bytes, rows, nexp};
+  const cuuint64_t strides[2] = {row_bytes, rec_bytes};
+  const cuuint32_t box[3] = {box_bytes, (cuuint32_t)kURows, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, es,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  std::memcpy(out, &m, sizeof m);
+  return true;
+}
+
+// Ring slots and shared memory of the tcgen05 matvecs, and their tensor maps.  The
+// tcgen05 kernels run when FMOE_GROUPED_TCGEN05=1 asks for them and the shape fits
+// and the maps can be encoded; otherwise the layer keeps the mma.sync kernels (the
+// faster of the two on the measured workloads).
+template <int BITS>
+void plan_umma_bits(fmoe_layer* L, size_t room) {
+  const fmoe_config& c = L->cfg;
+  int sg = 0, sd = 0;
+  for (int s = kUMaxSlots; s >= 2 && !sg; --s)
+    if (umma_smem_bytes<BITS, false>(s) <= room) sg = s;
+  for (int s = kUMaxSlots; s >= 2 && !sd; --s)
+    if (umma_smem_bytes<BITS, true>(s) <= room) sd = s;
+  if (sg < 2 || sd < 2) return;  // at least double-buffered
+  const uint8_t* e = static_cast<const uint8_t*>(L->w.experts);
+  const uint64_t nexp = (uint64_t)c.n_experts + c.has_shared, rb = L->rec.size;
+  if (!encode_rows(L->u_maps[0], e, L->rec.qh, 2ull * c.inter, nexp, rb, kUCodeBox, true) ||
+      !encode_rows(L->u_maps[1], e + L->rec.o_gu_sb, L->rec.sh, 2ull * c.inter, nexp, rb, UGeom<BITS>::kSbBox, false) ||
+      !encode_rows(L->u_maps[2], e + L->rec.o_d_q, L->rec.qi, (uint64_t)c.hidden, nexp, rb, kUCodeBox, true) ||
+      !encode_rows(L->u_maps[3], e + L->rec.o_d_sb, L->rec.si, (uint64_t)c.hidden, nexp, rb, UGeom<BITS>::kSbBox,
+                   false))
+    return;
+  L->u_gu_slots = sg;
+  L->u_dn_slots = sd;
+  // more than half of the SM's shared memory: one block per SM, so that a block's
+  // tensor-memory allocation never waits for another block of the same kernel
+  L->u_gu_smem = std::max((int)umma_smem_bytes<BITS, false>(sg), kMaxSmem / 2 + 1024);
+  L->u_dn_smem = std::max((int)umma_smem_bytes<BITS, true>(sd), kMaxSmem / 2 + 1024);
+  L->umma = 1;
+}
+
+void plan_umma(fmoe_layer* L, size_t room) {
+  L->umma = 0;
+  const char* want = std::getenv("FMOE_GROUPED_TCGEN05");
+  if (!want || want[0] != '1' || !umma_shape_ok(L->cfg)) return;
+  if (L->cfg.bits == 4)
+    plan_umma_bits<4>(L, room);
+  else
+    plan_umma_bits<2>(L, room);
+}
+
 // Shared-memory plan of the batched kernels for up to T tokens per call.
 fmoe_status plan_batched(fmoe_layer* L, int T) {
   const fmoe_config& c = L->cfg;
@@ -321,6 +423,7 @@ fmoe_status plan_batched(fmoe_layer* L, int T) {
   L->g_topk_smem = (int)tsm;
   L->g_gu_smem = (int)gsm;
   L->g_dn_smem = (int)dsm;
+  plan_umma(L, room);
   return FMOE_OK;
 }
 
@@ -362,14 +465,17 @@ GParams batch_params(const fmoe_layer* L, int T) {
   p.lpart = reinterpret_cast<double*>(ws + b.lpart);
   p.hbuf = reinterpret_cast<float*>(ws + b.hbuf);
   p.obuf = reinterpret_cast<float*>(ws + b.obuf);
+  p.xg = b.xg ? ws + b.xg : nullptr;
+  p.hg = b.hg ? ws + b.hg : nullptr;
+  p.tile_tok = L->umma ? kUTileTok : kTileTok;
   p.wait_ns = L->wait_ns;
   return p;
 }
 
 // One launch, with programmatic stream serialization when the runtime allows it (the
 // kernels wait for their predecessor before reading anything).
-template <typename... A>
-cudaError_t launch_pdl(void (*kernel)(A...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, const GParams& p) {
+template <typename P, typename... A>
+cudaError_t launch_pdl(void (*kernel)(A...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, const P& p) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -395,12 +501,33 @@ fmoe_status launch_batched(const fmoe_layer* L, GParams p, bool experts, cudaStr
   const int G = L->sms;
   cudaError_t e = launch_pdl(grouped_router_kernel, dim3(G), dim3(kThreads), L->g_router_smem, s, p);
   if (e == cudaSuccess) e = launch_pdl(grouped_topk_kernel, dim3(p.T), dim3(kThreads), L->g_topk_smem, s, p);
-  if (experts && e == cudaSuccess)
-    e = launch_pdl(L->cfg.bits == 4 ? grouped_matvec_kernel<4, false> : grouped_matvec_kernel<2, false>, dim3(G),
-                   dim3(kGThreads), L->g_gu_smem, s, p);
-  if (experts && e == cudaSuccess)
-    e = launch_pdl(L->cfg.bits == 4 ? grouped_matvec_kernel<4, true> : grouped_matvec_kernel<2, true>, dim3(G),
-                   dim3(kGThreads), L->g_dn_smem, s, p);
+  if (experts && e == cudaSuccess && L->umma) {
+    const bool b4 = L->cfg.bits == 4;
+    e = launch_pdl(b4 ? grouped_stage_x_kernel<4> : grouped_stage_x_kernel<2>, dim3(G), dim3(256), 0, s, p);
+    UParams up;
+    up.p = p;
+    if (e == cudaSuccess) {
+      std::memcpy(&up.tm_q, L->u_maps[0], sizeof(CUtensorMap));
+      std::memcpy(&up.tm_sb, L->u_maps[1], sizeof(CUtensorMap));
+      up.slots = L->u_gu_slots;
+      e = launch_pdl(b4 ? grouped_umma_kernel<4, false> : grouped_umma_kernel<2, false>, dim3(G), dim3(kUThreads),
+                     L->u_gu_smem, s, up);
+    }
+    if (e == cudaSuccess) {
+      std::memcpy(&up.tm_q, L->u_maps[2], sizeof(CUtensorMap));
+      std::memcpy(&up.tm_sb, L->u_maps[3], sizeof(CUtensorMap));
+      up.slots = L->u_dn_slots;
+      e = launch_pdl(b4 ? grouped_umma_kernel<4, true> : grouped_umma_kernel<2, true>, dim3(G), dim3(kUThreads),
+                     L->u_dn_smem, s, up);
+    }
+  } else {
+    if (experts && e == cudaSuccess)
+      e = launch_pdl(L->cfg.bits == 4 ? grouped_matvec_kernel<4, false> : grouped_matvec_kernel<2, false>, dim3(G),
+                     dim3(kGThreads), L->g_gu_smem, s, p);
+    if (experts && e == cudaSuccess)
+      e = launch_pdl(L->cfg.bits == 4 ? grouped_matvec_kernel<4, true> : grouped_matvec_kernel<2, true>, dim3(G),
+                     dim3(kGThreads), L->g_dn_smem, s, p);
+  }
   if (experts && e == cudaSuccess)
     e = launch_pdl(grouped_combine_kernel, dim3((p.H + 255) / 256, p.T), dim3(256), 0, s, p);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
@@ -621,7 +748,9 @@ fmoe_status fmoe_layer_set_batch_workspace(fmoe_layer_t L, void* dev_ptr, size_t
   // to the device maximum (a layer-sized value would break larger layers' launches)
   if (!set_smem_max(grouped_router_kernel) || !set_smem_max(grouped_topk_kernel) ||
       !set_smem_max(grouped_matvec_kernel<4, false>) || !set_smem_max(grouped_matvec_kernel<2, false>) ||
-      !set_smem_max(grouped_matvec_kernel<4, true>) || !set_smem_max(grouped_matvec_kernel<2, true>))
+      !set_smem_max(grouped_matvec_kernel<4, true>) || !set_smem_max(grouped_matvec_kernel<2, true>) ||
+      !set_smem_max(grouped_umma_kernel<4, false>) || !set_smem_max(grouped_umma_kernel<2, false>) ||
+      !set_smem_max(grouped_umma_kernel<4, true>) || !set_smem_max(grouped_umma_kernel<2, true>))
     return FMOE_ERR_CUDA;
   if (cudaMemset(dev_ptr, 0, bl.size) != cudaSuccess) return FMOE_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
@@ -630,6 +759,11 @@ fmoe_status fmoe_layer_set_batch_workspace(fmoe_layer_t L, void* dev_ptr, size_t
   L->max_tokens = max_tokens;
   L->bl = bl;
   return FMOE_OK;
+}
+
+int fmoe_layer_batched_kind(fmoe_layer_t L) {
+  if (!L || !L->bws) return 0;
+  return L->umma ? 2 : 1;
 }
 
 fmoe_status fmoe_route_batched(fmoe_layer_t L, const uint16_t* x, int T, int32_t* idx, float* w, float* shared_sigma,

@@ -41,7 +41,8 @@ constexpr int kMaxSeg = 64;    // tiles one block's unit range may touch
 constexpr int kRing = 2;       // bulk copies in flight per warp
 
 struct GTile {
-  int expert, p0, n, pad;
+  int expert, p0, n;
+  int tok16;  // the tile's first 16-pair block in the activation tile buffers (tcgen05 path)
 };
 
 // Work weight of one unit of a tile of n pairs (relative).  Every unit moves the same
@@ -75,6 +76,9 @@ struct GParams {
   double* lpart;     // [T][(E + 1) * nq]
   float* hbuf;       // [P][I]
   float* obuf;       // [P][H]
+  uint8_t* xg;       // tcgen05 path: gate/up activation tiles (x of each tile's pairs)
+  uint8_t* hg;       // tcgen05 path: down activation tiles (h of each tile's pairs)
+  int tile_tok;      // pairs per tile: kTileTok (mma.sync path) or kUTileTok (tcgen05 path)
   unsigned long long wait_ns;
 };
 
@@ -280,7 +284,7 @@ __host__ __device__ inline TopkSmem topk_smem(int E, int K, int T, int has_share
 // gives every pair its place without any serial scan: the pair (t, e) is number
 // popcount(mask[e] & ((1 << t) - 1)) of expert e.
 __device__ void build_groups(const GParams& p, uint8_t* smem, const TopkSmem& L) {
-  const int E = p.E, K = p.K, T = p.T;
+  const int E = p.E, K = p.K, T = p.T, TT = p.tile_tok;
   int* sidx = reinterpret_cast<int*>(smem + L.sidx);
   unsigned long long* mask = reinterpret_cast<unsigned long long*>(smem + L.mask);
   int* off = reinterpret_cast<int*>(smem + L.off);
@@ -301,7 +305,7 @@ __device__ void build_groups(const GParams& p, uint8_t* smem, const TopkSmem& L)
   for (int e = e0; e < e1; ++e) {
     const int c = __popcll(mask[e]);
     npairs += c;
-    ntl += (c + kTileTok - 1) / kTileTok;
+    ntl += (c + TT - 1) / TT;
   }
   long long tot_pairs, tot_tiles;
   const long long poff = block_scan_excl(npairs, wsum, &tot_pairs);
@@ -311,13 +315,13 @@ __device__ void build_groups(const GParams& p, uint8_t* smem, const TopkSmem& L)
     for (int e = e0; e < e1; ++e) {
       const int c = __popcll(mask[e]);
       off[e] = static_cast<int>(po);
-      for (int i = 0; i * kTileTok < c; ++i) {
-        const int n = min(kTileTok, c - i * kTileTok);
-        p.tiles[to + i] = GTile{e, static_cast<int>(po) + i * kTileTok, n, 0};
+      for (int i = 0; i * TT < c; ++i) {
+        const int n = min(TT, c - i * TT);
+        p.tiles[to + i] = GTile{e, static_cast<int>(po) + i * TT, n, 0};
         tn[to + i] = n;
       }
       po += c;
-      to += (c + kTileTok - 1) / kTileTok;
+      to += (c + TT - 1) / TT;
     }
   }
   __syncthreads();
@@ -335,25 +339,32 @@ __device__ void build_groups(const GParams& p, uint8_t* smem, const TopkSmem& L)
       p.pair_token[PR + t] = t;
       p.pidx[t * (K + 1) + K] = PR + t;
     }
-    const int nts = (T + kTileTok - 1) / kTileTok;
+    const int nts = (T + TT - 1) / TT;
     for (int i = threadIdx.x; i < nts; i += kThreads) {
-      const int n = min(kTileTok, T - i * kTileTok);
-      p.tiles[routed_tiles + i] = GTile{E, PR + i * kTileTok, n, 0};
+      const int n = min(TT, T - i * TT);
+      p.tiles[routed_tiles + i] = GTile{E, PR + i * TT, n, 0};
       tn[routed_tiles + i] = n;
     }
     ntiles += nts;
   }
   __syncthreads();
-  // prefix sums of the tiles' work weights (contiguous runs per thread)
+  // prefix sums of the tiles' work weights and of their 16-pair blocks (contiguous
+  // runs per thread)
   const int tper = (ntiles + kThreads - 1) / kThreads;
   const int i0 = min(ntiles, static_cast<int>(threadIdx.x) * tper), i1 = min(ntiles, i0 + tper);
-  long long wsl = 0;
-  for (int i = i0; i < i1; ++i) wsl += tile_weight(tn[i]);
-  long long wtot;
+  long long wsl = 0, b16 = 0;
+  for (int i = i0; i < i1; ++i) {
+    wsl += tile_weight(tn[i]);
+    b16 += (tn[i] + 15) / 16;
+  }
+  long long wtot, btot;
   long long c = block_scan_excl(wsl, wsum, &wtot);
+  long long c16 = block_scan_excl(b16, wsum, &btot);
   for (int i = i0; i < i1; ++i) {
     p.tcost[i] = c;
+    p.tiles[i].tok16 = static_cast<int>(c16);
     c += tile_weight(tn[i]);
+    c16 += (tn[i] + 15) / 16;
   }
   if (threadIdx.x == 0) {
     p.tcost[ntiles] = wtot;

@@ -31,6 +31,7 @@ EXPORTS = ["fmoe_record_bytes", "fmoe_workspace_bytes", "fmoe_layer_create", "fm
            "fmoe_layer_forward_noalloc", "fmoe_status_string", "fmoe_block_forward", "fmoe_stack_create",
            "fmoe_stack_destroy", "fmoe_stack_forward", "fmoe_stack_graph_create", "fmoe_graph_launch",
            "fmoe_graph_destroy", "fmoe_batch_workspace_bytes", "fmoe_layer_set_batch_workspace",
+           "fmoe_layer_batched_kind",
            "fmoe_route_batched", "fmoe_layer_forward_batched", "fmoe_block_forward_batched",
            "fmoe_tier_buffer_bytes", "fmoe_tier_create", "fmoe_tier_forward", "fmoe_tier_stats",
            "fmoe_tier_get_error", "fmoe_tier_destroy", "fmoe_gdn_step"]
@@ -83,6 +84,8 @@ def lib():
         L.fmoe_batch_workspace_bytes.restype = sz
         L.fmoe_batch_workspace_bytes.argtypes = [ctypes.POINTER(fmoe_config), i32]
         L.fmoe_layer_set_batch_workspace.argtypes = [vp, vp, sz, i32]
+        L.fmoe_layer_batched_kind.argtypes = [vp]
+        L.fmoe_layer_batched_kind.restype = i32
         L.fmoe_route_batched.argtypes = [vp, vp, i32, vp, vp, vp, vp]
         L.fmoe_layer_forward_batched.argtypes = [vp, vp, vp, i32, vp, vp]
         L.fmoe_block_forward_batched.argtypes = [vp, vp, i32, ctypes.c_double, vp, vp]
@@ -217,6 +220,11 @@ def fmoe_layer_set_batch_workspace(handle, ws, max_tokens: int):
            "fmoe_layer_set_batch_workspace")
 
 
+def fmoe_layer_batched_kind(handle) -> int:
+    """2: tcgen05 grouped matvecs, 1: mma.sync ones, 0: no batch workspace."""
+    return int(lib().fmoe_layer_batched_kind(handle))
+
+
 def fmoe_route_batched(handle, x, T, idx, w, shared_sigma=None, stream=None):
     _check(lib().fmoe_route_batched(handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(shared_sigma), _stream(stream)),
            "fmoe_route_batched")
@@ -326,6 +334,10 @@ class Layer:
         fmoe_layer_set_batch_workspace(self.handle, ws, max_tokens)
         self.batch_workspace = ws
         return self
+
+    def batched_kind(self) -> int:
+        """2: the batched matvecs run on tcgen05, 1: on mma.sync, 0: no batch workspace."""
+        return fmoe_layer_batched_kind(self.handle)
 
     def forward_batched(self, x, resid=None, y=None, stream=None):
         import torch

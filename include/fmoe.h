@@ -188,6 +188,14 @@ size_t fmoe_batch_workspace_bytes(const fmoe_config* cfg, int max_tokens);
  * kernels' shared-memory plan cannot hold), CUDA. */
 fmoe_status fmoe_layer_set_batch_workspace(fmoe_layer_t layer, void* dev_ptr, size_t bytes, int max_tokens);
 
+/* Which kernels run the batched path's grouped matvecs: 2 = the tcgen05 kernels (A =
+ * dequantised codes in tensor memory, TMA-staged codes), taken when the environment
+ * variable FMOE_GROUPED_TCGEN05 is "1" at the time the workspace is attached, hidden
+ * and inter are multiples of 256 (4-bit) or 512 (2-bit) and the expert records admit
+ * TMA tensor maps; 1 = the mma.sync kernels (the default); 0 = no batch workspace
+ * attached or layer NULL.  Both compute the same per-group folded sums. */
+int fmoe_layer_batched_kind(fmoe_layer_t layer);
+
 /* Routing of T <= max_tokens tokens in one batched pass: idx int32 [T][K], w fp32 [T][K],
  * shared_sigma fp32 [T] (may be NULL), as fmoe_route computes them. */
 fmoe_status fmoe_route_batched(fmoe_layer_t layer, const uint16_t* x, int T, int32_t* idx, float* w,

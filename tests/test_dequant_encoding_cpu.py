@@ -191,3 +191,43 @@ def test_fold_coefficients_exact_in_fp32_for_the_workload(bits):
         b = oracle.bf16_to_f64((sb >> 16).astype(np.uint16))
         f32 = (b.astype(np.float32) - (s * 2 ** bits).astype(np.float32)).astype(np.float64)
         assert np.array_equal(f32, b - s * 2 ** bits)
+
+
+# The tcgen05 form of the same product: a converter thread turns a group's code words
+# into 32 TMEM words (4-bit word m -> columns 4m + j, j = 0..3, pair (code j, code j+4);
+# 2-bit word m -> columns 8m + j, j = 0..7, pair (code j, code j+8)); the MMA reads a
+# TMEM column as K positions 2c (low half) and 2c + 1 (high half).  The activation
+# tiles put column col of a row at K position kpos(col); every code must meet its own
+# activation.
+def _kpos(bits, c):
+    if bits == 4:
+        return (c & ~7) + 2 * (c & 3) + ((c >> 2) & 1)
+    return (c & ~15) + 2 * (c & 7) + ((c >> 3) & 1)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_tcgen05_k_order_pairs_every_code_with_its_activation(bits):
+    rng = np.random.default_rng(40 + bits)
+    per = 32 // bits
+    assert sorted(_kpos(bits, c) for c in range(64)) == list(range(64))  # a permutation of the group
+    for _ in range(20):
+        words = [int(v) for v in rng.integers(0, 2 ** 32, 64 // per, dtype=np.uint64)]
+        x = rng.standard_normal(64)
+        cols = {}  # TMEM column -> 32-bit word
+        for m, w in enumerate(words):
+            if bits == 4:
+                for j in range(4):
+                    cols[4 * m + j] = (rotr(w, 4 * j - 3) & 0x00780078) | 0x3F803F80
+            else:
+                for j in range(8):
+                    cols[8 * m + j] = (rotr(w, 2 * j - 5) & 0x00600060) | 0x3F803F80
+        assert sorted(cols) == list(range(32))
+        a = np.zeros(64)
+        for c, r in cols.items():
+            a[2 * c], a[2 * c + 1] = bf16_value(r & 0xFFFF), bf16_value(r >> 16)
+        b = np.zeros(64)
+        for col in range(64):
+            b[_kpos(bits, col)] = x[col]
+        codes = [(words[col // per] >> (bits * (col % per))) & ((1 << bits) - 1) for col in range(64)]
+        want = sum((1 + codes[col] / 2 ** bits) * x[col] for col in range(64))
+        assert abs(float(a @ b) - want) <= 1e-12 * (1 + np.abs(x).sum())

@@ -93,6 +93,51 @@ def test_batched_layer_matches_oracle(cuda_lib, name, T):
         _assert_token(f"{name} T={T} token {t}", ys[t], idx, w, sig, t, olay.forward(xs[t]), shape.has_shared)
 
 
+def _umma_shape(shape):
+    pc = 256 if shape.bits == 4 else 512
+    return shape.hidden % pc == 0 and shape.inter % pc == 0
+
+
+def test_batched_kind_follows_the_shape(cuda_lib, monkeypatch):
+    """mma.sync by default; tcgen05 on request where the shape allows it."""
+    for name, shape in SHAPES.items():
+        L = _layer(cuda_lib, shape, seed=20, max_tokens=8)
+        assert L.batched_kind() == 1, name
+        L.close()
+        monkeypatch.setenv("FMOE_GROUPED_TCGEN05", "1")
+        L = _layer(cuda_lib, shape, seed=20, max_tokens=8)
+        monkeypatch.delenv("FMOE_GROUPED_TCGEN05")
+        assert L.batched_kind() == (2 if _umma_shape(shape) else 1), name
+        L.close()
+
+
+@pytest.mark.parametrize("name", ["rbias_k10", "mid_2bit"])
+@pytest.mark.parametrize("T", [7, 32])
+def test_batched_tcgen05_and_mma_sync_paths(cuda_lib, name, T, monkeypatch):
+    """The same layer on both kernels of the grouped matvecs: each against the oracle,
+    and the two within the rounding of their fp32 sums of each other."""
+    shape = SHAPES[name]
+    monkeypatch.setenv("FMOE_GROUPED_TCGEN05", "1")
+    L = _layer(cuda_lib, shape, seed=28)
+    monkeypatch.delenv("FMOE_GROUPED_TCGEN05")
+    Lm = _layer(cuda_lib, shape, seed=28)
+    assert L.batched_kind() == 2 and Lm.batched_kind() == 1
+    x = _x(28, 0, T, shape.hidden)
+    y = L.forward_batched(x)
+    ym = Lm.forward_batched(x)
+    torch.cuda.synchronize()
+    assert L.error() == 0 and Lm.error() == 0
+    olay = oracle.synthetic_layer(28, 0, shape, lazy=True)
+    ib, wb, sb = (a.cpu().numpy() for a in L.route_batched(x))
+    xs, ys, yms = _bf(x), _bf(y), _bf(ym)
+    for t in range(T):
+        r = olay.forward(xs[t])
+        _assert_token(f"{name} T={T} tcgen05 token {t}", ys[t], ib, wb, sb, t, r, True)
+        _assert_token(f"{name} T={T} mma.sync token {t}", yms[t], ib, wb, sb, t, r, True)
+    L.close()
+    Lm.close()
+
+
 def test_batched_in_place_deterministic_and_graph(cuda_lib):
     shape = SHAPES["rbias_k10"]
     L = _layer(cuda_lib, shape, seed=22)
