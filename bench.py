@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--ref-tokens", type=int, default=1,
                     help="tokens per step of the reference arm (the CPU oracle)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["gdn", "tier"], default=None,
+                    help="run one sub-record's workload alone and print it as the line")
     return ap.parse_args()
 
 
@@ -131,11 +133,13 @@ def kernel_source_digest(texts) -> str:
     return h.hexdigest()
 
 
-def profiled_traffic(key: str = "traffic_bytes_per_launch", summary: str = "fmoe_layer_kernel_layer4096.md"):
-    """DRAM bytes per launch of the layer kernel (`key`) from a committed ncu summary,
-    if the kernel source is the one that was profiled (else None)."""
+def profiled_traffic(key: str = "traffic_bytes_per_launch", summary: str = "fmoe_layer_kernel_layer4096.md",
+                     sources=None):
+    """DRAM bytes per launch of a kernel (`key`) from a committed ncu summary, if the
+    kernel's sources (default: the layer kernel's) are the ones that were profiled
+    (else None)."""
     texts = []
-    for f in KERNEL_SOURCES:
+    for f in sources or KERNEL_SOURCES:
         with open(os.path.join(ROOT, "bit_dequant_expert_softmax_b200", "csrc", f)) as fh:
             texts.append(fh.read())
     path = os.path.join(ROOT, "profiles", summary)
@@ -657,7 +661,9 @@ def bench_gdn(args, rank, layers: int = 45, heads: int = 64, dk: int = 128, dv: 
             "config": {"workload": f"gdn: {layers} layers, {heads} heads, state {dv}x{dk} fp32 ({layers * heads * dv * dk * 4 / 1e6:.0f} MB), "
                                    "one token per step through all layers (CUDA graph)"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                         "frac": round(achieved / peak, 4),
+                         "traffic": profiled_traffic(summary="gdn_step_kernel_gdn45.md", sources=("fmoe_gdn.cuh",)),
+                         "peak_kind": peak_kind,
                          "kernel": "gdn_step_kernel", "bytes_per_launch": per_launch_bytes,
                          "avg_launch_us": round(launch_s * 1e6, 3)},
             "gpu_launches": steps * layers, "clocks": clocks}
@@ -687,6 +693,11 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     cfg = synth.CONFIGS[args.config]
+    if args.only and world == 1:
+        line = bench_gdn(args, rank) if args.only == "gdn" else bench_tier(args, rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
     if cfg["layers"] > 1 or cfg["batch"] > 1:
         line = bench_stack(args, world, rank, args.config, args.steps, args.warmup,
                            0 if args.no_cpu_baseline else 2)
