@@ -15,6 +15,7 @@
 #include "fmoe_gdn.cuh"
 #include "fmoe_grouped.cuh"
 #include "fmoe_umma.cuh"
+#include "fmoe_gemv.cuh"
 #include "fmoe_layer.cuh"
 
 using namespace fmoe;
@@ -71,7 +72,8 @@ WsLayout ws_layout(const fmoe_config& c) {
 
 // Workspace of the batched path for up to max_tokens tokens per call.
 struct BatchLayout {
-  size_t err, ticket, ntiles, tiles, tcost, pair_token, pidx, idx, w, sig, lpart, hbuf, obuf, xn, xg, hg, size;
+  size_t err, ticket, ntiles, ntiles_s, tiles, tcost, tiles_s, tcost_s, tiles_all, pair_token, pidx, idx, w, sig,
+      lpart, hbuf, obuf, xn, xg, hg, size;
 };
 
 int batch_max_tiles(const fmoe_config& c, int T) { return T * c.top_k + (T + kTileTok - 1) / kTileTok; }
@@ -98,6 +100,7 @@ BatchLayout batch_layout(const fmoe_config& c, int T) {
   b.err = 0;
   b.ticket = 128;
   b.ntiles = 256;
+  b.ntiles_s = 384;
   size_t o = 512;
   auto take = [&](size_t bytes) {
     const size_t at = o;
@@ -106,6 +109,9 @@ BatchLayout batch_layout(const fmoe_config& c, int T) {
   };
   b.tiles = take(mt * sizeof(GTile));
   b.tcost = take((mt + 1) * sizeof(long long));
+  b.tiles_s = take(mt * sizeof(GTile));
+  b.tcost_s = take((mt + 1) * sizeof(long long));
+  b.tiles_all = take(mt * sizeof(GTile));
   b.pair_token = take(P * 4);
   b.pidx = take(P * 4);
   b.idx = take((size_t)T * c.top_k * 4);
@@ -162,6 +168,8 @@ struct fmoe_layer {
   int max_tokens;
   BatchLayout bl;
   int g_router_smem, g_topk_smem, g_gu_smem, g_dn_smem;
+  int small;                  // tiles of <= kSmallTok pairs on the CUDA-core kernels
+  int s_gu_smem, s_dn_smem;
   // tcgen05 path of the batched matvecs
   int umma;
   int u_gu_slots, u_dn_slots, u_gu_smem, u_dn_smem;
@@ -424,6 +432,14 @@ fmoe_status plan_batched(fmoe_layer* L, int T) {
   L->g_gu_smem = (int)gsm;
   L->g_dn_smem = (int)dsm;
   plan_umma(L, room);
+  // the small tiles' CUDA-core kernels, on request (FMOE_GROUPED_SMALL=1), beside the
+  // mma.sync kernels (slower than the mma.sync kernels alone on the measured workloads)
+  const uint32_t sg = c.bits == 4 ? small_smem_bytes<4>(false, c.hidden, c.inter) : small_smem_bytes<2>(false, c.hidden, c.inter);
+  const uint32_t sd = c.bits == 4 ? small_smem_bytes<4>(true, c.hidden, c.inter) : small_smem_bytes<2>(true, c.hidden, c.inter);
+  const char* want_small = std::getenv("FMOE_GROUPED_SMALL");
+  L->small = !L->umma && sg <= room && sd <= room && want_small && want_small[0] == '1';
+  L->s_gu_smem = (int)sg;
+  L->s_dn_smem = (int)sd;
   return FMOE_OK;
 }
 
@@ -457,6 +473,11 @@ GParams batch_params(const fmoe_layer* L, int T) {
   p.ntiles = reinterpret_cast<int*>(ws + b.ntiles);
   p.tiles = reinterpret_cast<GTile*>(ws + b.tiles);
   p.tcost = reinterpret_cast<long long*>(ws + b.tcost);
+  p.ntiles_s = reinterpret_cast<int*>(ws + b.ntiles_s);
+  p.tiles_s = reinterpret_cast<GTile*>(ws + b.tiles_s);
+  p.tcost_s = reinterpret_cast<long long*>(ws + b.tcost_s);
+  p.tiles_all = reinterpret_cast<GTile*>(ws + b.tiles_all);
+  p.small_tok = L->small ? kSmallTok : 0;
   p.pair_token = reinterpret_cast<int*>(ws + b.pair_token);
   p.pidx = reinterpret_cast<int*>(ws + b.pidx);
   p.idx = reinterpret_cast<int32_t*>(ws + b.idx);
@@ -521,11 +542,18 @@ fmoe_status launch_batched(const fmoe_layer* L, GParams p, bool experts, cudaStr
                      L->u_dn_smem, s, up);
     }
   } else {
+    const bool b4 = L->cfg.bits == 4;
+    if (experts && e == cudaSuccess && L->small)
+      e = launch_pdl(b4 ? grouped_small_kernel<4, false> : grouped_small_kernel<2, false>, dim3(G), dim3(kGThreads),
+                     L->s_gu_smem, s, p);
     if (experts && e == cudaSuccess)
-      e = launch_pdl(L->cfg.bits == 4 ? grouped_matvec_kernel<4, false> : grouped_matvec_kernel<2, false>, dim3(G),
+      e = launch_pdl(b4 ? grouped_matvec_kernel<4, false> : grouped_matvec_kernel<2, false>, dim3(G),
                      dim3(kGThreads), L->g_gu_smem, s, p);
+    if (experts && e == cudaSuccess && L->small)
+      e = launch_pdl(b4 ? grouped_small_kernel<4, true> : grouped_small_kernel<2, true>, dim3(G), dim3(kGThreads),
+                     L->s_dn_smem, s, p);
     if (experts && e == cudaSuccess)
-      e = launch_pdl(L->cfg.bits == 4 ? grouped_matvec_kernel<4, true> : grouped_matvec_kernel<2, true>, dim3(G),
+      e = launch_pdl(b4 ? grouped_matvec_kernel<4, true> : grouped_matvec_kernel<2, true>, dim3(G),
                      dim3(kGThreads), L->g_dn_smem, s, p);
   }
   if (experts && e == cudaSuccess)
@@ -750,7 +778,9 @@ fmoe_status fmoe_layer_set_batch_workspace(fmoe_layer_t L, void* dev_ptr, size_t
       !set_smem_max(grouped_matvec_kernel<4, false>) || !set_smem_max(grouped_matvec_kernel<2, false>) ||
       !set_smem_max(grouped_matvec_kernel<4, true>) || !set_smem_max(grouped_matvec_kernel<2, true>) ||
       !set_smem_max(grouped_umma_kernel<4, false>) || !set_smem_max(grouped_umma_kernel<2, false>) ||
-      !set_smem_max(grouped_umma_kernel<4, true>) || !set_smem_max(grouped_umma_kernel<2, true>))
+      !set_smem_max(grouped_umma_kernel<4, true>) || !set_smem_max(grouped_umma_kernel<2, true>) ||
+      !set_smem_max(grouped_small_kernel<4, false>) || !set_smem_max(grouped_small_kernel<2, false>) ||
+      !set_smem_max(grouped_small_kernel<4, true>) || !set_smem_max(grouped_small_kernel<2, true>))
     return FMOE_ERR_CUDA;
   if (cudaMemset(dev_ptr, 0, bl.size) != cudaSuccess) return FMOE_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return FMOE_ERR_CUDA;
@@ -763,7 +793,7 @@ fmoe_status fmoe_layer_set_batch_workspace(fmoe_layer_t L, void* dev_ptr, size_t
 
 int fmoe_layer_batched_kind(fmoe_layer_t L) {
   if (!L || !L->bws) return 0;
-  return L->umma ? 2 : 1;
+  return L->umma ? 2 : (L->small ? 3 : 1);
 }
 
 fmoe_status fmoe_route_batched(fmoe_layer_t L, const uint16_t* x, int T, int32_t* idx, float* w, float* shared_sigma,

@@ -228,7 +228,7 @@ struct Chunk {
     return ((((m >> 5) * kF4 + k) << 5) + (m & 31)) * 4 + e;
   }
   // (scale,bias) word index of chunk m within its row
-  __device__ __forceinline__ static int sb_index(int m) { return BITS == 4 ? (m >> 1) : m; }
+  __host__ __device__ __forceinline__ static int sb_index(int m) { return BITS == 4 ? (m >> 1) : m; }
 
   // One word pair W = {w_a, w_b} against its activation pairs (kF4PerPair float4 at
   // xv[0], xv[32], ... in the interleaved layout), accumulated into acc.

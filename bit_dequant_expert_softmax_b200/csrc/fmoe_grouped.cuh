@@ -65,9 +65,14 @@ struct GParams {
   float* sig_out;
   uint32_t* err;
   uint32_t* ticket;  // top-K blocks finished (the last one groups)
-  int* ntiles;
+  int* ntiles;        // tiles of more than small_tok pairs (the tensor-core kernels)
   GTile* tiles;
-  long long* tcost;  // [ntiles + 1] prefix sums of tile weights
+  long long* tcost;   // [ntiles + 1] prefix sums of tile weights
+  int* ntiles_s;      // tiles of at most small_tok pairs (the CUDA-core kernels)
+  GTile* tiles_s;
+  long long* tcost_s;
+  GTile* tiles_all;   // every tile, before the split
+  int small_tok;      // 0: every tile goes to the tensor-core kernels
   int* pair_token;   // [P] token of each pair
   int* pidx;         // [T][K + 1] pair of (token, slot)
   int32_t* idx;      // [T][K]
@@ -317,7 +322,7 @@ __device__ void build_groups(const GParams& p, uint8_t* smem, const TopkSmem& L)
       off[e] = static_cast<int>(po);
       for (int i = 0; i * TT < c; ++i) {
         const int n = min(TT, c - i * TT);
-        p.tiles[to + i] = GTile{e, static_cast<int>(po) + i * TT, n, 0};
+        p.tiles_all[to + i] = GTile{e, static_cast<int>(po) + i * TT, n, 0};
         tn[to + i] = n;
       }
       po += c;
@@ -342,33 +347,55 @@ __device__ void build_groups(const GParams& p, uint8_t* smem, const TopkSmem& L)
     const int nts = (T + TT - 1) / TT;
     for (int i = threadIdx.x; i < nts; i += kThreads) {
       const int n = min(TT, T - i * TT);
-      p.tiles[routed_tiles + i] = GTile{E, PR + i * TT, n, 0};
+      p.tiles_all[routed_tiles + i] = GTile{E, PR + i * TT, n, 0};
       tn[routed_tiles + i] = n;
     }
     ntiles += nts;
   }
   __syncthreads();
-  // prefix sums of the tiles' work weights and of their 16-pair blocks (contiguous
-  // runs per thread)
+  // split (stable) into the small tiles (<= small_tok pairs) and the others; prefix
+  // sums of each list's work weights and of the large tiles' 16-pair blocks
+  // (contiguous runs per thread)
   const int tper = (ntiles + kThreads - 1) / kThreads;
   const int i0 = min(ntiles, static_cast<int>(threadIdx.x) * tper), i1 = min(ntiles, i0 + tper);
-  long long wsl = 0, b16 = 0;
+  long long nsm = 0, nlg = 0, wsm = 0, wlg = 0, b16 = 0;
   for (int i = i0; i < i1; ++i) {
-    wsl += tile_weight(tn[i]);
-    b16 += (tn[i] + 15) / 16;
+    if (tn[i] <= p.small_tok) {
+      ++nsm;
+      wsm += tile_weight(tn[i]);
+    } else {
+      ++nlg;
+      wlg += tile_weight(tn[i]);
+      b16 += (tn[i] + 15) / 16;
+    }
   }
-  long long wtot, btot;
-  long long c = block_scan_excl(wsl, wsum, &wtot);
+  long long ns_tot, nl_tot, ws_tot, wl_tot, btot;
+  long long so = block_scan_excl(nsm, wsum, &ns_tot);
+  long long lo = block_scan_excl(nlg, wsum, &nl_tot);
+  long long cs = block_scan_excl(wsm, wsum, &ws_tot);
+  long long cl = block_scan_excl(wlg, wsum, &wl_tot);
   long long c16 = block_scan_excl(b16, wsum, &btot);
   for (int i = i0; i < i1; ++i) {
-    p.tcost[i] = c;
-    p.tiles[i].tok16 = static_cast<int>(c16);
-    c += tile_weight(tn[i]);
-    c16 += (tn[i] + 15) / 16;
+    GTile t = p.tiles_all[i];
+    if (tn[i] <= p.small_tok) {
+      p.tiles_s[so] = t;
+      p.tcost_s[so] = cs;
+      ++so;
+      cs += tile_weight(tn[i]);
+    } else {
+      t.tok16 = static_cast<int>(c16);
+      p.tiles[lo] = t;
+      p.tcost[lo] = cl;
+      ++lo;
+      cl += tile_weight(tn[i]);
+      c16 += (tn[i] + 15) / 16;
+    }
   }
   if (threadIdx.x == 0) {
-    p.tcost[ntiles] = wtot;
-    *p.ntiles = ntiles;
+    p.tcost[nl_tot] = wl_tot;
+    p.tcost_s[ns_tot] = ws_tot;
+    *p.ntiles = static_cast<int>(nl_tot);
+    *p.ntiles_s = static_cast<int>(ns_tot);
     *p.ticket = 0;  // ready for the next launch (every block of this one has counted)
   }
 }

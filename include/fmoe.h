@@ -188,12 +188,18 @@ size_t fmoe_batch_workspace_bytes(const fmoe_config* cfg, int max_tokens);
  * kernels' shared-memory plan cannot hold), CUDA. */
 fmoe_status fmoe_layer_set_batch_workspace(fmoe_layer_t layer, void* dev_ptr, size_t bytes, int max_tokens);
 
-/* Which kernels run the batched path's grouped matvecs: 2 = the tcgen05 kernels (A =
- * dequantised codes in tensor memory, TMA-staged codes), taken when the environment
- * variable FMOE_GROUPED_TCGEN05 is "1" at the time the workspace is attached, hidden
- * and inter are multiples of 256 (4-bit) or 512 (2-bit) and the expert records admit
- * TMA tensor maps; 1 = the mma.sync kernels (the default); 0 = no batch workspace
- * attached or layer NULL.  Both compute the same per-group folded sums. */
+/* Which kernels run the batched path's grouped matvecs:
+ *   1 = the default: the mma.sync tensor-core kernels for every tile;
+ *   3 = tiles of at most 2 pairs on CUDA-core dequantising matvecs (the single-token
+ *       path's dot), larger tiles on the mma.sync kernels: taken when the environment
+ *       variable FMOE_GROUPED_SMALL is "1" when the workspace is attached and their
+ *       shared memory fits;
+ *   2 = the tcgen05 kernels (A = dequantised codes in tensor memory, TMA-staged codes),
+ *       taken when FMOE_GROUPED_TCGEN05 is "1" at attach time, hidden and inter are
+ *       multiples of 256 (4-bit) or 512 (2-bit) and the expert records admit TMA
+ *       tensor maps (it takes precedence over FMOE_GROUPED_SMALL);
+ *   0 = no batch workspace attached or layer NULL.
+ * All compute the same per-(pair, row) sums to within fp32 rounding. */
 int fmoe_layer_batched_kind(fmoe_layer_t layer);
 
 /* Routing of T <= max_tokens tokens in one batched pass: idx int32 [T][K], w fp32 [T][K],

@@ -98,44 +98,51 @@ def _umma_shape(shape):
     return shape.hidden % pc == 0 and shape.inter % pc == 0
 
 
+def _layer_kind(cuda_lib, shape, seed, env, monkeypatch, max_tokens=64):
+    """A layer attached with the environment variable `env` set to "1" (or none)."""
+    if env:
+        monkeypatch.setenv(env, "1")
+    try:
+        return _layer(cuda_lib, shape, seed=seed, max_tokens=max_tokens)
+    finally:
+        if env:
+            monkeypatch.delenv(env)
+
+
 def test_batched_kind_follows_the_shape(cuda_lib, monkeypatch):
-    """mma.sync by default; tcgen05 on request where the shape allows it."""
+    """mma.sync by default; CUDA-core small tiles or tcgen05 on request (tcgen05 where
+    the shape allows it)."""
     for name, shape in SHAPES.items():
-        L = _layer(cuda_lib, shape, seed=20, max_tokens=8)
-        assert L.batched_kind() == 1, name
-        L.close()
-        monkeypatch.setenv("FMOE_GROUPED_TCGEN05", "1")
-        L = _layer(cuda_lib, shape, seed=20, max_tokens=8)
-        monkeypatch.delenv("FMOE_GROUPED_TCGEN05")
-        assert L.batched_kind() == (2 if _umma_shape(shape) else 1), name
-        L.close()
+        for env, want in ((None, 1), ("FMOE_GROUPED_SMALL", 3),
+                          ("FMOE_GROUPED_TCGEN05", 2 if _umma_shape(shape) else 1)):
+            L = _layer_kind(cuda_lib, shape, 20, env, monkeypatch, max_tokens=8)
+            assert L.batched_kind() == want, (name, env)
+            L.close()
 
 
-@pytest.mark.parametrize("name", ["rbias_k10", "mid_2bit"])
-@pytest.mark.parametrize("T", [7, 32])
-def test_batched_tcgen05_and_mma_sync_paths(cuda_lib, name, T, monkeypatch):
-    """The same layer on both kernels of the grouped matvecs: each against the oracle,
-    and the two within the rounding of their fp32 sums of each other."""
+@pytest.mark.parametrize("name", ["rbias_k10", "mid_2bit", "tiny", "e40_noshared"])
+@pytest.mark.parametrize("T", [1, 7, 32])
+def test_batched_kernel_variants(cuda_lib, name, T, monkeypatch):
+    """The same layer on each kernel configuration of the grouped matvecs (mma.sync,
+    CUDA-core small tiles + mma.sync, tcgen05 where the shape allows it): each against
+    the oracle, routing identical."""
     shape = SHAPES[name]
-    monkeypatch.setenv("FMOE_GROUPED_TCGEN05", "1")
-    L = _layer(cuda_lib, shape, seed=28)
-    monkeypatch.delenv("FMOE_GROUPED_TCGEN05")
-    Lm = _layer(cuda_lib, shape, seed=28)
-    assert L.batched_kind() == 2 and Lm.batched_kind() == 1
+    envs = [None, "FMOE_GROUPED_SMALL"] + (["FMOE_GROUPED_TCGEN05"] if _umma_shape(shape) else [])
     x = _x(28, 0, T, shape.hidden)
-    y = L.forward_batched(x)
-    ym = Lm.forward_batched(x)
-    torch.cuda.synchronize()
-    assert L.error() == 0 and Lm.error() == 0
     olay = oracle.synthetic_layer(28, 0, shape, lazy=True)
-    ib, wb, sb = (a.cpu().numpy() for a in L.route_batched(x))
-    xs, ys, yms = _bf(x), _bf(y), _bf(ym)
-    for t in range(T):
-        r = olay.forward(xs[t])
-        _assert_token(f"{name} T={T} tcgen05 token {t}", ys[t], ib, wb, sb, t, r, True)
-        _assert_token(f"{name} T={T} mma.sync token {t}", yms[t], ib, wb, sb, t, r, True)
-    L.close()
-    Lm.close()
+    xs = _bf(x)
+    refs = [olay.forward(xs[t]) for t in range(T)]
+    for env in envs:
+        L = _layer_kind(cuda_lib, shape, 28, env, monkeypatch)
+        y = L.forward_batched(x)
+        ib, wb, sb = (a.cpu().numpy() for a in L.route_batched(x))
+        torch.cuda.synchronize()
+        assert L.error() == 0, env
+        ys = _bf(y)
+        for t in range(T):
+            _assert_token(f"{name} T={T} {env or 'default'} token {t}", ys[t], ib, wb, sb, t, refs[t],
+                          shape.has_shared)
+        L.close()
 
 
 def test_batched_in_place_deterministic_and_graph(cuda_lib):
