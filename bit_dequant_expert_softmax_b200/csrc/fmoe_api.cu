@@ -848,11 +848,30 @@ fmoe_status fmoe_gdn_step(float* state, const float* q, const float* k, const fl
   if (heads == 0) return FMOE_OK;
   if (!state || !q || !k || !v || !alpha || !beta || !o) return FMOE_ERR_INVALID_ARG;
   if (!aligned(state, 16) || !aligned(q, 16) || !aligned(k, 16)) return FMOE_ERR_INVALID_ARG;
-  const long long rows = (long long)heads * dv;
-  const long long blocks = (rows + kGdnWarps - 1) / kGdnWarps;
+  // rows per warp: 8 for dk <= 128, 2 for longer rows (the loads of a warp in flight
+  // together, 32 float4 registers either way)
+  const bool narrow = dk <= 128;
+  const int R = narrow ? 8 : 2;
+  const long long warps = (long long)heads * ((dv + R - 1) / R);
+  const long long blocks = (warps + kGdnWarps - 1) / kGdnWarps;
   if (blocks > 0x7fffffffLL) return FMOE_ERR_UNSUPPORTED;
-  gdn_step_kernel<<<(unsigned)blocks, kGdnWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(state, q, k, v, alpha,
-                                                                                            beta, o, heads, dk, dv);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(kGdnWarps * 32);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_pdl_ok.load(std::memory_order_relaxed) ? 1 : 0;
+  auto kernel = narrow ? gdn_step_kernel<1, 8> : gdn_step_kernel<kGdnMaxChunks, 2>;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, state, q, k, v, alpha, beta, o, heads, dk, dv);
+  if (e != cudaSuccess && cfg.numAttrs == 1) {
+    cudaGetLastError();
+    cfg.numAttrs = 0;
+    e = cudaLaunchKernelEx(&cfg, kernel, state, q, k, v, alpha, beta, o, heads, dk, dv);
+  }
+  if (e != cudaSuccess) return FMOE_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FMOE_OK : FMOE_ERR_CUDA;
 }
 
