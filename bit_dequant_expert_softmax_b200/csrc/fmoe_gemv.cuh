@@ -13,12 +13,12 @@
 // mma.sync kernels on the same tiles (8 warps per SM leave its FMA chains short of
 // issue slots), so the layer runs it only on request (FMOE_GROUPED_SMALL=1).
 //
-// Work: persistent blocks of 8 warps over a contiguous, weight-balanced range of units
+// Work: persistent blocks of kGWarps warps over a contiguous, weight-balanced range of units
 // (tile, 16 rows): gate/up units are the gate rows 8u..8u+7 and the up rows of the same
 // r (rows 0-7 and 8-15 of the unit), down units 16 output rows.  Per tile a block
 // stages the activations of the tile's pairs (x, or h for down) in the pre-scaled,
 // lane-interleaved layout; each warp streams its units' 16 rows x 32 chunks per piece
-// through a private two-slot ring of bulk copies; lane l takes chunk l of every row of
+// through a private ring of bulk copies; lane l takes chunk l of every row of
 // the piece (rows i and i + 8 together, sharing the activation loads); each row pair's
 // partials are reduced over the warp and lane i keeps row i's sums for the unit.
 #pragma once

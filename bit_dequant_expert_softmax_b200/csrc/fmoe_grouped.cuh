@@ -12,7 +12,7 @@
 //            expert, each with a work weight
 //   gate/up  persistent blocks, each a contiguous, weight-balanced range of
 //            (tile, 8 row pairs) units: a tile's activations are staged once, every
-//            warp streams its own units' rows through a two-slot ring of bulk copies
+//            warp streams its own units' rows through a one-slot ring of bulk copies
 //            and multiplies them on the tensor cores (mma.sync, exact bf16 operands);
 //            h = silu(W_g x) * (W_u x) for each pair of the tile
 //   down     the same over (tile, 16 output rows) units, activations = h of the
@@ -38,7 +38,7 @@ constexpr int kTileTok = 8;    // pairs of one expert whose activations are stag
 constexpr int kRouterTok = 8;  // tokens per pass of the batched router
 constexpr int kMaxBatch = 64;  // tokens one batched call may have
 constexpr int kMaxSeg = 64;    // tiles one block's unit range may touch
-constexpr int kRing = 2;       // bulk copies in flight per warp
+constexpr int kRing = 1;       // bulk copies in flight per warp (16 warps: latency is hidden across warps)
 
 struct GTile {
   int expert, p0, n;
@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_topk_kernel(const __grid_
 //   k = 2q+j      <-> column c0 + q + 8j
 //   k = 8 + 2q+j  <-> column c0 + q + 4 + 8j
 // where q = lane % 4 and j in {0, 1}.
-constexpr int kGWarps = 8;  // warps of a grouped matvec block
+constexpr int kGWarps = 16;  // warps of a grouped matvec block
 constexpr int kGThreads = kGWarps * 32;
 constexpr int kPieceCols = 1024;  // columns of one staged piece of a unit's 16 rows
 
