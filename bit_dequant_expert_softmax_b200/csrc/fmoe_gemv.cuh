@@ -10,8 +10,9 @@
 // group's scale and bias once.  This kernel takes the tiles of at most kSmallTok
 // pairs, the tensor-core kernels the rest; the arithmetic per (pair, row) is the
 // single-token kernel's.  Measured on the 32-token top-10 layer it is slower than the
-// mma.sync kernels on the same tiles (8 warps per SM leave its FMA chains short of
-// issue slots), so the layer runs it only on request (FMOE_GROUPED_SMALL=1).
+// mma.sync kernels on the same tiles (a warp reduction per row pair and piece and the
+// per-row addressing outweigh the cheaper products), so the layer runs it only on
+// request (FMOE_GROUPED_SMALL=1).
 //
 // Work: persistent blocks of kGWarps warps over a contiguous, weight-balanced range of units
 // (tile, 16 rows): gate/up units are the gate rows 8u..8u+7 and the up rows of the same
