@@ -93,7 +93,14 @@ size_t umma_max_blocks16(const fmoe_config& c, int T) {
   return (P + 15) / 16 + tiles;
 }
 
-BatchLayout batch_layout(const fmoe_config& c, int T) {
+// The tcgen05 kernels are asked for through FMOE_GROUPED_TCGEN05=1.
+bool umma_requested() {
+  const char* want = std::getenv("FMOE_GROUPED_TCGEN05");
+  return want && want[0] == '1';
+}
+
+// umma_tiles: room for the tcgen05 kernels' activation tiles (shapes they take only)
+BatchLayout batch_layout(const fmoe_config& c, int T, bool umma_tiles) {
   BatchLayout b;
   const size_t nq = (size_t)router_splits(c.hidden);
   const size_t P = (size_t)T * (c.top_k + 1), mt = (size_t)batch_max_tiles(c, T);
@@ -122,7 +129,7 @@ BatchLayout batch_layout(const fmoe_config& c, int T) {
   b.obuf = take(P * c.hidden * 4);
   b.xn = take((size_t)T * c.hidden * 2);
   b.xg = b.hg = 0;
-  if (umma_shape_ok(c)) {
+  if (umma_tiles && umma_shape_ok(c)) {
     const size_t nb = umma_max_blocks16(c, T);
     b.xg = take(nb * xg_bytes_per16(c.hidden));
     b.hg = take(nb * hg_bytes_per16(c.inter));
@@ -393,10 +400,9 @@ void plan_umma_bits(fmoe_layer* L, size_t room) {
   L->umma = 1;
 }
 
-void plan_umma(fmoe_layer* L, size_t room) {
+void plan_umma(fmoe_layer* L, size_t room, bool want) {
   L->umma = 0;
-  const char* want = std::getenv("FMOE_GROUPED_TCGEN05");
-  if (!want || want[0] != '1' || !umma_shape_ok(L->cfg)) return;
+  if (!want || !umma_shape_ok(L->cfg)) return;
   if (L->cfg.bits == 4)
     plan_umma_bits<4>(L, room);
   else
@@ -404,7 +410,7 @@ void plan_umma(fmoe_layer* L, size_t room) {
 }
 
 // Shared-memory plan of the batched kernels for up to T tokens per call.
-fmoe_status plan_batched(fmoe_layer* L, int T) {
+fmoe_status plan_batched(fmoe_layer* L, int T, bool want_umma) {
   const fmoe_config& c = L->cfg;
   const int G = L->sms;
   const int rows = c.n_experts + c.has_shared;
@@ -431,7 +437,7 @@ fmoe_status plan_batched(fmoe_layer* L, int T) {
   L->g_topk_smem = (int)tsm;
   L->g_gu_smem = (int)gsm;
   L->g_dn_smem = (int)dsm;
-  plan_umma(L, room);
+  plan_umma(L, room, want_umma);
   // the small tiles' CUDA-core kernels, on request (FMOE_GROUPED_SMALL=1), beside the
   // mma.sync kernels (slower than the mma.sync kernels alone on the measured workloads)
   const uint32_t sg = c.bits == 4 ? small_smem_bytes<4>(false, c.hidden, c.inter) : small_smem_bytes<2>(false, c.hidden, c.inter);
@@ -762,15 +768,21 @@ fmoe_status fmoe_block_forward(fmoe_layer_t L, const uint16_t* h, int T, double 
 
 size_t fmoe_batch_workspace_bytes(const fmoe_config* cfg, int max_tokens) {
   if (!config_ok(cfg) || max_tokens < 1 || max_tokens > kMaxBatch) return 0;
-  return batch_layout(*cfg, max_tokens).size;
+  return batch_layout(*cfg, max_tokens, umma_requested()).size;
 }
 
 fmoe_status fmoe_layer_set_batch_workspace(fmoe_layer_t L, void* dev_ptr, size_t bytes, int max_tokens) {
   if (!L || !dev_ptr || !aligned(dev_ptr, 256) || max_tokens < 1 || max_tokens > kMaxBatch)
     return FMOE_ERR_INVALID_ARG;
-  const BatchLayout bl = batch_layout(L->cfg, max_tokens);
+  // the tcgen05 kernels only when asked for and the workspace has their tiles' room
+  bool want_umma = umma_requested() && umma_shape_ok(L->cfg);
+  BatchLayout bl = batch_layout(L->cfg, max_tokens, want_umma);
+  if (want_umma && bytes < bl.size) {
+    want_umma = false;
+    bl = batch_layout(L->cfg, max_tokens, false);
+  }
   if (bytes < bl.size) return FMOE_ERR_NO_WORKSPACE;
-  const fmoe_status st = plan_batched(L, max_tokens);
+  const fmoe_status st = plan_batched(L, max_tokens, want_umma);
   if (st != FMOE_OK) return st;
   // the attribute is an upper bound shared by every layer using these kernels: set it
   // to the device maximum (a layer-sized value would break larger layers' launches)

@@ -178,7 +178,10 @@ fmoe_status fmoe_block_forward(fmoe_layer_t layer, const uint16_t* h, int T, dou
  * top-K per token plus the grouping, grouped gate/up + SwiGLU, grouped down, combine. */
 
 /* Bytes of the batched-path workspace for up to max_tokens (1..64) tokens per call (0
- * for an invalid config or max_tokens). */
+ * for an invalid config or max_tokens).  With the environment variable
+ * FMOE_GROUPED_TCGEN05 = "1" at the time of the call it includes the tcgen05 kernels'
+ * activation tiles (shapes they take only; see fmoe_layer_batched_kind); a workspace
+ * sized without them runs the mma.sync kernels. */
 size_t fmoe_batch_workspace_bytes(const fmoe_config* cfg, int max_tokens);
 
 /* Attaches a caller-owned device workspace for the batched entry points (separate from

@@ -160,3 +160,16 @@ def test_tier_buffer_bytes_and_host_checks(lib):
     # NULL host records, NULL buffer: rejected before any device call
     assert L.fmoe_tier_create(ctypes.byref(cfg), None, None, None, None, None, None, n8, 8, 1, ctypes.byref(h)) == 1
     assert L.fmoe_tier_destroy(None) == 0
+
+
+def test_batch_workspace_holds_tcgen05_tiles_only_on_request(lib, monkeypatch):
+    """The tcgen05 kernels' activation tiles are sized into the batch workspace only
+    when FMOE_GROUPED_TCGEN05=1 asks for them, and only for the shapes they take."""
+    full = lib.fmoe_config(4096, 1024, 512, 10, 4, 1, 1)
+    tiny = lib.fmoe_config(512, 128, 32, 4, 4, 1, 0)
+    plain_full, plain_tiny = lib.fmoe_batch_workspace_bytes(full, 32), lib.fmoe_batch_workspace_bytes(tiny, 32)
+    monkeypatch.setenv("FMOE_GROUPED_TCGEN05", "1")
+    with_full, with_tiny = lib.fmoe_batch_workspace_bytes(full, 32), lib.fmoe_batch_workspace_bytes(tiny, 32)
+    assert with_tiny == plain_tiny
+    # 16-pair blocks of x (2 B per column + a sum per 64) and of h (hi + lo + sums)
+    assert with_full - plain_full >= 22 * 16 * (2 * 4096 + 4096 // 16) + 22 * 16 * (4 * 1024 + 1024 // 16)
