@@ -479,6 +479,15 @@ constexpr int kGWarps = 16;  // warps of a grouped matvec block
 constexpr int kGThreads = kGWarps * 32;
 constexpr int kPieceCols = 1024;  // columns of one staged piece of a unit's 16 rows
 
+__device__ __forceinline__ unsigned long long f32x2(float lo, float hi) {
+  return (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -743,7 +752,8 @@ struct GroupedKernel {
 
   // ---- one piece: 16 rows x the piece's columns against the tile's pairs, folded
   // per group into acc (rows g and g+8 of the unit, pairs 2q and 2q+1)
-  __device__ __forceinline__ void piece(const uint8_t* sl, int u, int pc, float (&acc)[4]) const {
+  // acc: (row g, pairs 2q and 2q + 1) and (row g + 8, same pairs) as packed f32x2
+  __device__ __forceinline__ void piece(const uint8_t* sl, int u, int pc, unsigned long long (&acc)[2]) const {
     const int g = lane >> 2, q = lane & 3;
     const int c0 = pc * G.kc, cols = min(G.kc, G.ncol - c0);
     const uint8_t* ra = sl + g * G.code_stride;
@@ -801,18 +811,22 @@ struct GroupedKernel {
           }
         }
       }
-      const float2 X = *reinterpret_cast<const float2*>(xsum + ((c0 >> 6) + grp) * kTileTok + 2 * q);
+      const unsigned long long X2 =
+          *reinterpret_cast<const unsigned long long*>(xsum + ((c0 >> 6) + grp) * kTileTok + 2 * q);
       const uint32_t wsa = sa[grp], wsb = sb[grp];
       const float s16a = kScaleMul * sb_scale(wsa), s16b = kScaleMul * sb_scale(wsb);
       const float cba = sb_bias(wsa) - s16a, cbb = sb_bias(wsb) - s16b;
-      acc[0] = fmaf(s16a, d[0] + e[0], fmaf(cba, X.x, acc[0]));
-      acc[1] = fmaf(s16a, d[1] + e[1], fmaf(cba, X.y, acc[1]));
-      acc[2] = fmaf(s16b, d[2] + e[2], fmaf(cbb, X.x, acc[2]));
-      acc[3] = fmaf(s16b, d[3] + e[3], fmaf(cbb, X.y, acc[3]));
+      // acc = s16 (d + e) + (cb X + acc), two pairs per packed operation
+      fma2(acc[0], f32x2(cba, cba), X2);
+      fma2(acc[1], f32x2(cbb, cbb), X2);
+      fma2(acc[0], f32x2(s16a, s16a), add2(f32x2(d[0], d[1]), f32x2(e[0], e[1])));
+      fma2(acc[1], f32x2(s16b, s16b), add2(f32x2(d[2], d[3]), f32x2(e[2], e[3])));
     }
   }
 
-  __device__ __forceinline__ void epilogue(const GTile& tl, int u, const float (&acc)[4]) const {
+  __device__ __forceinline__ void epilogue(const GTile& tl, int u, const unsigned long long (&acc2)[2]) const {
+    const float acc[4] = {__uint_as_float(static_cast<uint32_t>(acc2[0])), __uint_as_float(static_cast<uint32_t>(acc2[0] >> 32)),
+                          __uint_as_float(static_cast<uint32_t>(acc2[1])), __uint_as_float(static_cast<uint32_t>(acc2[1] >> 32))};
     const int g = lane >> 2, q = lane & 3;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -859,7 +873,7 @@ struct GroupedKernel {
       __syncthreads();
       if (!ok) continue;
       for (int u = hdr->seg_ra[s] + warp; u < hdr->seg_rb[s] && ok; u += kGWarps) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        unsigned long long acc[2] = {0ull, 0ull};
         for (int pc = 0; pc < G.npiece; ++pc) {
           const int slot = static_cast<int>(k % kRing);
           const bool arrived = mbar_wait_bounded(&hdr->bars[warp][slot], (k / kRing) & 1u, p.wait_ns, p.err);
