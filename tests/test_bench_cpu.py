@@ -55,3 +55,12 @@ def test_profiled_traffic_only_for_the_captured_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic() == 123456
     first.write_text(first.read_text() + "\nnamespace fmoe { constexpr int kChanged = 1; }\n")
     assert bench.profiled_traffic() is None
+
+
+def test_committed_profiles_match_the_kernel_sources():
+    """The ncu summaries the bench line takes its DRAM traffic from were captured from
+    the kernel sources as they are (a kernel change needs a new capture)."""
+    import bench
+    assert bench.profiled_traffic() is not None
+    assert bench.profiled_traffic("traffic_warm_bytes_per_launch") is not None
+    assert bench.profiled_traffic(summary="gdn_step_kernel_gdn45.md", sources=("fmoe_gdn.cuh",)) is not None
