@@ -415,10 +415,10 @@ fmoe_status plan_batched(fmoe_layer* L, int T, bool want_umma) {
   const int G = L->sms;
   const int rows = c.n_experts + c.has_shared;
   // router: the block's router slices (fp32) plus kRouterTok token rows of the column
-  // splits it touches (fp64)
+  // splits it touches (fp32, exact for bf16)
   const int nq = router_splits(c.hidden), hc = c.hidden / nq;
   const size_t rsm = 128 + r128((uint32_t)(((long long)rows * nq + G - 1) / G) * hc * 4u) +
-                     (size_t)kRouterTok * router_splits_touched(rows, nq, G) * hc * 8;
+                     (size_t)kRouterTok * router_splits_touched(rows, nq, G) * hc * 4;
   uint32_t tsm = 0;
   topk_smem(c.n_experts, c.top_k, T, c.has_shared, &tsm);
   auto mv_smem = [&](bool down) {

@@ -35,7 +35,7 @@
 namespace fmoe {
 
 constexpr int kTileTok = 8;    // pairs of one expert whose activations are staged together (MMA N)
-constexpr int kRouterTok = 8;  // tokens per pass of the batched router
+constexpr int kRouterTok = 16;  // tokens per pass of the batched router
 constexpr int kMaxBatch = 64;  // tokens one batched call may have
 constexpr int kMaxSeg = 64;    // tiles one block's unit range may touch
 constexpr int kRing = 1;       // bulk copies in flight per warp (16 warps: latency is hidden across warps)
@@ -91,7 +91,8 @@ struct GParams {
 // Units are (row, column split q) in split-major order (u = q * rows + row; the shared
 // gate vector is row E), so a block's contiguous range of units touches at most a
 // couple of column splits.  Block b stages its units' router slices by bulk copies and,
-// kRouterTok tokens at a time, the activations of those splits as doubles (all loads
+// kRouterTok tokens at a time, the activations of those splits as floats (exact for
+// bf16; widened to fp64 where they are used; all loads
 // in flight); a warp per unit, every lane accumulating each token in the single-token
 // kernel's order, so the logits are bit-identical to that path.
 __host__ __device__ inline int router_splits_touched(int rows, int nq, int G) {
@@ -116,8 +117,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_router_kernel(const __gri
   const int nqs = nu > 0 ? (u1 - 1) / rows - q0 + 1 : 0;  // splits touched
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
   float* wr = reinterpret_cast<float*>(smem + 128);               // [nu][hc]
-  double* xd = reinterpret_cast<double*>(smem + 128 + r128(static_cast<uint32_t>(nu) * hc * 4u));
-  // xd: [kRouterTok][nqs * hc] doubles of the touched splits
+  float* xd = reinterpret_cast<float*>(smem + 128 + r128(static_cast<uint32_t>(nu) * hc * 4u));
+  // xd: [kRouterTok][nqs * hc] floats of the touched splits
   __shared__ int fail;
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
@@ -135,12 +136,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_router_kernel(const __gri
       bulk_g2s(wr + static_cast<size_t>(u - u0) * hc, src, static_cast<uint32_t>(hc) * 4u, bar);
     }
   }
-  const int xw = nqs * hc / 2;  // double2 per staged token row in each of the two arrays
-  const int n4 = nqs * hc / 4;
+  const int n4 = nqs * hc / 4;  // float2 per staged token row in each of the two arrays
   // xa[t][k] = (x[4k], x[4k+1]), xb[t][k] = (x[4k+2], x[4k+3]) of the touched splits:
-  // a warp's 16-byte loads of consecutive k are conflict-free
-  double2* xa = reinterpret_cast<double2*>(xd);
-  double2* xb = xa + static_cast<size_t>(kRouterTok) * (xw / 2);
+  // a warp's 8-byte loads of consecutive k are conflict-free
+  float2* xa = reinterpret_cast<float2*>(xd);
+  float2* xb = xa + static_cast<size_t>(kRouterTok) * n4;
   constexpr int KU = 8;
   for (int tg = 0; tg < p.T; tg += kRouterTok) {
     const int nt = min(kRouterTok, p.T - tg);
@@ -162,9 +162,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_router_kernel(const __gri
         if (i < nt * n4) {
           const int t = i / n4, c4 = i % n4;
           xa[static_cast<size_t>(t) * n4 + c4] =
-              make_double2(__uint_as_float(v[k].x << 16), __uint_as_float(v[k].x & 0xFFFF0000u));
+              make_float2(__uint_as_float(v[k].x << 16), __uint_as_float(v[k].x & 0xFFFF0000u));
           xb[static_cast<size_t>(t) * n4 + c4] =
-              make_double2(__uint_as_float(v[k].y << 16), __uint_as_float(v[k].y & 0xFFFF0000u));
+              make_float2(__uint_as_float(v[k].y << 16), __uint_as_float(v[k].y & 0xFFFF0000u));
         }
       }
     }
@@ -196,19 +196,25 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_router_kernel(const __gri
         for (int t = 0; t < kTT; ++t) {
           if (t0 + t < nt) {
             const size_t xt = static_cast<size_t>(t0 + t) * n4 + k;
-            const double2 xa0 = xa[xt + ka];
-            const double2 xb0 = xb[xt + ka];
-            a0[t] = fma(wa0, xa0.x, a0[t]);
-            a1[t] = fma(wa1, xa0.y, a1[t]);
-            a0[t] = fma(wa2, xb0.x, a0[t]);
-            a1[t] = fma(wa3, xb0.y, a1[t]);
+            const float2 fa0 = xa[xt + ka], fb0 = xb[xt + ka];
+            const double xa0x = fa0.x, xa0y = fa0.y, xb0x = fb0.x, xb0y = fb0.y;
+            a0[t] = fma(wa0, xa0x, a0[t]);
+            a1[t] = fma(wa1, xa0y, a1[t]);
+            a0[t] = fma(wa2, xb0x, a0[t]);
+            a1[t] = fma(wa3, xb0y, a1[t]);
             // the second unit usually shares the split (and so the loads)
-            const double2 xa1 = kb == ka ? xa0 : xa[xt + kb];
-            const double2 xb1 = kb == ka ? xb0 : xb[xt + kb];
-            b0[t] = fma(wb0, xa1.x, b0[t]);
-            b1[t] = fma(wb1, xa1.y, b1[t]);
-            b0[t] = fma(wb2, xb1.x, b0[t]);
-            b1[t] = fma(wb3, xb1.y, b1[t]);
+            double xa1x = xa0x, xa1y = xa0y, xb1x = xb0x, xb1y = xb0y;
+            if (kb != ka) {
+              const float2 fa1 = xa[xt + kb], fb1 = xb[xt + kb];
+              xa1x = fa1.x;
+              xa1y = fa1.y;
+              xb1x = fb1.x;
+              xb1y = fb1.y;
+            }
+            b0[t] = fma(wb0, xa1x, b0[t]);
+            b1[t] = fma(wb1, xa1y, b1[t]);
+            b0[t] = fma(wb2, xb1x, b0[t]);
+            b1[t] = fma(wb3, xb1y, b1[t]);
           }
         }
       }
