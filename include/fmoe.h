@@ -173,9 +173,15 @@ fmoe_status fmoe_block_forward(fmoe_layer_t layer, const uint16_t* h, int T, dou
  * another order: the T*K (token, slot) pairs are grouped by expert, so each active
  * expert's weights stream from HBM once for all of its tokens.  The pages decode one
  * token at a time; grouping several tokens' pairs by expert is this library's
- * addition for batched decode, kept to the same arithmetic per (token, expert).
+ * addition for batched decode.  Each (token, expert) output is the same quantity as
+ * on the single-token path; the grouped matvecs compute it on the tensor cores (codes
+ * entered as exact bf16 1 + c/2^b, exact products, fp32 sums folded with the scale
+ * and bias once per 64-column group).
  * Launch sequence per call: router (fp64, all tokens in one pass over the router),
- * top-K per token plus the grouping, grouped gate/up + SwiGLU, grouped down, combine. */
+ * top-K per token plus the grouping, grouped gate/up + SwiGLU, grouped down, combine
+ * (plus the small-tile kernels before each grouped phase, or a staging kernel before
+ * gate/up on the tcgen05 kernels, when those are selected; see
+ * fmoe_layer_batched_kind). */
 
 /* Bytes of the batched-path workspace for up to max_tokens (1..64) tokens per call (0
  * for an invalid config or max_tokens).  With the environment variable
