@@ -395,13 +395,14 @@ struct LayerKernel {
   // ---------------------------------------------------------------- dot products
   // Lane partial of sum_c W[r][c] v[c] over the lane's chunks, for one or two rows
   // sharing the activation loads (W = scale*code + bias; v pre-scaled, interleaved).
+  // The lane takes chunks m0, m0 + mstep, ... (by default its lane index, stride 32).
   template <bool TWO>
   __device__ __forceinline__ void dotn(const uint8_t* q0, const uint32_t* s0, const uint8_t* q1,
                                        const uint32_t* s1, const float* vs, const float2* vsum, int nch, float& r0,
-                                       float& r1) const {
+                                       float& r1, int m0 = -1, int mstep = 32) const {
     const int lane = threadIdx.x & 31;
 #pragma unroll 2
-    for (int m = lane; m < nch; m += 32) {
+    for (int m = m0 < 0 ? lane : m0; m < nch; m += mstep) {
       const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(q0 + 16 * m);
       ulonglong2 b = make_ulonglong2(0ull, 0ull);
       if (TWO) b = *reinterpret_cast<const ulonglong2*>(q1 + 16 * m);
@@ -605,6 +606,44 @@ struct LayerKernel {
     const uint32_t lead = static_cast<uint32_t>((p.o_d_sb + static_cast<unsigned long long>(ja) * p.si) & 15ull);
     const int nch = p.I / C::kCols;
     float pa = 0.f, pb = 0.f;
+    if constexpr (BITS == 2) {
+      if (nch <= 16) {
+        // a row of at most 16 chunks would leave half the lanes idle: each half-warp
+        // takes every other slot (lanes 0-15 the even slots, 16-31 the odd ones)
+        const int half = lane >> 4;
+        for (int s0 = 0; s0 < nslots; s0 += 2) {
+          const int s = s0 + half;
+          float oa = 0.f, ob = 0.f;
+          if (s < nslots) {
+            const uint8_t* blk = stage + off + s * g.dn_slot(n);
+            const uint32_t* sbase = reinterpret_cast<const uint32_t*>(blk + g.dn_q(n) + lead);
+            const float* hsl = hs + static_cast<size_t>(s) * g.padded(p.I);
+            const float2* hsm = hsum + static_cast<size_t>(s) * nch;
+            if (two)
+              dotn<true>(blk + static_cast<uint32_t>(ia) * p.qi, sbase + ia * (p.si / 4),
+                         blk + static_cast<uint32_t>(ib) * p.qi, sbase + ib * (p.si / 4), hsl, hsm, nch, oa, ob,
+                         lane & 15, 16);
+            else
+              dotn<false>(blk + static_cast<uint32_t>(ia) * p.qi, sbase + ia * (p.si / 4), nullptr, nullptr, hsl,
+                          hsm, nch, oa, ob, lane & 15, 16);
+            const float ws = hdr->wsl[s];
+            pa = fmaf(ws, oa, pa);
+            pb = fmaf(ws, ob, pb);
+          }
+        }
+        pa = warp_sum(pa);
+        pb = warp_sum(pb);
+        if (lane == 0) {
+          if (!NORM) {
+            ra = bf16_to_f32(resid_t[ja + ia]);
+            if (two) rb = bf16_to_f32(resid_t[ja + ib]);
+          }
+          y_t[ja + ia] = f32_to_bf16(ra + pa);
+          if (two) y_t[ja + ib] = f32_to_bf16(rb + pb);
+        }
+        return true;
+      }
+    }
     for (int s = 0; s < nslots; ++s) {
       const uint8_t* blk = stage + off + s * g.dn_slot(n);
       const uint32_t* sbase = reinterpret_cast<const uint32_t*>(blk + g.dn_q(n) + lead);
